@@ -1,0 +1,388 @@
+"""Benchmark of Loki sparse decode-step attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One timed step = one Loki decode layer-step (rotate q, low-rank scores, top-k,
+gather attention, combine) through the C ABI on a cache already resident in
+HBM.  Each step also appends the step's new token first (timed separately) and
+runs the in-library dense decode on the same cache (timed separately).  L2 is
+flushed before every step by writing a buffer twice the L2 size; the flush is
+outside the timed events.  Device time from CUDA events on the launching
+stream, summed over the K steps, max over ranks.
+
+With N GPUs (torchrun) each rank runs the whole workload on its own batch
+shard of an N-times larger global batch: weak scaling, no data-path
+collective.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from workloads import get_workload  # noqa: E402
+from workloads import generators as gen  # noqa: E402
+
+METRIC = "Loki decode attention µs/layer-step and achieved HBM GB/s vs peak, vs dense"
+UNIT = "us/layer-step"
+DEFAULT_WORKLOAD = "llama2-7b-decode"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha1()
+    d = os.path.join(ROOT, "sparse_decode_attention_loki_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t[kernel][workload]
+        if e.get("source_hash") == source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def workload_config(w, n_gpus):
+    return {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * n_gpus,
+            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "seq_len": w.seq_len, "d": w.d, "k": w.k, "d_f": w.d_f, "k_f": w.k_f,
+            "cache_dtype": w.dtype, "keys": f"{w.generator} spectrum (alpha {w.alpha})",
+            "l2": "flushed before every timed step (write of 2x L2, outside the timed events)",
+            "parallelism": f"weak: batch shard per GPU, {n_gpus} GPU(s), no collective"}
+
+
+# ------------------------------------------------------------------------------------ oracle arm
+def oracle_sample_us(w, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle decode on whole (batch, KV head) rows of the
+    workload, one row at a time, until budget_s of CPU time is spent; scale the
+    mean row time to one layer-step (all B*Hkv rows).  Returns (us per
+    layer-step, rows timed, threads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    P32 = np.stack([oracle.pca_basis(gen.calibration_keys(w, g))[0]
+                    for g in range(w.n_kv_heads)]).astype(np.float32).astype(np.float64)
+    rng = np.random.default_rng(seed)
+    G = w.group
+    times = []
+    t_start = time.perf_counter()
+    while True:
+        b, g = int(rng.integers(0, w.batch)), int(rng.integers(0, w.n_kv_heads))
+        _, k64 = gen.to_cache_dtype(gen.row_keys(w, b, g, w.seq_len), w.dtype)
+        _, v64 = gen.to_cache_dtype(gen.row_values(w, b, g, w.seq_len), w.dtype)
+        _, q64 = gen.to_cache_dtype(gen.queries(w, b)[g * G:(g + 1) * G][None], w.dtype)
+        K_hat = oracle.rotate_keys(k64[None, None], P32[g:g + 1], w.dtype)
+        t0 = time.perf_counter()
+        oracle.loki_decode(q64, K_hat, v64[None, None], P32[g:g + 1], w.seq_len, w.d, w.k)
+        times.append(time.perf_counter() - t0)
+        if sum(times) >= budget_s or time.perf_counter() - t_start > 3 * budget_s or len(times) >= 4096:
+            break
+    per_row = float(np.mean(times))
+    return per_row * w.rows * 1e6, len(times), threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = get_workload(args.workload)
+    budget = args.cpu_budget
+    for _ in range(args.warmup if args.warmup > 0 else 0):
+        oracle_sample_us(w, budget_s=0.0, seed=1)
+    per_step = []
+    rows = 0
+    threads = 1
+    for s in range(args.steps):
+        us, n, threads = oracle_sample_us(w, budget_s=budget / max(1, args.steps), seed=100 + s)
+        per_step.append(us)
+        rows += n
+    value = float(np.mean(per_step))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": value / 1000.0,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} whole (batch, KV head) rows of the workload, fp64 numpy oracle, "
+                                   f"scaled to all {w.rows} rows"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.proc = None
+        self.gpu_index = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_decode_attention_loki_b200 as L
+    from sparse_decode_attention_loki_b200.calibration import pca_bases
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = get_workload(args.workload)
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    S, B, Hkv, Hq, D = w.seq_len, w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
+    stream = torch.cuda.current_stream(dev)
+
+    # offline calibration (host) and cache prefill: S-1 tokens; each step appends token S-1
+    P = pca_bases([gen.calibration_keys(w, g) for g in range(Hkv)]).to(dev)
+    cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev)
+    g_dev = torch.Generator(device=dev)
+    g_dev.manual_seed(w.seed * 131 + rank)
+    if S > 1:
+        k_pre = torch.empty((B, Hkv, S - 1, D), dtype=td, device=dev)
+        for h in range(Hkv):
+            k_pre[:, h] = gen.device_keys(gen.make_key_model(w, h), B, S - 1, g_dev, dev, td)
+        v_pre = torch.randn((B, Hkv, S - 1, D), generator=g_dev, device=dev).to(td)
+        L.loki_append(cache, 0, k_pre, v_pre, P)
+        del k_pre, v_pre
+    NSET = 4
+    qs = [torch.randn((B, Hq, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
+    kn = [torch.randn((B, Hkv, 1, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
+    vn = [torch.randn((B, Hkv, 1, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
+    dout = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        j = i % NSET
+        flush.fill_(float(i & 7))
+        if ev is not None:
+            ev[0].record(stream)
+        L.loki_append(cache, S - 1, kn[j], vn[j], P)
+        if ev is not None:
+            ev[1].record(stream)
+        L.loki_decode_attention(cache, S, qs[j], P, w.d, w.k, out=out, idx=idx)
+        if ev is not None:
+            ev[2].record(stream)
+        L.dense_decode_attention(cache, S, qs[j], P, out=dout)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---------------- device-timed region
+    CH = 256
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(min(CH, args.steps))]
+    t_app = t_loki = t_dense = 0.0
+    per_step_loki = []
+    pr = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0")
+    time.sleep(0.3)  # let nvidia-smi take its first sample
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    done = 0
+    while done < args.steps:
+        n = min(CH, args.steps - done)
+        for i in range(n):
+            step(done + i, evs[i])
+        torch.cuda.synchronize()
+        for i in range(n):
+            e = evs[i]
+            a, b_, c = e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])
+            t_app += a
+            t_loki += b_
+            t_dense += c
+            per_step_loki.append(b_)
+        done += n
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+
+    # ---------------- end to end through host buffers (pinned), copies inside the events
+    q_host = [q.cpu().pin_memory() for q in qs]
+    out_host = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    idx_host = torch.empty((B, Hkv, w.k), dtype=torch.int32).pin_memory()
+    q_dev = torch.empty_like(qs[0])
+    e2e_steps = min(args.steps, 2000)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CH, e2e_steps))]
+    t_e2e = 0.0
+    for i in range(args.warmup):
+        q_dev.copy_(q_host[i % NSET], non_blocking=True)
+        L.loki_decode_attention(cache, S, q_dev, P, w.d, w.k, out=out, idx=idx)
+        out_host.copy_(out, non_blocking=True)
+        idx_host.copy_(idx, non_blocking=True)
+    torch.cuda.synchronize()
+    done = 0
+    while done < e2e_steps:
+        n = min(CH, e2e_steps - done)
+        for i in range(n):
+            flush.fill_(float(i & 7))
+            e2e_ev[i][0].record(stream)
+            q_dev.copy_(q_host[(done + i) % NSET], non_blocking=True)
+            L.loki_decode_attention(cache, S, q_dev, P, w.d, w.k, out=out, idx=idx)
+            out_host.copy_(out, non_blocking=True)
+            idx_host.copy_(idx, non_blocking=True)
+            e2e_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_e2e += e2e_ev[i][0].elapsed_time(e2e_ev[i][1])
+        done += n
+    h2d = q_host[0].numel() * q_host[0].element_size()
+    d2h = out_host.numel() * 4 + idx_host.numel() * 4
+
+    # ---------------- max over ranks
+    tt = torch.tensor([t_loki, t_dense, t_app, t_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    t_loki, t_dense, t_app, t_e2e = [float(x) for x in tt.tolist()]
+    cl, ct = L.loki_decode_launch_shape(cache, S, Hq)
+    dcl, dct = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
+
+    if rank == 0:
+        K = args.steps
+        loki_us = t_loki * 1000.0 / K
+        dense_us = t_dense * 1000.0 / K
+        app_us = t_app * 1000.0 / K
+        e2e_us = t_e2e * 1000.0 / e2e_steps
+        peak, peak_kind = peaks()
+        lb, db = w.loki_bytes(), w.dense_bytes()
+        ach = lb / (loki_us * 1e-6) / 1e9
+        dach = db / (dense_us * 1e-6) / 1e9
+        line = {
+            "metric": METRIC, "value": loki_us / world, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": loki_us / 1000.0, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(w, world),
+            "us_per_layer_step_per_gpu": loki_us,
+            "hbm_gbs": ach,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                         "traffic": measured_traffic("loki_decode_kernel", w.name),
+                         "kernel": "loki_decode_kernel", "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+                         "algorithmic_bytes_per_launch": lb},
+            "dense": {"us": dense_us, "hbm_gbs": dach, "frac": dach / peak, "bytes_per_launch": db,
+                      "launch": {"cluster_ctas": dcl, "ctas": dct}},
+            "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
+            "append_us": app_us,
+            "launch": {"cluster_ctas": cl, "ctas": ct, "threads_per_cta": 256},
+            "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": 3 * K,
+            "clocks": clocks,
+            "wall_s_timed_region": wall,
+            "per_step_loki_us": {"p50": float(np.percentile(per_step_loki, 50)) * 1000.0,
+                                 "p10": float(np.percentile(per_step_loki, 10)) * 1000.0,
+                                 "p90": float(np.percentile(per_step_loki, 90)) * 1000.0},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            cus, rows, threads = oracle_sample_us(w, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {"value": cus, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"{rows} whole (batch, KV head) rows, fp64 numpy oracle, "
+                                              f"scaled to all {w.rows} rows of one layer-step"}
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle CPU time")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps; the number is not a valid bench value", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+/*
+ * loki.h -- C ABI of libloki.so: Loki sparse decode-step attention on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("Loki: Low-rank Keys for Efficient Sparse Attention",
+ * atlas.scime.ai summary, sections "Approach" and the summary paragraph;
+ * mlsanity.com arXiv record 2406.02542, "Abstract"):  keys and queries are
+ * projected into a PCA basis P calibrated offline; every cached token is ranked
+ * by its attention score computed on the first d principal dimensions only; the
+ * k best tokens are kept and exact softmax attention is computed over them.
+ * No cache entry is ever deleted.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All pointers are DEVICE pointers of the current CUDA device unless stated,
+ *    owned by the caller.  The library never allocates, frees or synchronises;
+ *    it keeps no state between calls except per-device attribute caches.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream) and runs asynchronously.  A call returns after the
+ *    launch is enqueued; results are ready when the stream reaches that point.
+ *  - Tensors are dense, row-major (last index fastest), with no padding.
+ *  - dtype LOKI_F32 (fp32) or LOKI_BF16 (bfloat16) applies to the cache and to
+ *    q, k_new and v_new.  P is always fp32.  Outputs `out` are always fp32.
+ *  - Validation happens on the host before anything is launched.  On invalid
+ *    arguments the call returns LOKI_ERR_INVALID_ARG (or LOKI_ERR_UNSUPPORTED
+ *    for a valid but unimplemented shape) and enqueues nothing.  A failed launch
+ *    returns LOKI_ERR_CUDA.  loki_last_error() gives a one-line message for the
+ *    calling thread's last failure.  Kernels never trap or assert.
+ *  - Inputs must be finite (no NaN or Inf); this precondition is not checked.
+ *
+ * Sizes:  B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0, G = Hq / Hkv
+ * query heads share KV head g = h / G), D head dimension (64 or 128), S_cap
+ * cache capacity in tokens, seq_len tokens currently attended.
+ */
+#ifndef LOKI_H
+#define LOKI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LOKI_VERSION 1
+
+/* Symbols are exported from the shared object; everything else is hidden. */
+#if defined(LOKI_BUILD) && defined(__GNUC__)
+#define LOKI_API __attribute__((visibility("default")))
+#else
+#define LOKI_API
+#endif
+
+typedef enum {
+  LOKI_OK = 0,
+  LOKI_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or range           */
+  LOKI_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement     */
+  LOKI_ERR_CUDA = 3          /* the CUDA runtime refused a launch or attribute  */
+} loki_status;
+
+typedef enum { LOKI_F32 = 0, LOKI_BF16 = 1 } loki_dtype;
+
+/* A rotated-key KV cache in caller-owned device memory.
+ *   k_hat : [B, Hkv, S_cap, D] keys already rotated into the PCA basis
+ *           (k_hat = k . P_g), in `dtype`; 16-byte aligned.
+ *   v     : [B, Hkv, S_cap, D] values, unrotated, in `dtype`; 16-byte aligned.
+ * The cache holds every token ever appended: entries are never evicted, so its
+ * footprint equals a dense cache ("Limitations" section of the summary page). */
+typedef struct {
+  int32_t dtype;       /* loki_dtype                                          */
+  int32_t batch;       /* B >= 1                                              */
+  int32_t n_kv_heads;  /* Hkv >= 1                                            */
+  int32_t head_dim;    /* D: 64 or 128                                        */
+  int32_t capacity;    /* S_cap >= 1                                          */
+  void *k_hat;
+  void *v;
+} loki_cache;
+
+/* loki_append -- rotate new keys into the PCA basis and append them, with
+ * their values, at token positions [pos, pos + n_new) of every (batch, KV head)
+ * row.  Source: summary page, section "Approach" ("PCA-project ... keys") and
+ * "Surprising findings" (appending KV-cache entries is a large share of
+ * inference time).
+ *   k_new, v_new : [B, Hkv, n_new, D] in the cache dtype, 16-byte aligned.
+ *   P            : [Hkv, D, D] fp32; P[g][i][j] is component i of the j-th
+ *                  principal direction of KV head g (column j = direction j,
+ *                  sorted by descending eigenvalue).  16-byte aligned.
+ * Computes k_hat[b][g][pos+t][j] = round_to_dtype( sum_i k_new[b][g][t][i] *
+ * P[g][i][j] ) with fp32 accumulation and round-to-nearest-even, and copies
+ * v_new unchanged.  Entries outside [pos, pos + n_new) are not touched.
+ * Requires 0 <= pos, 1 <= n_new, pos + n_new <= S_cap. */
+LOKI_API loki_status loki_append(const loki_cache *cache, int32_t pos, int32_t n_new,
+                        const void *k_new, const void *v_new, const float *P,
+                        void *stream);
+
+/* loki_decode_attention -- one Loki decode step over tokens [0, seq_len).
+ * Source: summary page, summary paragraph and section "Approach"; arXiv
+ * record "Abstract".
+ *   q     : [B, Hq, D] queries in the cache dtype (NOT rotated), 16-byte aligned.
+ *   P     : [Hkv, D, D] fp32, the basis the cache keys were rotated with;
+ *           16-byte aligned.
+ *   d     : reduced dimension, 1 <= d <= D (the first d principal dims).
+ *   k     : key budget, 1 <= k <= seq_len.
+ *   scale : softmax scale of the exact attention; <= 0 selects 1/sqrt(D).
+ *   out   : [B, Hq, D] fp32 output (written).
+ *   idx   : [B, Hkv, k] int32 selected token indices (written), ascending.
+ * Per (b, g): q_hat_h = q_h . P_g (fp32, never rounded to the cache dtype);
+ * score_i = sum over the G query heads h of group g of q_hat_h[:d] . k_hat_i[:d];
+ * the k tokens with the largest scores are selected, ties going to the lower
+ * index; out_h = softmax(scale * q_hat_h . k_hat_i over the selected i, full D)
+ * weighted sum of v_i.  Requires seq_len <= S_cap, G in {1, 2, 4, 8}, and
+ * seq_len small enough for the per-row scores to stay on chip (about 8e5
+ * tokens); otherwise LOKI_ERR_UNSUPPORTED.  Needs no workspace. */
+LOKI_API loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len,
+                                  int32_t n_q_heads, const void *q, const float *P,
+                                  int32_t d, int32_t k, float scale, float *out,
+                                  int32_t *idx, void *stream);
+
+/* dense_decode_attention -- full softmax attention over every token
+ * [0, seq_len) of the same rotated cache: the "Full Attention" baseline of the
+ * summary page, section "Experimental setup".  Arguments as above; q is rotated
+ * by P so that q_hat . k_hat = q . k.  out: [B, Hq, D] fp32. */
+LOKI_API loki_status dense_decode_attention(const loki_cache *cache, int32_t seq_len,
+                                   int32_t n_q_heads, const void *q,
+                                   const float *P, float scale, float *out,
+                                   void *stream);
+
+/* Launch shape a decode call with these sizes would use, for logging and
+ * tests: *cluster_ctas CTAs per (batch, KV head) row in one thread-block
+ * cluster, *ctas the total grid.  `dense` selects the dense kernel.  Reads the
+ * current device's attributes; launches nothing.  Output pointers are host
+ * pointers. */
+LOKI_API loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len,
+                                     int32_t n_q_heads, int32_t dense,
+                                     int32_t *cluster_ctas, int32_t *ctas);
+
+/* Static description of a status code (never NULL). */
+LOKI_API const char *loki_status_string(loki_status s);
+
+/* Message of the calling thread's last failed call ("" if none). */
+LOKI_API const char *loki_last_error(void);
+
+/* LOKI_VERSION of the built library. */
+LOKI_API int32_t loki_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOKI_H */

@@ -103,7 +103,7 @@ def pca_basis(calib_keys) -> tuple:
     lead = np.argmax(np.abs(V), axis=0)
     signs = np.sign(V[lead, np.arange(D)])
     signs[signs == 0] = 1.0
-    return V * signs[None, :], w
+    return np.ascontiguousarray(V * signs[None, :]), w
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,34 @@
+"""Loki sparse decode-step attention for NVIDIA B200 (sm_100a).
+
+Keys and queries are rotated into an offline PCA basis, every cached token is
+scored on its first d principal dimensions, the k best tokens of each (batch,
+KV head) row are selected, and exact softmax attention runs over those rows
+("Loki: Low-rank Keys for Efficient Sparse Attention", atlas.scime.ai summary,
+section "Approach").  The work is done by hand-written CUDA kernels behind the
+C ABI of include/loki.h (libloki.so); this package is its Python binding.
+"""
+from ._lib import LIB_PATH, LokiError, load as load_library
+from .api import (
+    LokiCache,
+    dense_decode_attention,
+    loki_append,
+    loki_decode_attention,
+    loki_decode_launch_shape,
+    loki_status_string,
+    loki_version,
+)
+from .sharding import shard_batches
+
+__all__ = [
+    "LIB_PATH",
+    "LokiError",
+    "load_library",
+    "LokiCache",
+    "loki_append",
+    "loki_decode_attention",
+    "dense_decode_attention",
+    "loki_decode_launch_shape",
+    "loki_status_string",
+    "loki_version",
+    "shard_batches",
+]

@@ -1,0 +1,135 @@
+"""Python binding of the Loki decode-step library.
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, then their device pointers and the current CUDA stream are passed
+to libloki.so.  Every step of the computation runs in the library's CUDA
+kernels; PyTorch provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.float32: _lib.LOKI_F32, torch.bfloat16: _lib.LOKI_BF16}
+
+
+def _stream_ptr(device: torch.device, stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...], device: torch.device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class LokiCache:
+    """A rotated-key KV cache in device memory: k_hat and v of shape
+    [B, Hkv, capacity, D].  Keys are stored already rotated into the PCA basis;
+    nothing is ever evicted."""
+
+    def __init__(self, batch: int, n_kv_heads: int, head_dim: int, capacity: int,
+                 dtype: torch.dtype = torch.bfloat16, device=None,
+                 k_hat: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None):
+        if dtype not in _DTYPES:
+            raise ValueError(f"cache dtype must be float32 or bfloat16, got {dtype}")
+        device = torch.device(device if device is not None else "cuda")
+        if device.type != "cuda":
+            raise ValueError("the cache must live in CUDA device memory")
+        if device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        shape = (batch, n_kv_heads, capacity, head_dim)
+        self.k_hat = k_hat if k_hat is not None else torch.empty(shape, dtype=dtype, device=device)
+        self.v = v if v is not None else torch.empty(shape, dtype=dtype, device=device)
+        _need(self.k_hat, "k_hat", dtype, shape, device)
+        _need(self.v, "v", dtype, shape, device)
+        self.batch, self.n_kv_heads, self.head_dim, self.capacity = batch, n_kv_heads, head_dim, capacity
+        self.dtype = dtype
+        self.device = device
+        self._desc = _lib.loki_cache(_DTYPES[dtype], batch, n_kv_heads, head_dim, capacity,
+                                     self.k_hat.data_ptr(), self.v.data_ptr())
+
+    def desc(self) -> ctypes.POINTER(_lib.loki_cache):
+        return ctypes.byref(self._desc)
+
+
+def loki_append(cache: LokiCache, pos: int, k_new: torch.Tensor, v_new: torch.Tensor, P: torch.Tensor,
+                stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Rotate k_new [B, Hkv, n_new, D] by P [Hkv, D, D] (fp32) and append it with
+    v_new at positions [pos, pos + n_new)."""
+    n_new = k_new.shape[2] if k_new.dim() == 4 else -1
+    shp = (cache.batch, cache.n_kv_heads, n_new, cache.head_dim)
+    _need(k_new, "k_new", cache.dtype, shp, cache.device)
+    _need(v_new, "v_new", cache.dtype, shp, cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    _lib.check(_lib.load().loki_append(cache.desc(), int(pos), int(n_new), _ptr(k_new), _ptr(v_new), _ptr(P),
+                                       _stream_ptr(cache.device, stream)))
+
+
+def loki_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: torch.Tensor, d: int, k: int,
+                          scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                          idx: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One Loki decode step.  q: [B, Hq, D] in the cache dtype.  Returns
+    (out [B, Hq, D] fp32, idx [B, Hkv, k] int32 ascending)."""
+    B, Hq, D = q.shape if q.dim() == 3 else (-1, -1, -1)
+    _need(q, "q", cache.dtype, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    if out is None:
+        out = torch.empty((cache.batch, Hq, cache.head_dim), dtype=torch.float32, device=cache.device)
+    if idx is None:
+        idx = torch.empty((cache.batch, cache.n_kv_heads, int(k)), dtype=torch.int32, device=cache.device)
+    _need(out, "out", torch.float32, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(idx, "idx", torch.int32, (cache.batch, cache.n_kv_heads, int(k)), cache.device)
+    _lib.check(_lib.load().loki_decode_attention(cache.desc(), int(seq_len), int(Hq), _ptr(q), _ptr(P), int(d),
+                                                 int(k), float(scale), _ptr(out), _ptr(idx),
+                                                 _stream_ptr(cache.device, stream)))
+    return out, idx
+
+
+def dense_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: torch.Tensor, scale: float = 0.0,
+                           out: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Full attention over tokens [0, seq_len) of the same rotated cache."""
+    B, Hq, D = q.shape if q.dim() == 3 else (-1, -1, -1)
+    _need(q, "q", cache.dtype, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    if out is None:
+        out = torch.empty((cache.batch, Hq, cache.head_dim), dtype=torch.float32, device=cache.device)
+    _need(out, "out", torch.float32, (cache.batch, Hq, cache.head_dim), cache.device)
+    _lib.check(_lib.load().dense_decode_attention(cache.desc(), int(seq_len), int(Hq), _ptr(q), _ptr(P),
+                                                  float(scale), _ptr(out), _stream_ptr(cache.device, stream)))
+    return out
+
+
+def loki_decode_launch_shape(cache: LokiCache, seq_len: int, n_q_heads: int, dense: bool = False) -> Tuple[int, int]:
+    """(CTAs per (batch, KV head) row, total CTAs) of the decode launch."""
+    c, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    with torch.cuda.device(cache.device):
+        _lib.check(_lib.load().loki_decode_launch_shape(cache.desc(), int(seq_len), int(n_q_heads), int(bool(dense)),
+                                                        ctypes.byref(c), ctypes.byref(n)))
+    return c.value, n.value
+
+
+def loki_status_string(status: int) -> str:
+    return _lib.load().loki_status_string(int(status)).decode()
+
+
+def loki_version() -> int:
+    return int(_lib.load().loki_version())

@@ -1,0 +1,118 @@
+// Device helpers shared by the Loki kernels (sm_100a).
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace loki {
+
+namespace cg = cooperative_groups;
+
+constexpr int kThreads = 256;            // every kernel runs 8 warps per CTA
+constexpr int kWarps = kThreads / 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Elements per 16-byte vector.
+template <typename T> struct VecN;
+template <> struct VecN<float> { static constexpr int value = 4; };
+template <> struct VecN<__nv_bfloat16> { static constexpr int value = 8; };
+
+// 16-byte streaming load that does not allocate in L1 (cache rows are read
+// once per call).  Only used on data no thread writes during the kernel.
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+// Widen a 16-byte vector to fp32 (exact for both dtypes).
+__device__ __forceinline__ void unpack16(const uint4 &r, float (&f)[4]) {
+  f[0] = __uint_as_float(r.x);
+  f[1] = __uint_as_float(r.y);
+  f[2] = __uint_as_float(r.z);
+  f[3] = __uint_as_float(r.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 &r, float (&f)[8]) {
+  // bf16 is the upper half of an fp32; element 2i sits in the low 16 bits.
+  f[0] = __uint_as_float(r.x << 16);
+  f[1] = __uint_as_float(r.x & 0xffff0000u);
+  f[2] = __uint_as_float(r.y << 16);
+  f[3] = __uint_as_float(r.y & 0xffff0000u);
+  f[4] = __uint_as_float(r.z << 16);
+  f[5] = __uint_as_float(r.z & 0xffff0000u);
+  f[6] = __uint_as_float(r.w << 16);
+  f[7] = __uint_as_float(r.w & 0xffff0000u);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ void from_f32(float x, float *dst) { *dst = x; }
+__device__ __forceinline__ void from_f32(float x, __nv_bfloat16 *dst) {
+  *dst = __float2bfloat16_rn(x);  // round to nearest even
+}
+
+// Order-preserving map fp32 -> uint32: a > b  <=>  key(a) > key(b) for finite
+// a, b.  -0 and +0 map to the same key so that equal scores tie (and the lower
+// index wins) regardless of the sign of zero.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t b = __float_as_uint(s);
+  if ((b << 1) == 0u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Split cluster barrier (arrive with release, wait with acquire).  Every thread
+// of every CTA in the cluster must execute each of them the same number of times.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Sum of v over all threads with a larger threadIdx.x (exclusive suffix sum).
+// wtot: kWarps words of shared memory.  Contains two __syncthreads().
+__device__ __forceinline__ uint32_t block_excl_suffix_sum(uint32_t v, uint32_t *wtot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t s = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    uint32_t t = __shfl_down_sync(kFull, s, off);
+    if (lane + off < 32) s += t;
+  }
+  if (lane == 0) wtot[warp] = s;
+  __syncthreads();
+  uint32_t higher = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w > warp) higher += wtot[w];
+  __syncthreads();
+  return higher + (s - v);
+}
+
+// Sum over the CTA; the result is returned to every thread.
+// wtot: kWarps words of shared memory.  Contains two __syncthreads().
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t *wtot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  if (lane == 0) wtot[warp] = v;
+  __syncthreads();
+  uint32_t s = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) s += wtot[w];
+  __syncthreads();
+  return s;
+}
+
+}  // namespace loki

@@ -1,0 +1,109 @@
+"""The C-ABI library loads, exports every entry point include/loki.h declares,
+and rejects invalid arguments on the host before any CUDA call.  No test here
+launches a kernel: every call below fails host validation (or only reads device
+attributes), so the file is safe with or without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "loki.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return re.findall(r"LOKI_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_decode_attention_loki_b200 import _lib
+    return _lib.load()
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    assert set(names) == {"loki_append", "loki_decode_attention", "dense_decode_attention",
+                          "loki_decode_launch_shape", "loki_status_string", "loki_last_error", "loki_version"}
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from sparse_decode_attention_loki_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    # the binding declares a signature for each of them, and nothing else
+    assert set(_lib.SIGNATURES) == set(_declared())
+
+
+def test_library_is_built_for_sm100a():
+    from sparse_decode_attention_loki_b200 import build
+    cmd = " ".join(build.command())
+    assert "arch=compute_100a,code=sm_100a" in cmd
+
+
+def test_version_and_status_strings(lib):
+    assert lib.loki_version() == 1
+    for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
+        assert word in lib.loki_status_string(s)
+    assert lib.loki_status_string(99) == b"unknown loki_status"
+
+
+def _cache(dtype=1, B=1, H=2, D=128, cap=64, k=4096, v=8192):
+    from sparse_decode_attention_loki_b200 import _lib
+    return _lib.loki_cache(dtype, B, H, D, cap, k, v)
+
+
+FAKE = 1 << 20   # aligned non-null address; never dereferenced because validation fails first
+
+
+@pytest.mark.parametrize("cache_kw,seq,hq,d,k,status", [
+    (dict(dtype=7), 10, 2, 8, 4, 1),              # bad dtype
+    (dict(B=0), 10, 2, 8, 4, 1),                  # empty batch
+    (dict(D=96), 10, 2, 8, 4, 2),                 # unsupported head dim
+    (dict(k=0), 10, 2, 8, 4, 1),                  # null cache pointer
+    (dict(k=4100), 10, 2, 8, 4, 1),               # misaligned cache pointer
+    (dict(), 0, 2, 8, 4, 1),                      # empty sequence
+    (dict(), 65, 2, 8, 4, 1),                     # seq_len > capacity
+    (dict(), 10, 3, 8, 4, 1),                     # Hq not a multiple of Hkv
+    (dict(), 10, 6, 8, 4, 2),                     # group size 3 unsupported
+    (dict(), 10, 2, 0, 4, 1),                     # d = 0
+    (dict(), 10, 2, 129, 4, 1),                   # d > D
+    (dict(), 10, 2, 8, 0, 1),                     # k = 0
+    (dict(), 10, 2, 8, 11, 1),                    # k > seq_len
+])
+def test_decode_validation(lib, cache_kw, seq, hq, d, k, status):
+    c = _cache(**cache_kw)
+    r = lib.loki_decode_attention(ctypes.byref(c), seq, hq, FAKE, FAKE, d, k, 0.0, FAKE, FAKE, None)
+    assert r == status, lib.loki_last_error()
+    assert lib.loki_last_error() != b""
+
+
+def test_decode_null_pointers(lib):
+    c = _cache()
+    assert lib.loki_decode_attention(None, 10, 2, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE, None) == 1
+    for args in [(None, FAKE, FAKE, FAKE), (FAKE, None, FAKE, FAKE), (FAKE, FAKE, None, FAKE), (FAKE, FAKE, FAKE, None)]:
+        q, P, out, idx = args
+        assert lib.loki_decode_attention(ctypes.byref(c), 10, 2, q, P, 8, 4, 0.0, out, idx, None) == 1
+    assert lib.loki_decode_attention(ctypes.byref(c), 10, 2, FAKE + 8, FAKE, 8, 4, 0.0, FAKE, FAKE, None) == 1
+    assert lib.dense_decode_attention(ctypes.byref(c), 10, 2, None, FAKE, 0.0, FAKE, None) == 1
+    assert lib.dense_decode_attention(ctypes.byref(c), 0, 2, FAKE, FAKE, 0.0, FAKE, None) == 1
+
+
+@pytest.mark.parametrize("pos,n_new,status", [(-1, 1, 1), (0, 0, 1), (60, 5, 1), (64, 1, 1)])
+def test_append_validation(lib, pos, n_new, status):
+    c = _cache()
+    assert lib.loki_append(ctypes.byref(c), pos, n_new, FAKE, FAKE, FAKE, None) == status
+
+
+def test_append_pointer_validation(lib):
+    c = _cache()
+    assert lib.loki_append(ctypes.byref(c), 0, 1, None, FAKE, FAKE, None) == 1
+    assert lib.loki_append(ctypes.byref(c), 0, 1, FAKE, FAKE + 4, FAKE, None) == 1
+    assert lib.loki_append(ctypes.byref(c), 0, 1, FAKE, FAKE, None, None) == 1
+    assert lib.loki_append(None, 0, 1, FAKE, FAKE, FAKE, None) == 1

@@ -1,0 +1,328 @@
+"""Parity of the CUDA path (through the C ABI of libloki.so) with the fp64
+oracle, on seeded synthetic inputs.
+
+The cache contents the decode kernels read are the oracle's rotated keys
+(oracle.rotate_keys, rounded to the cache dtype) uploaded as they are, so that
+both sides score exactly the same K_hat; the GPU append kernel is checked on its
+own against the exact rotation.
+"""
+import contextlib
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from workloads import Workload, get_workload, mistral_sweep_points
+from workloads import generators as gen
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def L():
+    import sparse_decode_attention_loki_b200 as lib
+    return lib
+
+
+@contextlib.contextmanager
+def forced_cluster(n):
+    old = os.environ.get("LOKI_CLUSTER")
+    if n is None:
+        os.environ.pop("LOKI_CLUSTER", None)
+    else:
+        os.environ["LOKI_CLUSTER"] = str(n)
+    try:
+        yield
+    finally:
+        if old is None:
+            os.environ.pop("LOKI_CLUSTER", None)
+        else:
+            os.environ["LOKI_CLUSTER"] = old
+
+
+def small_workload(dtype, D, G, S, Hkv=2, B=2, generator="powerlaw", seed=77):
+    return Workload(name=f"small-{dtype}-D{D}-G{G}-S{S}", dtype=dtype, batch=B, n_q_heads=Hkv * G,
+                    n_kv_heads=Hkv, head_dim=D, seq_len=S, d_f=0.25, k_f=0.25, generator=generator,
+                    alpha=1.5, n_calib=max(4 * D, 512), seed=seed)
+
+
+def basis(w):
+    """P from the oracle's PCA of each head's calibration batch, as fp32."""
+    return np.ascontiguousarray(np.stack([oracle.pca_basis(gen.calibration_keys(w, g))[0]
+                                          for g in range(w.n_kv_heads)]), dtype=np.float32)
+
+
+def upload_case(w, inp, P32, capacity=None):
+    """Cache filled with the oracle's rotated keys; returns (cache, K_hat64, V64, q_dev, P_dev)."""
+    S = inp["seq_len"]
+    cap = capacity or S
+    K_hat = oracle.rotate_keys(inp["keys64"], P32.astype(np.float64), w.dtype)
+    td = TORCH_DTYPE[w.dtype]
+    cache = L().LokiCache(len(inp["batches"]), w.n_kv_heads, w.head_dim, cap, dtype=td, device=DEV)
+    cache.k_hat.zero_()
+    cache.v.zero_()
+    cache.k_hat[:, :, :S] = torch.from_numpy(K_hat).to(td).to(DEV)
+    cache.v[:, :, :S] = inp["values"].to(DEV)
+    return cache, K_hat, inp["values64"], inp["q"].to(DEV), torch.from_numpy(P32).to(DEV)
+
+
+def run_decode(w, S, d, k, ncta=None, scale=0.0, inp=None, P32=None, capacity=None):
+    inp = inp or gen.decode_inputs(w, seq_len=S)
+    P32 = basis(w) if P32 is None else P32
+    cache, K_hat, V, q, P = upload_case(w, inp, P32, capacity)
+    with forced_cluster(ncta):
+        out, idx = L().loki_decode_attention(cache, S, q, P, d, k, scale=scale)
+    torch.cuda.synchronize()
+    sc = None if scale <= 0 else scale
+    ref = oracle.loki_decode(inp["q64"], K_hat, V, P32.astype(np.float64), S, d, k, scale=sc)
+    return out.cpu().numpy(), idx.cpu().numpy(), ref, K_hat, V, inp, P32, cache, q, P
+
+
+# ----------------------------------------------------------------------------- append
+@pytest.mark.parametrize("dtype,D,n_new,pos,B,Hkv", [
+    ("bf16", 128, 1, 0, 2, 3),
+    ("bf16", 128, 37, 5, 3, 2),
+    ("bf16", 128, 300, 100, 2, 2),
+    ("bf16", 64, 9, 3, 1, 4),
+    ("f32", 64, 1, 7, 2, 2),
+    ("f32", 128, 41, 0, 2, 3),
+])
+def test_append_matches_exact_rotation(dtype, D, n_new, pos, B, Hkv):
+    w = small_workload(dtype, D, 1, n_new, Hkv=Hkv, B=B)
+    inp = gen.decode_inputs(w, seq_len=n_new)
+    P32 = basis(w)
+    cap = pos + n_new + 11
+    td = TORCH_DTYPE[dtype]
+    cache = L().LokiCache(B, Hkv, D, cap, dtype=td, device=DEV)
+    cache.k_hat.fill_(7.0)
+    cache.v.fill_(-3.0)
+    L().loki_append(cache, pos, inp["keys"].to(DEV), inp["values"].to(DEV), torch.from_numpy(P32).to(DEV))
+    torch.cuda.synchronize()
+    kh = cache.k_hat.to(torch.float64).cpu().numpy()
+    vv = cache.v.to(torch.float64).cpu().numpy()
+    st = parity.check_append(kh[:, :, pos:pos + n_new], inp["keys64"], P32.astype(np.float64), dtype)
+    if dtype == "bf16":
+        assert st["mismatch"] <= 0.05 * st["n"]   # sanity: most values round exactly like the oracle
+    np.testing.assert_array_equal(vv[:, :, pos:pos + n_new], inp["values64"])
+    # nothing outside [pos, pos + n_new) is touched
+    assert np.all(kh[:, :, :pos] == 7.0) and np.all(kh[:, :, pos + n_new:] == 7.0)
+    assert np.all(vv[:, :, :pos] == -3.0) and np.all(vv[:, :, pos + n_new:] == -3.0)
+
+
+def test_append_identity_basis_is_a_copy():
+    w = small_workload("bf16", 128, 1, 64)
+    inp = gen.decode_inputs(w, seq_len=64)
+    P = torch.eye(128, dtype=torch.float32).expand(2, 128, 128).contiguous().to(DEV)
+    cache = L().LokiCache(2, 2, 128, 64, dtype=torch.bfloat16, device=DEV)
+    L().loki_append(cache, 0, inp["keys"].to(DEV), inp["values"].to(DEV), P)
+    torch.cuda.synchronize()
+    assert torch.equal(cache.k_hat.cpu(), inp["keys"])
+
+
+# ----------------------------------------------------------------------------- decode, small shapes
+DECODE_CASES = [
+    # dtype, D, G, S, d, k
+    ("f32", 64, 1, 256, 16, 64),
+    ("bf16", 128, 1, 1000, 32, 250),
+    ("bf16", 128, 4, 3001, 64, 375),
+    ("bf16", 64, 2, 777, 8, 100),
+    ("f32", 128, 8, 513, 128, 512),
+    ("bf16", 128, 1, 300, 1, 1),
+    ("bf16", 128, 4, 2048, 16, 2047),
+    ("bf16", 128, 1, 1500, 32, 1500),
+    ("f32", 64, 4, 100, 3, 17),
+    ("bf16", 128, 8, 4097, 33, 1024),
+    ("f32", 128, 2, 1, 7, 1),
+]
+
+
+@pytest.mark.parametrize("ncta", [None, 1, 4, 16])
+@pytest.mark.parametrize("dtype,D,G,S,d,k", DECODE_CASES)
+def test_decode_matches_oracle(dtype, D, G, S, d, k, ncta):
+    w = small_workload(dtype, D, G, S)
+    out, idx, ref, K_hat, V, inp, P32, *_ = run_decode(w, S, d, k, ncta=ncta)
+    parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(D), dtype)
+
+
+def test_tiny_fp32_workload():
+    w = get_workload("tiny-fp32")
+    out, idx, ref, K_hat, V, *_ = run_decode(w, w.seq_len, w.d, w.k)
+    st = parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(w.head_dim), w.dtype)
+    assert st["swapped_rows"] == 0
+
+
+def test_decode_explicit_scale_and_capacity():
+    w = small_workload("bf16", 128, 4, 900)
+    out, idx, ref, K_hat, V, *_ = run_decode(w, 900, 32, 200, scale=0.3, capacity=1500)
+    parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, 0.3, "bf16")
+
+
+@pytest.mark.parametrize("ncta", [1, 8])
+def test_exact_ties_take_lowest_index(ncta):
+    # identity basis, small-integer keys and queries: every score is an exact
+    # integer on both sides, with many exact ties; the selection must match the
+    # oracle exactly (lower index wins)
+    rng = np.random.default_rng(5)
+    B, Hkv, G, D, S, d, k = 2, 2, 2, 128, 2000, 16, 333
+    keys = rng.integers(-2, 3, (B, Hkv, S, D)).astype(np.float64)
+    vals = rng.standard_normal((B, Hkv, S, D))
+    q = rng.integers(-1, 2, (B, Hkv * G, D)).astype(np.float64)
+    P = np.ascontiguousarray(np.broadcast_to(np.eye(D, dtype=np.float32), (Hkv, D, D)))
+    vt, v64 = gen.to_cache_dtype(vals, "bf16")
+    kt, k64 = gen.to_cache_dtype(keys, "bf16")
+    qt, q64 = gen.to_cache_dtype(q, "bf16")
+    inp = dict(keys64=k64, values=vt, values64=v64, q=qt, q64=q64, batches=list(range(B)), seq_len=S)
+    w = small_workload("bf16", D, G, S, Hkv=Hkv, B=B)
+    out, idx, ref, K_hat, V, *_ = run_decode(w, S, d, k, ncta=ncta, inp=inp, P32=P)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(D), "bf16")
+
+
+@pytest.mark.parametrize("ncta", [None, 16])
+def test_zero_query_selects_first_k(ncta):
+    w = small_workload("bf16", 128, 4, 1234)
+    inp = gen.decode_inputs(w, seq_len=1234)
+    inp["q"] = torch.zeros_like(inp["q"])
+    inp["q64"] = np.zeros_like(inp["q64"])
+    k = 77
+    out, idx, ref, K_hat, V, *_ = run_decode(w, 1234, 32, k, ncta=ncta, inp=inp)
+    assert np.all(idx == np.arange(k, dtype=np.int32))
+    for h in range(w.n_q_heads):
+        np.testing.assert_allclose(out[:, h], V[:, h // 4, :k].mean(axis=1), atol=5e-3)
+
+
+def test_full_budget_equals_dense():
+    w = small_workload("bf16", 128, 4, 700)
+    out, idx, ref, K_hat, V, inp, P32, cache, q, P = run_decode(w, 700, 128, 700)
+    dense = L().dense_decode_attention(cache, 700, q, P).cpu().numpy()
+    ref_dense = oracle.dense_decode(inp["q64"], K_hat, V, P32.astype(np.float64), 700)
+    parity.check_dense(dense, ref_dense, "bf16")
+    parity.check_dense(out, ref_dense, "bf16")
+    assert np.all(idx == np.arange(700))
+
+
+# ----------------------------------------------------------------------------- dense, small shapes
+@pytest.mark.parametrize("ncta", [None, 1, 16])
+@pytest.mark.parametrize("dtype,D,G,S", [
+    ("f32", 64, 1, 256), ("bf16", 128, 1, 4096), ("bf16", 128, 4, 3001), ("f32", 128, 8, 77),
+    ("bf16", 64, 2, 1), ("bf16", 128, 8, 1025),
+])
+def test_dense_matches_oracle(dtype, D, G, S, ncta):
+    w = small_workload(dtype, D, G, S)
+    inp = gen.decode_inputs(w, seq_len=S)
+    P32 = basis(w)
+    cache, K_hat, V, q, P = upload_case(w, inp, P32, capacity=S + 5)
+    with forced_cluster(ncta):
+        out = L().dense_decode_attention(cache, S, q, P)
+    torch.cuda.synchronize()
+    ref = oracle.dense_decode(inp["q64"], K_hat, V, P32.astype(np.float64), S)
+    parity.check_dense(out.cpu().numpy(), ref, dtype)
+
+
+# ----------------------------------------------------------------------------- errors
+def test_invalid_arguments_raise_without_launch():
+    lib = L()
+    cache = lib.LokiCache(1, 2, 128, 64, dtype=torch.bfloat16, device=DEV)
+    q = torch.zeros((1, 2, 128), dtype=torch.bfloat16, device=DEV)
+    P = torch.zeros((2, 128, 128), dtype=torch.float32, device=DEV)
+    for d, k, S in [(0, 1, 10), (129, 1, 10), (8, 0, 10), (8, 11, 10), (8, 1, 65), (8, 1, 0)]:
+        with pytest.raises(lib.LokiError) as e:
+            lib.loki_decode_attention(cache, S, q, P, d, k)
+        assert e.value.status == 1
+    q3 = torch.zeros((1, 6, 128), dtype=torch.bfloat16, device=DEV)   # G = 3
+    with pytest.raises(lib.LokiError) as e:
+        lib.loki_decode_attention(cache, 10, q3, P, 8, 4)
+    assert e.value.status == 2
+    with pytest.raises(lib.LokiError) as e:
+        lib.loki_append(cache, 60, torch.zeros((1, 2, 5, 128), dtype=torch.bfloat16, device=DEV),
+                        torch.zeros((1, 2, 5, 128), dtype=torch.bfloat16, device=DEV), P)
+    assert e.value.status == 1
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------------------------- full-size workloads
+def fill_cache_on_device(w, P_dev, S, capacity, seed=123):
+    """Whole cache through the GPU append kernel from device-drawn keys."""
+    td = TORCH_DTYPE[w.dtype]
+    cache = L().LokiCache(w.batch, w.n_kv_heads, w.head_dim, capacity, dtype=td, device=DEV)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    k_new = torch.empty((w.batch, w.n_kv_heads, S, w.head_dim), dtype=td, device=DEV)
+    for h in range(w.n_kv_heads):
+        k_new[:, h] = gen.device_keys(gen.make_key_model(w, h), w.batch, S, g, DEV, td)
+    v_new = torch.randn((w.batch, w.n_kv_heads, S, w.head_dim), generator=g, device=DEV).to(td)
+    L().loki_append(cache, 0, k_new, v_new, P_dev)
+    del k_new, v_new
+    return cache
+
+
+def full_size_check(w, S=None, n_rows=3, seed=0):
+    S = S or w.seq_len
+    k = w.k if S == w.seq_len else max(1, min(S, int(np.floor(w.k_f * S + 1e-9))))
+    d = w.d
+    P32 = basis(w)
+    P_dev = torch.from_numpy(P32).to(DEV)
+    cache = fill_cache_on_device(w, P_dev, S, S)
+    rng = np.random.default_rng(seed)
+    rows = sorted({(int(rng.integers(0, w.batch)), int(rng.integers(0, w.n_kv_heads))) for _ in range(n_rows)})
+    G = w.group
+    td = TORCH_DTYPE[w.dtype]
+    host = {}
+    for (b, g) in rows:
+        keys = gen.row_keys(w, b, g, S)
+        kt, k64 = gen.to_cache_dtype(keys, w.dtype)
+        vt, v64 = gen.to_cache_dtype(gen.row_values(w, b, g, S), w.dtype)
+        K_hat = oracle.rotate_keys(k64[None, None], P32[g:g + 1].astype(np.float64), w.dtype)
+        cache.k_hat[b, g, :S] = torch.from_numpy(K_hat[0, 0]).to(td).to(DEV)
+        cache.v[b, g, :S] = vt.to(DEV)
+        host[(b, g)] = (K_hat, v64[None, None])
+    Q = np.stack([gen.queries(w, b) for b in range(w.batch)])
+    qt, q64 = gen.to_cache_dtype(Q, w.dtype)
+    out, idx = L().loki_decode_attention(cache, S, qt.to(DEV), P_dev, d, k)
+    dense = L().dense_decode_attention(cache, S, qt.to(DEV), P_dev)
+    torch.cuda.synchronize()
+    out, idx, dense = out.cpu().numpy(), idx.cpu().numpy(), dense.cpu().numpy()
+    for (b, g), (K_hat, V) in host.items():
+        qs = q64[b:b + 1, g * G:(g + 1) * G]
+        Pg = P32[g:g + 1].astype(np.float64)
+        ref = oracle.loki_decode(qs, K_hat, V, Pg, S, d, k)
+        parity.check_decode(out[b:b + 1, g * G:(g + 1) * G], idx[b:b + 1, g:g + 1], ref, ref["q_hat"], K_hat, V,
+                            oracle.default_scale(w.head_dim), w.dtype)
+        rd = oracle.dense_decode(qs, K_hat, V, Pg, S)
+        parity.check_dense(dense[b:b + 1, g * G:(g + 1) * G], rd, w.dtype)
+    # every row's selection is structurally valid
+    assert idx.min() >= 0 and idx.max() < S
+    assert np.all(np.diff(idx, axis=-1) > 0)
+    del cache
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["llama2-7b-decode", "llama3-8b-gqa-decode"])
+def test_full_size_workload(name):
+    full_size_check(get_workload(name))
+
+
+@pytest.mark.parametrize("S", [3073, 3328, 3584])
+def test_llama2_13b_generation_lengths(S):
+    w = get_workload("llama2-13b-generation")
+    full_size_check(w, S=S, n_rows=2)
+
+
+SWEEP_SAMPLE = [
+    "mistral-7b-gqa-s4096-b1-d0.25-k0.25",
+    "mistral-7b-gqa-s16384-b8-d0.125-k0.5",
+    "mistral-7b-gqa-s65536-b1-d0.5-k0.125",
+    "mistral-7b-gqa-s131072-b1-d0.25-k0.25",
+    "mistral-7b-gqa-s131072-b8-d0.125-k0.125",
+]
+
+
+@pytest.mark.parametrize("name", SWEEP_SAMPLE)
+def test_mistral_sweep_points(name):
+    w = next(p for p in mistral_sweep_points() if p.name == name)
+    full_size_check(w, n_rows=2)

@@ -166,3 +166,27 @@ def decode_inputs(w: Workload, seq_len: Optional[int] = None,
     calib = [calibration_keys(w, g) for g in range(w.n_kv_heads)]
     return dict(keys=kt, values=vt, q=qt, keys64=k64, values64=v64, q64=q64,
                 calib=calib, batches=bs, seq_len=S)
+
+
+def device_keys(model: KeyModel, batch: int, n: int, gen, device, dtype) -> "torch.Tensor":
+    """Keys of one KV head for a whole batch drawn on the GPU: the same
+    distribution as draw_keys with torch's generator `gen` (so not the same
+    numbers).  Returns [batch, n, D] in the torch dtype `dtype`.  Used to fill
+    large caches quickly; rows checked against the oracle are overwritten with
+    host draws."""
+    import torch
+    D = model.D
+    if model.kind == "rank8":
+        A = torch.as_tensor(model.A, dtype=torch.float32, device=device)
+        Z = torch.randn((batch, n, 8), generator=gen, device=device)
+        N = torch.randn((batch, n, D), generator=gen, device=device)
+        return (Z @ A + 0.05 * N).to(dtype)
+    U = torch.as_tensor(model.U, dtype=torch.float32, device=device)
+    sl = torch.as_tensor(np.sqrt(model.lam), dtype=torch.float32, device=device)
+    mu = torch.as_tensor(model.mu, dtype=torch.float32, device=device)
+    out = torch.empty((batch, n, D), dtype=dtype, device=device)
+    step = max(1, (1 << 24) // max(1, n * D))   # bound the fp32 temporaries
+    for b0 in range(0, batch, step):
+        Z = torch.randn((min(step, batch - b0), n, D), generator=gen, device=device)
+        out[b0:b0 + Z.shape[0]] = (mu + (Z * sl) @ U.T).to(dtype)
+    return out

@@ -6,9 +6,11 @@
 //
 // k_hat[b][g][pos+t][j] = round( sum_i k_new[b][g][t][i] * P[g][i][j] ), fp32
 // accumulation in increasing i, round to nearest even into the cache dtype;
-// v_new is copied unchanged.  Grid (Hkv, chunks): a CTA holds P_g in shared
-// memory (64 KB for D = 128) and rotates a chunk of the B*n_new vectors of
-// KV head g, 8 at a time.
+// v_new is copied unchanged.  Grid (Hkv, D/32, chunks): a CTA holds a 32-column
+// slice of P_g in shared memory (16 KB for D = 128) and produces those 32
+// output columns for a chunk of the B*n_new vectors of KV head g, 8 vectors at
+// a time (one vector per warp, one column per lane).  CTAs of column block 0
+// also copy the values.
 #pragma once
 
 #include "common.cuh"
@@ -30,30 +32,37 @@ struct AppendArgs {
   int32_t per_cta;   // vectors per CTA (multiple of kAppendBatch)
 };
 
-constexpr int kAppendBatch = 8;
+constexpr int kAppendBatch = kWarps;   // vectors per batch: one per warp
+constexpr int kAppendCols = 32;        // output columns per CTA: one per lane
 
-__host__ __device__ inline int append_smem_words(int D) { return D * D + kAppendBatch * D; }
+__host__ __device__ inline int append_smem_words(int D) { return D * kAppendCols + kAppendBatch * D; }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendArgs<T> a) {
   extern __shared__ __align__(16) float asmem[];
-  float *Ps = asmem;               // [D][D]
-  float *ks = asmem + D * D;       // [kAppendBatch][D]
-  const int g = blockIdx.x;
-  const int tid = threadIdx.x;
-  const int f_begin = blockIdx.y * a.per_cta;
+  float *Ps = asmem;                   // [D][32]: columns cb*32 .. cb*32+31 of P_g
+  float *ks = asmem + D * kAppendCols; // [8][D]
+  const int g = blockIdx.x, cb = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int f_begin = blockIdx.z * a.per_cta;
   const int f_end = min(a.n_vec, f_begin + a.per_cta);
   if (f_begin >= f_end) return;  // uniform over the CTA; no barrier has been reached
 
   {
-    const float4 *src = reinterpret_cast<const float4 *>(a.P + (size_t)g * D * D);
-    float4 *dst = reinterpret_cast<float4 *>(Ps);
-    for (int i = tid; i < D * D / 4; i += kThreads) dst[i] = __ldg(src + i);
+    // P_g[i][cb*32 .. +32): 8 float4 per row, all issued before any is stored
+    constexpr int N4 = D * kAppendCols / 4;
+    const float *src = a.P + (size_t)g * D * D + cb * kAppendCols;
+    float4 r[N4 / kThreads];
+#pragma unroll
+    for (int x = 0; x < N4 / kThreads; ++x) {
+      const int q = x * kThreads + tid;
+      r[x] = __ldg(reinterpret_cast<const float4 *>(src + (size_t)(q / 8) * D) + (q % 8));
+    }
+#pragma unroll
+    for (int x = 0; x < N4 / kThreads; ++x) reinterpret_cast<float4 *>(Ps)[x * kThreads + tid] = r[x];
   }
 
-  constexpr int GROUPS = kThreads / D;                 // 2 (D=128) or 4 (D=64)
-  constexpr int VPT = kAppendBatch / GROUPS;           // vectors per thread per batch
-  const int j = tid % D, grp = tid / D;
+  const int j = cb * kAppendCols + lane;
   for (int f0 = f_begin; f0 < f_end; f0 += kAppendBatch) {
     __syncthreads();  // P staged / previous batch consumed
     for (int e = tid; e < kAppendBatch * D; e += kThreads) {
@@ -66,25 +75,18 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
       ks[e] = x;
     }
     __syncthreads();
-    float acc[VPT];
-#pragma unroll
-    for (int x = 0; x < VPT; ++x) acc[x] = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < D; ++i) {
-      const float p = Ps[i * D + j];
-#pragma unroll
-      for (int x = 0; x < VPT; ++x) acc[x] = fmaf(ks[(grp + x * GROUPS) * D + i], p, acc[x]);
-    }
-#pragma unroll
-    for (int x = 0; x < VPT; ++x) {
-      const int f = f0 + grp + x * GROUPS;
-      if (f < f_end) {
-        const int b = f / a.n_new, t = f % a.n_new;
-        from_f32(acc[x], a.k_hat + (((size_t)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * D + j);
-      }
+    const float *kv = ks + warp * D;
+    float acc = 0.f;
+#pragma unroll 16
+    for (int i = 0; i < D; ++i) acc = fmaf(kv[i], Ps[i * kAppendCols + lane], acc);
+    const int f = f0 + warp;
+    if (f < f_end) {
+      const int b = f / a.n_new, t = f % a.n_new;
+      from_f32(acc, a.k_hat + (((size_t)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * D + j);
     }
   }
 
+  if (cb != 0) return;
   // values: straight 16-byte copies
   constexpr int VEC = VecN<T>::value;
   constexpr int VPR = D / VEC;  // vectors per row

@@ -29,6 +29,25 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p) {
   return r;
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), completed by
+// cp.async.wait_group.  Both addresses must be 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem_src) : "memory");
+}
+// Same, but copies `valid ? 16 : 0` bytes and zero-fills the rest (the source
+// is not read when invalid; it must still be a mapped address).
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem_src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Widen a 16-byte vector to fp32 (exact for both dtypes).
 __device__ __forceinline__ void unpack16(const uint4 &r, float (&f)[4]) {
   f[0] = __uint_as_float(r.x);
@@ -55,6 +74,46 @@ __device__ __forceinline__ void from_f32(float x, float *dst) { *dst = x; }
 __device__ __forceinline__ void from_f32(float x, __nv_bfloat16 *dst) {
   *dst = __float2bfloat16_rn(x);  // round to nearest even
 }
+
+// ---- warp-level tensor-core helpers (bf16 operands, fp32 accumulation) ----
+// Four 8x8 b16 matrices from shared memory; lane l supplies the address of row
+// l%8 of matrix l/8.  Thread (g = lane/4, t = lane%4) receives row g, columns
+// 2t and 2t+1 of each matrix (.trans: row 2t and 2t+1, column g).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                              uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D[16x8] += A[16x16] . B[16x8]
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// D[16x8] += A[16x8] . B[8x8]
+__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+// (x0, x1) as two bf16 pairs hi + lo with x ~= hi + lo to about 2^-17 relative:
+// hi = RNE(x), lo = RNE(x - hi); element 0 in the low half of each word.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 // Order-preserving map fp32 -> uint32: a > b  <=>  key(a) > key(b) for finite
 // a, b.  -0 and +0 map to the same key so that equal scores tie (and the lower

@@ -7,26 +7,34 @@
 // Attention" baseline (same page, "Experimental setup").
 //
 // B200 design.  One thread-block cluster of `ncta` CTAs owns one (batch, KV
-// head) row.  CTA r of the cluster owns the contiguous token range
-// [r*chunk, (r+1)*chunk).  The whole decode step is one kernel:
-//   1. every CTA rotates the G queries of its KV group (q . P, fp32) and forms
-//      the group's low-rank query u = sum_h q_hat_h[:d];
-//   2. it streams K_hat[i, :d] of its range with 16-byte loads, one score per
-//      token, and keeps the scores as order-preserving uint32 keys in shared
-//      memory -- scores never go to HBM;
-//   3. the cluster finds the k-th largest key by an 11/11/10-bit radix select:
-//      each CTA histograms its keys and adds the histogram into the leader
-//      CTA's shared memory through distributed shared memory (DSMEM);
+// head) row; CTA r owns the contiguous token range [r*chunk, (r+1)*chunk).
+// The whole decode step is one kernel:
+//   1. the first stages of the low-rank key stream are put in flight
+//      (cp.async into a shared-memory ring), then every CTA rotates the G
+//      queries of its KV group (q . P, fp32) and forms the group's low-rank
+//      query u = sum_h q_hat_h[:d] while those loads land;
+//   2. the CTA streams K_hat[i, :d] of its range through the ring and keeps one
+//      order-preserving uint32 key per token in shared memory -- scores never
+//      go to HBM;
+//   3. the cluster finds the k-th largest key by a radix select over 8-bit
+//      digits (at most 4 passes, usually 2-3): each CTA histograms its keys and
+//      stores the 256 counts into its slot in EVERY CTA of the cluster through
+//      distributed shared memory (16-byte DSMEM stores, double-buffered), so
+//      that after one cluster barrier every CTA derives the same digit, the
+//      per-CTA counts, and finally its own share of the ties and its offset;
 //   4. each CTA writes its selected token indices, ascending, at its offset in
 //      idx (ties at the threshold go to the lower index);
 //   5. the k selected tokens are split evenly over the cluster; each CTA
-//      gathers full K_hat and V rows and keeps an online softmax per query
-//      head (log2 domain, fp32);
+//      gathers full K_hat and V rows through the ring and keeps an online
+//      softmax per query head (log2 domain, fp32);
 //   6. the CTAs' partial (max, sum, acc) states are merged through DSMEM with
-//      the log-sum-exp rule and the leader-free combine writes out.
-// No workspace, no atomics in global memory, no spin-waits: every cross-CTA
-// step is a hardware cluster barrier.
+//      the log-sum-exp rule, and the output is written.
+// No workspace, no atomics in global memory, no software spin-waits: every
+// cross-CTA step is a hardware cluster barrier and every async copy is waited
+// for with cp.async.wait_group.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -46,73 +54,97 @@ struct DecodeArgs {
   int32_t d;
   int32_t k;
   int32_t chunk;       // tokens per CTA
-  int32_t lpt;         // lanes per token in the score loop (power of two)
-  int32_t dpad;        // d rounded up to a whole 16-byte vector
+  int32_t lpt;         // 16-byte chunks per token in the score stream (power of two)
+  int32_t nck;         // chunks that hold the first d dims: ceil(d / elements per chunk)
   float scale_log2;    // softmax scale * log2(e)
 };
 
-// Shared-memory layout, in 4-byte words.  Identical on host and device.
+// ---------------------------------------------------------------------------
+// shared memory
+// Every warp streams through its own slice of the ring: kStages stages of
+// kWarpStageBytes, kStages-1 of them in flight while it computes on one.
+// Warps synchronise only with __syncwarp() inside the streams.
+constexpr int kStages = 4;
+constexpr int kWarpStageBytes = 2048;
+constexpr int kWarpRingBytes = kStages * kWarpStageBytes;
+constexpr int kRingWords = kWarps * kWarpRingBytes / 4;
+constexpr int kBins = 256;                 // 8-bit radix digits; one bin per thread
+static_assert(kThreads == kBins, "the select maps one histogram bin to each thread");
+
+__host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
+
+// rotation scratch: q staging + partial dot products
+__host__ __device__ inline int rot_words(int G, int D) { return G * D + (kThreads / D) * G * D; }
+
 struct SmemLayout {
-  int qhat, u, pm, pl, pacc, ctl, scratch, keys, words;
+  int qhat, u, pm, pl, pacc, ctl, lhist, slots, ring, keys, words;
 };
 
-__host__ __device__ inline int scratch_words(int G, int D) {
-  int a = 4 * 2048;                          // local histogram + 3 cluster histograms
-  int b = G * D + (kThreads / D) * G * D;    // query staging + partial dot products
-  int c = kWarps * G * (D + 2);              // per-warp softmax states
-  int m = a > b ? a : b;
-  return m > c ? m : c;
-}
-
-__host__ __device__ inline SmemLayout decode_layout(int G, int D, int chunk, bool with_keys) {
+// Layout in 4-byte words, identical on host and device.  `slots` also serves
+// as the rotation scratch (before the CTA arrives on the first cluster
+// barrier no other CTA writes it) and, once the select is over, as the bf16
+// query tiles of the tensor-core attention; the ring also holds the per-warp
+// softmax states after the attention loop.
+__host__ __device__ inline SmemLayout decode_layout(int G, int D, int chunk, int ncta, bool loki) {
   SmemLayout L;
   int o = 0;
-  L.qhat = o;    o += G * D;
-  L.u = o;       o += D;
-  L.pm = o;      o += 16;
-  L.pl = o;      o += 16;
-  L.pacc = o;    o += G * D;
-  L.ctl = o;     o += 128;
-  L.scratch = o; o += scratch_words(G, D);
-  L.keys = o;    o += with_keys ? chunk : 0;
-  L.words = (o + 3) & ~3;
+  L.qhat = o;  o += G * D;
+  L.u = o;     o += round4(D);
+  L.pm = o;    o += 16;
+  L.pl = o;    o += 16;
+  L.pacc = o;  o += G * D;
+  L.ctl = o;   o += 128;
+  L.lhist = o; o += loki ? kBins : 0;
+  L.slots = o;
+  {
+    const int s = loki ? 2 * ncta * kBins : 0;
+    const int r = rot_words(G, D);
+    const int q = 8 * D;  // bf16 query tiles of the tensor-core attention: 2 x 8 rows x D
+    const int m = s > r ? s : r;
+    o += round4(m > q ? m : q);
+  }
+  L.ring = o;  o += kRingWords;
+  L.keys = o;  o += loki ? round4(chunk) : 0;
+  L.words = o;
   return L;
 }
 
-// ctl word offsets
-constexpr int kCtlBucket = 0;    // [0..2]: bucket, count above it, count in it
-constexpr int kCtlWtot = 4;      // [4..11]: warp totals for block scans
-constexpr int kCtlMine = 12;     // [12..13]: this CTA's (#above, #in bucket)
-constexpr int kCtlGt = 16;       // [16..31]: #above per CTA of the cluster
-constexpr int kCtlEq = 32;       // [32..47]: #in bucket per CTA of the cluster
-constexpr int kCtlWarpGt = 48;   // [48..55]
-constexpr int kCtlWarpEq = 56;   // [56..63]
+// ctl word offsets (per CTA)
+constexpr int kCtlWtot = 0;       // [0..7]: warp totals for block scans
+constexpr int kCtlBucket = 8;     // [8..10]: bucket, count above it, count in it
+constexpr int kCtlGtAcc = 16;     // [16..31]: per-CTA count strictly above the prefix
+constexpr int kCtlIn = 32;        // [32..47]: per-CTA count in the bucket
+constexpr int kCtlWarpGt = 48;    // [48..55]
+constexpr int kCtlWarpEq = 56;    // [56..63]
+static_assert(kWarps == 8, "ctl layout assumes 8 warps");
 
 // ---------------------------------------------------------------------------
 // 1. query rotation: q_hat_h = q_h . P_g for the G heads of KV head g, and
 //    u = sum_h q_hat_h[:d] (zero beyond d).  q_hat is then pre-scaled by
-//    scale*log2(e) for the log2-domain softmax.  Ends with __syncthreads().
-template <typename T, int D, int G>
+//    scale*log2(e) for the log2-domain softmax.  The loads of P are issued
+//    first; `after_loads()` runs while they are in flight (the caller puts its
+//    first stream stages in flight there).  Ends with __syncthreads().
+template <typename T, int D, int G, typename F>
 __device__ __forceinline__ void rotate_queries(const DecodeArgs<T> &a, int b, int g,
                                                float *qhat, float *u, float *scratch,
-                                               bool want_u) {
+                                               bool want_u, F &&after_loads) {
   const int tid = threadIdx.x;
   const int Hq = a.n_kv_heads * G;
   const T *qg = a.q + ((size_t)b * Hq + (size_t)g * G) * D;
-  float *qs = scratch;  // [G][D]
-  for (int i = tid; i < G * D; i += kThreads) qs[i] = to_f32(qg[i]);
-  __syncthreads();
-
   constexpr int PARTS = kThreads / D;
   constexpr int IPP = D / PARTS;
   const int j = tid % D, part = tid / D;
   const float *Pg = a.P + (size_t)g * D * D + (size_t)part * IPP * D + j;
-  float acc[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) acc[h] = 0.f;
   float pv[IPP];
 #pragma unroll
   for (int ii = 0; ii < IPP; ++ii) pv[ii] = __ldg(Pg + (size_t)ii * D);
+  float *qs = scratch;  // [G][D]
+  for (int i = tid; i < G * D; i += kThreads) qs[i] = to_f32(qg[i]);
+  after_loads();
+  __syncthreads();
+  float acc[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) acc[h] = 0.f;
 #pragma unroll
   for (int ii = 0; ii < IPP; ++ii) {
 #pragma unroll
@@ -145,183 +177,208 @@ __device__ __forceinline__ void rotate_queries(const DecodeArgs<T> &a, int b, in
 }
 
 // ---------------------------------------------------------------------------
-// 2. low-rank scores of tokens [t0, t0+len): key = score_key(u . K_hat[i, :d]).
-//    LPT lanes cooperate on one token (16 bytes each); a warp load instruction
-//    covers 32/LPT consecutive tokens.
+// 2. low-rank score stream.  The CTA's tokens are cut into blocks of
+//    TS = kWarpStageBytes/(16*LPT) tokens; warp w streams blocks w, w+8, ...
+//    through its own ring slice.  Token t of a block keeps its LPT 16-byte
+//    chunks at byte (t*LPT + c)*16 of the stage; chunks c >= nck (beyond the
+//    first d dims) are neither copied nor used.  Each score becomes an
+//    order-preserving key in keys[], and the histogram of the keys' top byte
+//    (the first radix digit) is accumulated in lhist on the way.
 template <typename T, int D, int LPT>
-__device__ __forceinline__ void score_tokens(const T *__restrict__ Krow, int t0, int len,
-                                             int dpad, const float *u, uint32_t *keys) {
-  constexpr int VEC = VecN<T>::value;
-  constexpr int TPW = 32 / LPT;
-  constexpr int TPB = TPW * kWarps;
-  constexpr int UNR = (LPT >= 8) ? 4 : 8;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane % LPT;
-  const int slot = warp * TPW + lane / LPT;
-  const bool active = sub * VEC < dpad;
-  float uv[VEC];
+struct ScoreStream {
+  static constexpr int VEC = VecN<T>::value;
+  static constexpr int TS = kWarpStageBytes / (16 * LPT);
+  static constexpr int TPW = 32 / LPT;  // tokens per warp instruction
+
+  __device__ __forceinline__ static void issue(const T *Krow, int t0, int len, int nck, int s,
+                                               unsigned char *wring) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
+    const int base = (s * kWarps + warp) * TS;
 #pragma unroll
-  for (int x = 0; x < VEC; ++x) uv[x] = u[sub * VEC + x];
-  const T *base = Krow + (size_t)t0 * D + sub * VEC;
-  for (int s0 = 0; s0 < len; s0 += TPB * UNR) {
-    uint4 r[UNR];
-#pragma unroll
-    for (int x = 0; x < UNR; ++x) {
-      const int j = s0 + x * TPB + slot;
-      r[x] = (active && j < len) ? ld_stream16(base + (size_t)j * D) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int x = 0; x < UNR; ++x) {
-      float f[VEC];
-      unpack16(r[x], f);
-      float s = 0.f;
-#pragma unroll
-      for (int y = 0; y < VEC; ++y) s = fmaf(uv[y], f[y], s);
-#pragma unroll
-      for (int off = LPT / 2; off > 0; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
-      const int j = s0 + x * TPB + slot;
-      if (sub == 0 && j < len) keys[j] = score_key(s);
+    for (int it = 0; it < TS * LPT / 32; ++it) {
+      const int q = it * 32 + lane;
+      const int t = q / LPT, c = q % LPT;
+      if (base + t < len && c < nck) cp_async16(st + q * 16, Krow + (size_t)(t0 + base + t) * D + c * VEC);
     }
   }
-}
 
-template <typename T, int D>
-__device__ __forceinline__ void score_dispatch(int lpt, const T *Krow, int t0, int len, int dpad,
-                                               const float *u, uint32_t *keys) {
-  constexpr int MAXL = D / VecN<T>::value;
-  switch (lpt) {
-    case 1: score_tokens<T, D, 1>(Krow, t0, len, dpad, u, keys); break;
-    case 2: score_tokens<T, D, 2>(Krow, t0, len, dpad, u, keys); break;
-    case 4: score_tokens<T, D, 4>(Krow, t0, len, dpad, u, keys); break;
-    case 8: score_tokens<T, D, 8>(Krow, t0, len, dpad, u, keys); break;
-    case 16:
-      if constexpr (MAXL >= 16) score_tokens<T, D, 16>(Krow, t0, len, dpad, u, keys);
-      break;
-    default:
-      if constexpr (MAXL >= 32) score_tokens<T, D, 32>(Krow, t0, len, dpad, u, keys);
-      break;
+  __device__ __forceinline__ static void consume(int len, int nck, int s, const unsigned char *wring,
+                                                 const float (&uv)[VEC], uint32_t *keys, uint32_t *lhist) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
+    const int c = lane % LPT;
+    const int base = (s * kWarps + warp) * TS;
+#pragma unroll
+    for (int step = 0; step < TS / TPW; ++step) {
+      const int t = step * TPW + lane / LPT;
+      float sc = 0.f;
+      if (c < nck) {
+        const uint4 r = *reinterpret_cast<const uint4 *>(st + (t * LPT + c) * 16);
+        float f[VEC];
+        unpack16(r, f);
+#pragma unroll
+        for (int y = 0; y < VEC; ++y) sc = fmaf(uv[y], f[y], sc);
+      }
+#pragma unroll
+      for (int off = LPT / 2; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
+      const bool mine = c == 0 && base + t < len;
+      uint32_t bin = 0xffffffffu;
+      if (mine) {
+        const uint32_t key = score_key(sc);
+        keys[base + t] = key;
+        bin = key >> 24;
+      }
+      const uint32_t peers = __match_any_sync(kFull, bin);
+      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&lhist[bin], (uint32_t)__popc(peers));
+    }
   }
-}
 
-// ---------------------------------------------------------------------------
-// 3. cluster radix select.  Finds (prefix, mask, remaining) such that the
-//    selected set is {key: key&mask > prefix} plus the first `remaining` (by
-//    token index) of {key: key&mask == prefix}.  merged: the three cluster
-//    histograms (local address; the leader's copy is the one used), zeroed by
-//    the leader before its cluster_arrive().  Pass 0 performs the matching
-//    cluster_wait().
-struct SelectState {
-  uint32_t prefix, mask, remaining;
+  __device__ __forceinline__ static int warp_stages(int len) {
+    const int warp = threadIdx.x >> 5;
+    const int blocks = (len + TS - 1) / TS;
+    return blocks > warp ? (blocks - warp + kWarps - 1) / kWarps : 0;
+  }
 };
 
-__device__ __forceinline__ SelectState radix_select(cg::cluster_group &cluster, const uint32_t *keys,
-                                                    int len, uint32_t k, uint32_t *hist,
-                                                    uint32_t *merged, uint32_t *ctl) {
-  const int tid = threadIdx.x, lane = tid & 31;
+// Prologue: put the first kStages-1 stages of this warp in flight.
+template <typename T, int D, int LPT>
+__device__ __forceinline__ void score_prologue(const T *Krow, int t0, int len, int nck, unsigned char *ring) {
+  using SS = ScoreStream<T, D, LPT>;
+  unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    SS::issue(Krow, t0, len, nck, s, wring);
+    cp_async_commit();
+  }
+}
+
+template <typename T, int D, int LPT>
+__device__ __forceinline__ void score_loop(const T *Krow, int t0, int len, int nck, unsigned char *ring,
+                                           const float *u, uint32_t *keys, uint32_t *lhist) {
+  using SS = ScoreStream<T, D, LPT>;
+  constexpr int VEC = VecN<T>::value;
+  unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+  const int c = (threadIdx.x & 31) % LPT;
+  float uv[VEC];
+#pragma unroll
+  for (int y = 0; y < VEC; ++y) uv[y] = u[(c * VEC + y) % D];
+  const int ns = SS::warp_stages(len);
+  for (int s = 0; s < ns; ++s) {
+    cp_async_wait<kStages - 2>();
+    __syncwarp();
+    SS::issue(Krow, t0, len, nck, s + kStages - 1, wring);
+    cp_async_commit();
+    SS::consume(len, nck, s, wring, uv, keys, lhist);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
+#define LOKI_LPT_DISPATCH(lpt, MAXL, CALL)                 \
+  switch (lpt) {                                           \
+    case 1: { constexpr int L_ = 1; CALL; } break;         \
+    case 2: { constexpr int L_ = 2; CALL; } break;         \
+    case 4: { constexpr int L_ = 4; CALL; } break;         \
+    case 8: { constexpr int L_ = 8; CALL; } break;         \
+    case 16:                                               \
+      if constexpr (MAXL >= 16) { constexpr int L_ = 16; CALL; } \
+      break;                                               \
+    default:                                               \
+      if constexpr (MAXL >= 32) { constexpr int L_ = 32; CALL; } \
+      break;                                               \
+  }
+
+// ---------------------------------------------------------------------------
+// 3. cluster radix select over 8-bit digits, most significant first.  Every
+//    CTA keeps the same (prefix, mask, remaining) and per-CTA counts; after it,
+//    this CTA's selected set is {key: key&mask > prefix} plus its first `take`
+//    keys (in token order) with key&mask == prefix, written from position
+//    `offset` of the row.  slots: [2][ncta][256] words; pass p stores this
+//    CTA's histogram into slot [p&1][rank] of every CTA.  On entry lhist holds
+//    the histogram of the keys' top byte (pass 0).  The caller zeroes
+//    ctl[kCtlGtAcc..kCtlIn+15] and performs cluster_arrive() before; pass 0
+//    performs the matching cluster_wait().
+struct SelectState {
+  uint32_t prefix, mask, take, offset;
+};
+
+__device__ __forceinline__ SelectState radix_select(cg::cluster_group &cluster, int ncta, int rank,
+                                                    const uint32_t *keys, int len, uint32_t k,
+                                                    uint32_t *lhist, uint32_t *slots, uint32_t *ctl) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0u, mask = 0u, remaining = k;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const int nbits = pass == 2 ? 10 : 11;
-    const uint32_t nb = 1u << nbits;
-    for (uint32_t i = tid; i < nb; i += kThreads) hist[i] = 0u;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    // the pass-0 histogram was accumulated by the score stream
+    if (pass > 0) lhist[tid] = 0u;
     __syncthreads();
     // warp-aggregated shared atomics: lanes with the same bin add once
-    for (int j0 = 0; j0 < len; j0 += kThreads) {
+    for (int j0 = 0; pass > 0 && j0 < len; j0 += kThreads) {
       const int j = j0 + tid;
       uint32_t bin = 0xffffffffu;
       if (j < len) {
         const uint32_t key = keys[j];
-        if ((key & mask) == prefix) bin = (key >> shift) & (nb - 1u);
+        if ((key & mask) == prefix) bin = (key >> shift) & (kBins - 1u);
       }
       const uint32_t peers = __match_any_sync(kFull, bin);
-      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&lhist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (pass == 0) cluster_wait();  // leader histograms zeroed; all CTAs running
-    uint32_t *dst = cluster.map_shared_rank(merged + pass * 2048, 0);
-    for (uint32_t i = tid; i < nb; i += kThreads) {
-      const uint32_t c = hist[i];
-      if (c) atomicAdd(dst + i, c);
+    if (pass == 0) cluster_wait();  // every CTA of the cluster is running
+    uint32_t *buf = slots + (pass & 1) * ncta * kBins;
+    for (int q = tid; q < ncta * (kBins / 4); q += kThreads) {
+      const int dst = q / (kBins / 4), part = q % (kBins / 4);
+      uint4 *p = reinterpret_cast<uint4 *>(cluster.map_shared_rank(buf + rank * kBins, dst));
+      p[part] = reinterpret_cast<const uint4 *>(lhist)[part];
     }
     cluster.sync();
-    // every CTA scans the merged histogram from the top bin down
-    const int bpt = (int)(nb / kThreads);  // 8 or 4
-    uint32_t c[8];
-    uint32_t sum = 0u;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      c[x] = (x < bpt) ? dst[tid * bpt + x] : 0u;
-      sum += c[x];
-    }
-    const uint32_t above = block_excl_suffix_sum(sum, ctl + kCtlWtot);
-    if (above < remaining && above + sum >= remaining) {
-      uint32_t cum = above;
-      bool found = false;
-#pragma unroll
-      for (int x = 7; x >= 0; --x) {
-        if (!found && x < bpt) {
-          if (cum + c[x] >= remaining) {
-            ctl[kCtlBucket + 0] = (uint32_t)(tid * bpt + x);
-            ctl[kCtlBucket + 1] = cum;
-            ctl[kCtlBucket + 2] = c[x];
-            found = true;
-          } else {
-            cum += c[x];
-          }
-        }
-      }
+    uint32_t tot = 0u;
+    for (int r = 0; r < ncta; ++r) tot += buf[r * kBins + tid];
+    const uint32_t above = block_excl_suffix_sum(tot, ctl + kCtlWtot);  // bins > tid
+    if (above < remaining && above + tot >= remaining) {
+      ctl[kCtlBucket + 0] = (uint32_t)tid;
+      ctl[kCtlBucket + 1] = above;
+      ctl[kCtlBucket + 2] = tot;
     }
     __syncthreads();
     const uint32_t bucket = ctl[kCtlBucket + 0];
     const uint32_t cnt_above = ctl[kCtlBucket + 1];
     const uint32_t cnt_in = ctl[kCtlBucket + 2];
-    __syncthreads();
+    for (int r = warp; r < ncta; r += kWarps) {
+      uint32_t gt = 0u;
+      for (int x = lane; x < kBins; x += 32)
+        if ((uint32_t)x > bucket) gt += buf[r * kBins + x];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) gt += __shfl_xor_sync(kFull, gt, off);
+      if (lane == 0) {
+        ctl[kCtlGtAcc + r] += gt;
+        ctl[kCtlIn + r] = buf[r * kBins + bucket];
+      }
+    }
     remaining -= cnt_above;
     prefix |= bucket << shift;
-    mask |= (nb - 1u) << shift;
-    if (cnt_in == remaining) break;  // the whole bucket is taken: done
+    mask |= (kBins - 1u) << shift;
+    __syncthreads();
+    if (cnt_in == remaining) break;  // the whole bucket is taken
   }
-  return SelectState{prefix, mask, remaining};
-}
-
-// ---------------------------------------------------------------------------
-// 4. write this CTA's selected indices, ascending, at its offset in the row of
-//    idx.  Ends with a cluster barrier after which the whole row of idx is
-//    written and visible to every CTA of the cluster.
-__device__ __forceinline__ void write_selection(cg::cluster_group &cluster, int ncta, int rank,
-                                                const uint32_t *keys, int len, int t0,
-                                                const SelectState &st, uint32_t k, uint32_t *ctl,
-                                                int32_t *idx_row) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t my_gt = 0u, my_eq = 0u;
-  for (int j = tid; j < len; j += kThreads) {
-    const uint32_t km = keys[j] & st.mask;
-    my_gt += km > st.prefix;
-    my_eq += km == st.prefix;
-  }
-  my_gt = block_sum(my_gt, ctl + kCtlWtot);
-  my_eq = block_sum(my_eq, ctl + kCtlWtot);
-  if (tid == 0) {
-    ctl[kCtlMine + 0] = my_gt;
-    ctl[kCtlMine + 1] = my_eq;
-  }
-  cluster.sync();
-  if (tid < ncta) {
-    const uint32_t *rc = cluster.map_shared_rank(ctl + kCtlMine, tid);
-    ctl[kCtlGt + tid] = rc[0];
-    ctl[kCtlEq + tid] = rc[1];
-  }
-  __syncthreads();
   // ties at the threshold are taken in token order: lower CTAs first
   uint32_t eq_before = 0u, offset = 0u;
   for (int r = 0; r < rank; ++r) {
-    const uint32_t want = st.remaining > eq_before ? st.remaining - eq_before : 0u;
-    offset += ctl[kCtlGt + r] + min(ctl[kCtlEq + r], want);
-    eq_before += ctl[kCtlEq + r];
+    const uint32_t want = remaining > eq_before ? remaining - eq_before : 0u;
+    offset += ctl[kCtlGtAcc + r] + min(ctl[kCtlIn + r], want);
+    eq_before += ctl[kCtlIn + r];
   }
-  const uint32_t take = min(ctl[kCtlEq + rank], st.remaining > eq_before ? st.remaining - eq_before : 0u);
+  const uint32_t take = min(ctl[kCtlIn + rank], remaining > eq_before ? remaining - eq_before : 0u);
+  return SelectState{prefix, mask, take, offset};
+}
 
-  // each warp owns a contiguous segment of the CTA's tokens
+// ---------------------------------------------------------------------------
+// 4. write this CTA's selected indices, ascending, from position st.offset of
+//    the row of idx.  Each warp owns a contiguous segment of the CTA's tokens.
+__device__ __forceinline__ void write_selection(const uint32_t *keys, int len, int t0, const SelectState &st,
+                                                uint32_t k, uint32_t *ctl, int32_t *idx_row) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int seg = (((len + kWarps - 1) / kWarps) + 31) & ~31;
   const int sbeg = min(len, warp * seg), send = min(len, sbeg + seg);
   uint32_t wg = 0u, we = 0u;
@@ -339,11 +396,11 @@ __device__ __forceinline__ void write_selection(cg::cluster_group &cluster, int 
   __syncthreads();
   uint32_t eq_base = 0u, sel_base = 0u;
   for (int w = 0; w < warp; ++w) {
-    const uint32_t want = take > eq_base ? take - eq_base : 0u;
+    const uint32_t want = st.take > eq_base ? st.take - eq_base : 0u;
     sel_base += ctl[kCtlWarpGt + w] + min(ctl[kCtlWarpEq + w], want);
     eq_base += ctl[kCtlWarpEq + w];
   }
-  int32_t *dst = idx_row + offset;
+  int32_t *dst = idx_row + st.offset;
   uint32_t run_eq = eq_base, run_sel = sel_base;
   const uint32_t lt = lanemask_lt();
   for (int j0 = sbeg; j0 < send; j0 += 32) {
@@ -354,34 +411,79 @@ __device__ __forceinline__ void write_selection(cg::cluster_group &cluster, int 
     const bool eq = in && km == st.prefix;
     const uint32_t eb = __ballot_sync(kFull, eq);
     const uint32_t eq_rank = run_eq + __popc(eb & lt);
-    const bool sel = gt || (eq && eq_rank < take);
+    const bool sel = gt || (eq && eq_rank < st.take);
     const uint32_t sb = __ballot_sync(kFull, sel);
     const uint32_t p = run_sel + __popc(sb & lt);
-    if (sel && offset + p < k) dst[p] = t0 + j;  // bound: the row holds k entries
+    if (sel && st.offset + p < k) dst[p] = t0 + j;  // bound: the row holds k entries
     run_eq += __popc(eb);
     run_sel += __popc(sb);
   }
-  cluster.sync();
 }
 
 // ---------------------------------------------------------------------------
-// 5. exact attention over `cnt` rows (gathered through ids[], or the
-//    contiguous rows tok0 .. tok0+cnt-1).  D/VEC lanes share one row; each
-//    lane keeps an online softmax (max, sum, acc over its VEC dims) per query
-//    head.  Leaves the CTA's merged state in pm/pl/pacc (not normalised).
+// 5. exact attention over `cnt` rows -- gathered through ids[] (shared memory,
+//    already clamped into the row) or the contiguous rows tok0 .. tok0+cnt-1.
+//    Rows are cut into blocks of TA = kWarpStageBytes/(2*row bytes); warp w
+//    streams blocks w, w+8, ... through its ring slice, each row as its K row
+//    followed by its V row.  D/VEC lanes share a row; each lane keeps an online
+//    softmax (max, sum, acc over its VEC dims) per query head.  Leaves the
+//    CTA's merged state in pm/pl/pacc (not normalised).
+template <typename T, int D, bool GATHER>
+struct RowStream {
+  static constexpr int VEC = VecN<T>::value;
+  static constexpr int RB = D * (int)sizeof(T);  // bytes per row
+  static constexpr int CPR = RB / 16;            // chunks per row
+  static constexpr int TA = kWarpStageBytes / (2 * RB);
+
+  __device__ __forceinline__ static void issue(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+                                               int s, unsigned char *wring) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
+    const int base = (s * kWarps + warp) * TA;
+#pragma unroll
+    for (int it = 0; it < TA * 2 * CPR / 32; ++it) {
+      const int q = it * 32 + lane;
+      const int t = q / (2 * CPR), c = q % (2 * CPR);
+      const int i = base + t;
+      if (i < cnt) {
+        const int tok = GATHER ? ids[i] : tok0 + i;
+        const T *src = (c < CPR ? Kb : Vb) + (size_t)tok * D + (c % CPR) * VEC;
+        cp_async16(st + q * 16, src);
+      }
+    }
+  }
+
+  __device__ __forceinline__ static int warp_stages(int cnt) {
+    const int warp = threadIdx.x >> 5;
+    const int blocks = (cnt + TA - 1) / TA;
+    return blocks > warp ? (blocks - warp + kWarps - 1) / kWarps : 0;
+  }
+};
+
+template <typename T, int D, bool GATHER>
+__device__ __forceinline__ void attend_prologue(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+                                                unsigned char *ring) {
+  unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    RowStream<T, D, GATHER>::issue(Kb, Vb, ids, tok0, cnt, s, wring);
+    cp_async_commit();
+  }
+}
+
 template <typename T, int D, int G, bool GATHER>
-__device__ __forceinline__ void attend_rows(const T *__restrict__ Kb, const T *__restrict__ Vb,
-                                            const int32_t *ids, int tok0, int cnt, int seq_len,
-                                            const float *qhat, float *wpart, float *pm,
-                                            float *pl, float *pacc) {
-  constexpr int VEC = VecN<T>::value;
+__device__ __forceinline__ void attend_loop(const T *__restrict__ Kb, const T *__restrict__ Vb,
+                                            const int32_t *ids, int tok0, int cnt, const float *qhat,
+                                            unsigned char *ring, float *pm, float *pl, float *pacc) {
+  using RS = RowStream<T, D, GATHER>;
+  constexpr int VEC = RS::VEC;
   constexpr int LPR = D / VEC;
-  constexpr int RG = 32 / LPR;
-  constexpr int U = (G >= 8) ? 2 : 4;
-  constexpr int STRIDE = kWarps * RG;
+  constexpr int RG = 32 / LPR;                  // rows per warp instruction
+  constexpr int U = RS::TA / RG;                // rows per lane group per stage
+  static_assert(RS::TA % RG == 0, "a stage must be a whole number of warp steps");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sub = lane % LPR, grp = lane / LPR;
-  const int slot = warp * RG + grp;
+  unsigned char *wring = ring + warp * kWarpRingBytes;
 
   float qv[G][VEC];
 #pragma unroll
@@ -397,43 +499,31 @@ __device__ __forceinline__ void attend_rows(const T *__restrict__ Kb, const T *_
     for (int x = 0; x < VEC; ++x) acc[h][x] = 0.f;
   }
 
-  for (int base = 0; base < cnt; base += STRIDE * U) {
-    int tok[U];
+  const int ns = RS::warp_stages(cnt);
+  for (int s = 0; s < ns; ++s) {
+    cp_async_wait<kStages - 2>();
+    __syncwarp();
+    RS::issue(Kb, Vb, ids, tok0, cnt, s + kStages - 1, wring);
+    cp_async_commit();
+    const unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
+    const int base = (s * kWarps + warp) * RS::TA;
+    float lg[U][G];
     bool ok[U];
 #pragma unroll
     for (int x = 0; x < U; ++x) {
-      const int i = base + x * STRIDE + slot;
-      ok[x] = i < cnt;
-      if constexpr (GATHER) {
-        // indices come from this kernel's own selection; clamp them into the
-        // row so that no load can leave the cache even if they were wrong
-        tok[x] = ok[x] ? min(max(__ldcg(ids + i), 0), seq_len - 1) : 0;
-      } else {
-        tok[x] = tok0 + i;
-      }
-    }
-    uint4 kr[U], vr[U];
-#pragma unroll
-    for (int x = 0; x < U; ++x) {
-      if (ok[x]) {
-        kr[x] = ld_stream16(Kb + (size_t)tok[x] * D + sub * VEC);
-        vr[x] = ld_stream16(Vb + (size_t)tok[x] * D + sub * VEC);
-      } else {
-        kr[x] = make_uint4(0u, 0u, 0u, 0u);
-        vr[x] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    float lg[U][G];
-#pragma unroll
-    for (int x = 0; x < U; ++x) {
+      const int t = x * RG + grp;
+      ok[x] = base + t < cnt;
+      // rows past cnt were never copied: read zeros instead of stale memory
+      const uint4 kr = ok[x] ? *reinterpret_cast<const uint4 *>(st + t * 2 * RS::RB + sub * 16)
+                             : make_uint4(0u, 0u, 0u, 0u);
       float f[VEC];
-      unpack16(kr[x], f);
+      unpack16(kr, f);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float s = 0.f;
+        float a = 0.f;
 #pragma unroll
-        for (int y = 0; y < VEC; ++y) s = fmaf(qv[h][y], f[y], s);
-        lg[x][h] = s;
+        for (int y = 0; y < VEC; ++y) a = fmaf(qv[h][y], f[y], a);
+        lg[x][h] = a;
       }
     }
 #pragma unroll
@@ -442,9 +532,7 @@ __device__ __forceinline__ void attend_rows(const T *__restrict__ Kb, const T *_
       for (int x = 0; x < U; ++x)
 #pragma unroll
         for (int h = 0; h < G; ++h) lg[x][h] += __shfl_xor_sync(kFull, lg[x][h], off);
-    float vf[U][VEC];
-#pragma unroll
-    for (int x = 0; x < U; ++x) unpack16(vr[x], vf[x]);
+    float p[U][G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float mx = m[h];
@@ -458,14 +546,25 @@ __device__ __forceinline__ void attend_rows(const T *__restrict__ Kb, const T *_
       for (int y = 0; y < VEC; ++y) acc[h][y] *= corr;
 #pragma unroll
       for (int x = 0; x < U; ++x) {
-        const float p = ok[x] ? exp2f(lg[x][h] - mref) : 0.f;
-        l[h] += p;
-#pragma unroll
-        for (int y = 0; y < VEC; ++y) acc[h][y] = fmaf(p, vf[x][y], acc[h][y]);
+        p[x][h] = ok[x] ? exp2f(lg[x][h] - mref) : 0.f;
+        l[h] += p[x][h];
       }
       m[h] = mx;
     }
+#pragma unroll
+    for (int x = 0; x < U; ++x) {
+      const int t = x * RG + grp;
+      const uint4 vr = ok[x] ? *reinterpret_cast<const uint4 *>(st + t * 2 * RS::RB + RS::RB + sub * 16)
+                             : make_uint4(0u, 0u, 0u, 0u);
+      float f[VEC];
+      unpack16(vr, f);
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int y = 0; y < VEC; ++y) acc[h][y] = fmaf(p[x][h], f[y], acc[h][y]);
+    }
   }
+  cp_async_wait<0>();
 
   // merge the row groups of the warp (lanes that share `sub`)
 #pragma unroll
@@ -486,6 +585,8 @@ __device__ __forceinline__ void attend_rows(const T *__restrict__ Kb, const T *_
       m[h] = mx;
     }
   }
+  __syncthreads();  // every warp is done with the ring: it now holds the per-warp states
+  float *wpart = reinterpret_cast<float *>(ring);  // [kWarps][G][D+2]
   if (grp == 0) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -522,6 +623,238 @@ __device__ __forceinline__ void attend_rows(const T *__restrict__ Kb, const T *_
 }
 
 // ---------------------------------------------------------------------------
+// 5'. exact attention for bf16 caches on the tensor cores (warp-level mma.sync,
+//    bf16 operands, fp32 accumulation).  Rows are cut into tiles of 8 tokens;
+//    warp w streams tiles w, w+8, ... through its ring slice (cp.async, zero
+//    fill past cnt).  In a tile, token r's record is its K row then its V row,
+//    16-byte chunk c stored at chunk (c & ~7) | ((c ^ r) & 7) so that the eight
+//    rows an ldmatrix reads fall in distinct bank groups.  Per tile:
+//      logits  S[16 x 8] = Q[16 x D] . K^T   (rows: query heads, zero-padded
+//              to 16; columns: the 8 tokens; q_hat split into bf16 hi + lo);
+//      output  O^T[D x 8] += V^T[D x 8] . P^T[8 x 8]  (rows: dims; columns:
+//              query heads, padded to 8; P split into bf16 hi + lo), where the
+//              P fragment is exactly the S accumulator of the same lane.
+//    Thread (g = lane/4, t = lane%4) owns head g's logits for tokens 2t, 2t+1
+//    and the output of heads 2t, 2t+1 at dims 16j+g, 16j+g+8.
+template <int D, int G, bool GATHER>
+struct MmaRowStream {
+  static constexpr int RB = D * 2;            // bytes per row
+  static constexpr int REC = 2 * RB;          // K row + V row
+  static constexpr int CPT = REC / 16;        // chunks per token record
+  static constexpr int TILE = 8;
+  static constexpr int TB = TILE * REC;       // bytes per tile
+  static constexpr int NST = kWarpRingBytes / TB;
+  static_assert(NST >= 2, "ring slice must hold two tiles");
+
+  __device__ __forceinline__ static int swz(int c, int r) { return (c & ~7) | ((c ^ r) & 7); }
+
+  __device__ __forceinline__ static void issue(const __nv_bfloat16 *Kb, const __nv_bfloat16 *Vb,
+                                               const int32_t *ids, int tok0, int cnt, int s,
+                                               unsigned char *wring) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char *st = wring + (s % NST) * TB;
+    const int base = (s * kWarps + warp) * TILE;
+#pragma unroll
+    for (int x = 0; x < TILE * CPT / 32; ++x) {
+      const int q = x * 32 + lane;
+      const int r = q / CPT, c = q % CPT;
+      const int i = base + r;
+      const bool valid = i < cnt;
+      const int tok = valid ? (GATHER ? ids[i] : tok0 + i) : 0;
+      const __nv_bfloat16 *src = (c < CPT / 2 ? Kb : Vb) + (size_t)tok * D + (c % (CPT / 2)) * 8;
+      cp_async16_zfill(st + r * REC + swz(c, r) * 16, src, valid);
+    }
+  }
+
+  __device__ __forceinline__ static int warp_tiles(int cnt) {
+    const int warp = threadIdx.x >> 5;
+    const int tiles = (cnt + TILE - 1) / TILE;
+    return tiles > warp ? (tiles - warp + kWarps - 1) / kWarps : 0;
+  }
+};
+
+template <int D, int G, bool GATHER>
+__device__ __forceinline__ void attend_mma_prologue(const __nv_bfloat16 *Kb, const __nv_bfloat16 *Vb,
+                                                    const int32_t *ids, int tok0, int cnt, unsigned char *ring) {
+  using RS = MmaRowStream<D, G, GATHER>;
+  unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+#pragma unroll
+  for (int s = 0; s < RS::NST - 1; ++s) {
+    RS::issue(Kb, Vb, ids, tok0, cnt, s, wring);
+    cp_async_commit();
+  }
+}
+
+// The query operand: q_hat (pre-scaled, fp32) as two bf16 tiles hi and lo of
+// 8 rows x D (row h = head h, zero for h >= G), swizzled like the ring so
+// that ldmatrix reads them without bank conflicts.  Ends with __syncthreads().
+template <int D, int G>
+__device__ __forceinline__ void build_query_tiles(const float *qhat, unsigned char *qt) {
+  constexpr int RB = D * 2;
+  for (int e = threadIdx.x; e < 8 * D / 2; e += kThreads) {
+    const int r = e / (D / 2), c2 = e % (D / 2);  // row, pair of columns
+    float x0 = 0.f, x1 = 0.f;
+    if (r < G) {
+      x0 = qhat[r * D + 2 * c2];
+      x1 = qhat[r * D + 2 * c2 + 1];
+    }
+    uint32_t hi, lo;
+    split_bf16x2(x0, x1, hi, lo);
+    const int chunk = (2 * c2) / 8, within = (2 * c2) % 8;
+    const int off = r * RB + (((chunk & ~7) | ((chunk ^ r) & 7)) * 16) + within * 2;
+    *reinterpret_cast<uint32_t *>(qt + off) = hi;
+    *reinterpret_cast<uint32_t *>(qt + 8 * RB + off) = lo;
+  }
+  __syncthreads();
+}
+
+template <int D, int G, bool GATHER>
+__device__ __forceinline__ void attend_mma_loop(const __nv_bfloat16 *__restrict__ Kb,
+                                                const __nv_bfloat16 *__restrict__ Vb, const int32_t *ids,
+                                                int tok0, int cnt, const unsigned char *qt, unsigned char *ring,
+                                                float *pm, float *pl, float *pacc) {
+  using RS = MmaRowStream<D, G, GATHER>;
+  constexpr int KS = D / 16;  // k-steps of the logit product
+  constexpr int MT = D / 16;  // 16-dim tiles of the output product
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  unsigned char *wring = ring + warp * kWarpRingBytes;
+
+  float o[MT][4];
+#pragma unroll
+  for (int j = 0; j < MT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m = -INFINITY, lsum = 0.f;  // head g
+
+  const int nt = RS::warp_tiles(cnt);
+  const int r8 = lane & 7, mi = lane >> 3;
+  for (int s = 0; s < nt; ++s) {
+    cp_async_wait<RS::NST - 2>();
+    __syncwarp();
+    RS::issue(Kb, Vb, ids, tok0, cnt, s + RS::NST - 1, wring);
+    cp_async_commit();
+    const unsigned char *st = wring + (s % RS::NST) * RS::TB;
+    const int base = (s * kWarps + warp) * RS::TILE;
+
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int jj = 0; jj < KS / 2; ++jj) {
+      // rows 0-7 of the query tiles; rows 8-15 of the A operand are zero
+      const int qoff = r8 * (2 * D) + RS::swz(4 * jj + mi, r8) * 16;
+      uint32_t h0, h1, h2, h3, l0, l1, l2, l3, b0, b1, b2, b3;
+      ldsm_x4(smem_u32(qt + qoff), h0, h1, h2, h3);
+      ldsm_x4(smem_u32(qt + 8 * (2 * D) + qoff), l0, l1, l2, l3);
+      ldsm_x4(smem_u32(st + r8 * RS::REC + RS::swz(4 * jj + mi, r8) * 16), b0, b1, b2, b3);
+      mma_16816(sc, h0, 0u, h1, 0u, b0, b1);
+      mma_16816(sc, l0, 0u, l1, 0u, b0, b1);
+      mma_16816(sc, h2, 0u, h3, 0u, b2, b3);
+      mma_16816(sc, l2, 0u, l3, 0u, b2, b3);
+    }
+    const float s0 = (base + 2 * t < cnt) ? sc[0] : -INFINITY;
+    const float s1 = (base + 2 * t + 1 < cnt) ? sc[1] : -INFINITY;
+    float tmax = fmaxf(s0, s1);
+    tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
+    tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
+    const float mnew = fmaxf(m, tmax);
+    const float mref = (mnew == -INFINITY) ? 0.f : mnew;
+    const float corr = exp2f(m - mref);
+    const float p0 = exp2f(s0 - mref), p1 = exp2f(s1 - mref);
+    lsum = lsum * corr + p0 + p1;
+    m = mnew;
+    // this lane's output columns are heads 2t and 2t+1: their factors live in
+    // lanes 8t and 8t+4
+    const float ca = __shfl_sync(kFull, corr, 8 * t);
+    const float cb = __shfl_sync(kFull, corr, 8 * t + 4);
+#pragma unroll
+    for (int j = 0; j < MT; ++j) {
+      o[j][0] *= ca;
+      o[j][1] *= cb;
+      o[j][2] *= ca;
+      o[j][3] *= cb;
+    }
+    uint32_t ph, plo;
+    split_bf16x2(p0, p1, ph, plo);
+#pragma unroll
+    for (int jj = 0; jj < MT / 2; ++jj) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(smem_u32(st + r8 * RS::REC + RS::swz(RS::CPT / 2 + 4 * jj + mi, r8) * 16), a0, a1, a2, a3);
+      mma_1688(o[2 * jj], a0, a1, ph);
+      mma_1688(o[2 * jj], a0, a1, plo);
+      mma_1688(o[2 * jj + 1], a2, a3, ph);
+      mma_1688(o[2 * jj + 1], a2, a3, plo);
+    }
+  }
+  cp_async_wait<0>();
+  lsum += __shfl_xor_sync(kFull, lsum, 1);
+  lsum += __shfl_xor_sync(kFull, lsum, 2);
+
+  __syncthreads();  // every warp is done with the ring: it now holds the per-warp states
+  float *wpart = reinterpret_cast<float *>(ring);  // [kWarps][G][D+2]
+  const int h0 = 2 * t, h1 = 2 * t + 1;
+#pragma unroll
+  for (int j = 0; j < MT; ++j) {
+    if (h0 < G) {
+      wpart[(warp * G + h0) * (D + 2) + 16 * j + g] = o[j][0];
+      wpart[(warp * G + h0) * (D + 2) + 16 * j + g + 8] = o[j][2];
+    }
+    if (h1 < G) {
+      wpart[(warp * G + h1) * (D + 2) + 16 * j + g] = o[j][1];
+      wpart[(warp * G + h1) * (D + 2) + 16 * j + g + 8] = o[j][3];
+    }
+  }
+  if (t == 0 && g < G) {
+    wpart[(warp * G + g) * (D + 2) + D] = m;
+    wpart[(warp * G + g) * (D + 2) + D + 1] = lsum;
+  }
+  __syncthreads();
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int h = e / D, dim = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart[(w * G + h) * (D + 2) + D]);
+    const float mref = (M == -INFINITY) ? 0.f : M;
+    float A = 0.f, Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float *wp = wpart + (w * G + h) * (D + 2);
+      const float c = exp2f(wp[D] - mref);
+      A = fmaf(c, wp[dim], A);
+      Ls = fmaf(c, wp[D + 1], Ls);
+    }
+    pacc[e] = A;
+    if (dim == 0) {
+      pm[h] = M;
+      pl[h] = Ls;
+    }
+  }
+}
+
+// Dispatch: tensor cores for bf16 caches whose query group has G >= 4 heads
+// (there the CUDA-core loop, at 2G+1 instructions per cache element, can no
+// longer keep up with HBM); CUDA cores for smaller groups and for fp32 caches
+// (whose 1e-4 tolerance rules out bf16 operands).
+template <typename T, int D, int G, bool GATHER>
+__device__ __forceinline__ void attend_prologue_any(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+                                                    unsigned char *ring) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && G >= 4)
+    attend_mma_prologue<D, G, GATHER>(Kb, Vb, ids, tok0, cnt, ring);
+  else
+    attend_prologue<T, D, GATHER>(Kb, Vb, ids, tok0, cnt, ring);
+}
+
+// qtiles: 8*D words of shared memory that nothing else uses during the call.
+template <typename T, int D, int G, bool GATHER>
+__device__ __forceinline__ void attend_loop_any(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+                                                const float *qhat, unsigned char *qtiles, unsigned char *ring,
+                                                float *pm, float *pl, float *pacc) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && G >= 4) {
+    build_query_tiles<D, G>(qhat, qtiles);
+    attend_mma_loop<D, G, GATHER>(Kb, Vb, ids, tok0, cnt, qtiles, ring, pm, pl, pacc);
+  } else {
+    attend_loop<T, D, G, GATHER>(Kb, Vb, ids, tok0, cnt, qhat, ring, pm, pl, pacc);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 6. log-sum-exp combine of the cluster's partial states; CTA r writes the
 //    output elements r*256 + t (stride ncta*256).  Must follow a cluster
 //    barrier that orders every CTA's pm/pl/pacc writes.
@@ -545,43 +878,56 @@ __device__ __forceinline__ void cluster_combine(cg::cluster_group &cluster, int 
 
 // ---------------------------------------------------------------------------
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) loki_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
+__global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ncta = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int row = blockIdx.x / ncta;
   const int b = row / a.n_kv_heads, g = row % a.n_kv_heads;
-  const SmemLayout L = decode_layout(G, D, a.chunk, true);
+  const SmemLayout L = decode_layout(G, D, a.chunk, ncta, true);
   float *qhat = reinterpret_cast<float *>(smem + L.qhat);
   float *u = reinterpret_cast<float *>(smem + L.u);
   float *pm = reinterpret_cast<float *>(smem + L.pm);
   float *pl = reinterpret_cast<float *>(smem + L.pl);
   float *pacc = reinterpret_cast<float *>(smem + L.pacc);
   uint32_t *ctl = smem + L.ctl;
-  uint32_t *scratch = smem + L.scratch;
+  uint32_t *lhist = smem + L.lhist;
+  uint32_t *slots = smem + L.slots;
+  unsigned char *ring = reinterpret_cast<unsigned char *>(smem + L.ring);
   uint32_t *keys = smem + L.keys;
 
   const int t0 = min(a.seq_len, rank * a.chunk);
   const int len = min(a.seq_len, t0 + a.chunk) - t0;
-
-  rotate_queries<T, D, G>(a, b, g, qhat, u, reinterpret_cast<float *>(scratch), true);
-  if (rank == 0)
-    for (int i = threadIdx.x; i < 3 * 2048; i += kThreads) scratch[2048 + i] = 0u;
-  cluster_arrive();
-
   const size_t row_off = (size_t)row * a.capacity * D;
-  score_dispatch<T, D>(a.lpt, a.k_hat + row_off, t0, len, a.dpad, u, keys);
-  __syncthreads();
+  const T *Krow = a.k_hat + row_off;
+  constexpr int MAXL = D / VecN<T>::value;
 
-  const SelectState st = radix_select(cluster, keys, len, (uint32_t)a.k, scratch, scratch + 2048, ctl);
+  lhist[threadIdx.x] = 0u;  // ordered before the first atomic by the rotation's barriers
+  if (threadIdx.x < 32) ctl[kCtlGtAcc + threadIdx.x] = 0u;  // kCtlGtAcc and kCtlIn
+  rotate_queries<T, D, G>(a, b, g, qhat, u, reinterpret_cast<float *>(slots), true, [&] {
+    LOKI_LPT_DISPATCH(a.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.nck, ring)));
+  });
+  cluster_arrive();  // slots may now receive other CTAs' histograms
+  LOKI_LPT_DISPATCH(a.lpt, MAXL, (score_loop<T, D, L_>(Krow, t0, len, a.nck, ring, u, keys, lhist)));
+
+  const SelectState st = radix_select(cluster, ncta, rank, keys, len, (uint32_t)a.k, lhist, slots, ctl);
   int32_t *idx_row = a.idx + (size_t)row * a.k;
-  write_selection(cluster, ncta, rank, keys, len, t0, st, (uint32_t)a.k, ctl, idx_row);
+  write_selection(keys, len, t0, st, (uint32_t)a.k, ctl, idx_row);
+  cluster.sync();  // the whole row of idx is written and visible to the cluster
 
+  // this CTA's even share of the k selected rows; its indices are staged in
+  // shared memory (the score keys are dead now; the share is <= chunk), and
+  // clamped into the row so that no load can leave the cache even if they
+  // were wrong
   const int s0 = (int)(((long long)rank * a.k) / ncta);
   const int s1 = (int)(((long long)(rank + 1) * a.k) / ncta);
-  attend_rows<T, D, G, true>(a.k_hat + row_off, a.v + row_off, idx_row + s0, 0, s1 - s0, a.seq_len, qhat,
-                             reinterpret_cast<float *>(scratch), pm, pl, pacc);
+  int32_t *ids = reinterpret_cast<int32_t *>(keys);
+  for (int i = threadIdx.x; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), a.seq_len - 1);
+  __syncthreads();
+  attend_prologue_any<T, D, G, true>(Krow, a.v + row_off, ids, 0, s1 - s0, ring);
+  attend_loop_any<T, D, G, true>(Krow, a.v + row_off, ids, 0, s1 - s0, qhat,
+                                 reinterpret_cast<unsigned char *>(slots), ring, pm, pl, pacc);
   cluster.sync();
   const int Hq = a.n_kv_heads * G;
   cluster_combine<D, G>(cluster, ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);
@@ -589,27 +935,30 @@ __global__ void __launch_bounds__(kThreads) loki_decode_kernel(const __grid_cons
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) dense_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
+__global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ncta = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int row = blockIdx.x / ncta;
   const int b = row / a.n_kv_heads, g = row % a.n_kv_heads;
-  const SmemLayout L = decode_layout(G, D, a.chunk, false);
+  const SmemLayout L = decode_layout(G, D, a.chunk, ncta, false);
   float *qhat = reinterpret_cast<float *>(smem + L.qhat);
   float *u = reinterpret_cast<float *>(smem + L.u);
   float *pm = reinterpret_cast<float *>(smem + L.pm);
   float *pl = reinterpret_cast<float *>(smem + L.pl);
   float *pacc = reinterpret_cast<float *>(smem + L.pacc);
-  float *scratch = reinterpret_cast<float *>(smem + L.scratch);
+  float *scratch = reinterpret_cast<float *>(smem + L.slots);
+  unsigned char *ring = reinterpret_cast<unsigned char *>(smem + L.ring);
 
   const int t0 = min(a.seq_len, rank * a.chunk);
   const int len = min(a.seq_len, t0 + a.chunk) - t0;
-  rotate_queries<T, D, G>(a, b, g, qhat, u, scratch, false);
   const size_t row_off = (size_t)row * a.capacity * D;
-  attend_rows<T, D, G, false>(a.k_hat + row_off, a.v + row_off, nullptr, t0, len, a.seq_len, qhat, scratch,
-                              pm, pl, pacc);
+  rotate_queries<T, D, G>(a, b, g, qhat, u, scratch, false, [&] {
+    attend_prologue_any<T, D, G, false>(a.k_hat + row_off, a.v + row_off, nullptr, t0, len, ring);
+  });
+  attend_loop_any<T, D, G, false>(a.k_hat + row_off, a.v + row_off, nullptr, t0, len, qhat,
+                                  reinterpret_cast<unsigned char *>(scratch), ring, pm, pl, pacc);
   cluster.sync();
   const int Hq = a.n_kv_heads * G;
   cluster_combine<D, G>(cluster, ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);

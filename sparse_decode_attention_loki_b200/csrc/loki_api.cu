@@ -6,6 +6,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
 
 #include "loki.h"
 #include "append.cuh"
@@ -146,29 +149,8 @@ struct Plan {
   int smem;
 };
 
-int smem_bytes(int G, int D, int chunk, bool with_keys) {
-  return decode_layout(G, D, chunk, with_keys).words * 4;
-}
-
-loki_status plan(const DevInfo &di, const DecodeShape &sh, bool dense, Plan *p) {
-  const int rows = sh.B * sh.Hkv;
-  const long long target = 2LL * di.sms;      // aim for two resident CTAs per SM
-  constexpr int kMinTokens = 512;             // keep each CTA's stream long enough
-  int n = 1;
-  while (n < 16 && (long long)rows * n < target && (sh.S + 2 * n - 1) / (2 * n) >= kMinTokens) n *= 2;
-  const int limit = di.smem_optin;
-  while (n < 16 && smem_bytes(sh.G, sh.D, (sh.S + n - 1) / n, !dense) > limit) n *= 2;
-  const int forced = env_int("LOKI_CLUSTER", 0);
-  if (forced == 1 || forced == 2 || forced == 4 || forced == 8 || forced == 16) n = forced;
-  const int chunk = (sh.S + n - 1) / n;
-  const int smem = smem_bytes(sh.G, sh.D, chunk, !dense);
-  if (smem > limit)
-    return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d too long for on-chip scores (needs %d B of shared memory per CTA)",
-                sh.S, smem);
-  p->ncta = n;
-  p->chunk = chunk;
-  p->smem = smem;
-  return LOKI_OK;
+int smem_bytes(int G, int D, int chunk, int ncta, bool loki) {
+  return decode_layout(G, D, chunk, ncta, loki).words * 4;
 }
 
 void fill_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, const Plan &pl, int rows, void *stream) {
@@ -185,26 +167,82 @@ void fill_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, const Plan 
   cfg->numAttrs = 1;
 }
 
-// A 16-CTA cluster is non-portable: if the device cannot co-schedule one with
-// this much shared memory per CTA, fall back to 8 CTAs per row when the
-// scores still fit.
+// Co-resident clusters of `ncta` CTAs for a kernel with `smem` bytes of
+// dynamic shared memory (cached per device, kernel, cluster size and 4 KB
+// shared-memory bucket).  0 if the device cannot schedule such a cluster.
+struct OccEntry {
+  const void *kern;
+  int dev, ncta, smem_q, clusters;
+};
+std::mutex g_occ_mu;
+std::vector<OccEntry> g_occ;
+
 template <typename Kern>
-loki_status fit_cluster(Kern kern, const DecodeShape &sh, bool dense, int rows, Plan *pl, int smem_limit) {
-  if (pl->ncta <= 8) return LOKI_OK;
+int max_active_clusters(Kern kern, int dev, int ncta, int smem, int smem_limit) {
+  int smem_q = (smem + 4095) & ~4095;
+  if (smem_q > smem_limit) smem_q = smem;
+  {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    for (const OccEntry &e : g_occ)
+      if (e.kern == (const void *)kern && e.dev == dev && e.ncta == ncta && e.smem_q == smem_q) return e.clusters;
+  }
+  Plan pl{ncta, 0, smem_q};
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  fill_config(&cfg, attr, *pl, rows, nullptr);
-  int nclusters = 0;
-  cudaError_t e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
-  if (e == cudaSuccess && nclusters > 0) return LOKI_OK;
-  (void)cudaGetLastError();
-  const int chunk = (sh.S + 7) / 8;
-  const int smem = smem_bytes(sh.G, sh.D, chunk, !dense);
-  if (smem > smem_limit)
-    return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d needs 16-CTA clusters, which this device cannot schedule", sh.S);
-  pl->ncta = 8;
-  pl->chunk = chunk;
-  pl->smem = smem;
+  fill_config(&cfg, attr, pl, 1, nullptr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  g_occ.push_back(OccEntry{(const void *)kern, dev, ncta, smem_q, n});
+  return n;
+}
+
+// Launch plan: CTAs per row (cluster size) and tokens per CTA.  Among cluster
+// sizes whose per-CTA share is at least kMinTokens tokens and whose shared
+// memory fits, take the one that keeps the most CTAs busy per wave of
+// co-resident clusters (rows*n / waves); ties go to the smaller cluster, which
+// spends less on the cross-CTA steps.  LOKI_CLUSTER (tuning only) forces n.
+template <typename Kern>
+loki_status plan_for(Kern kern, const DevInfo &di, const DecodeShape &sh, bool dense, Plan *p) {
+  constexpr int kMinTokens = 256;
+  const int rows = sh.B * sh.Hkv;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int forced = env_int("LOKI_CLUSTER", 0);
+  double best = -1.0;
+  Plan bp{0, 0, 0};
+  int last_smem = 0;
+  for (int n = 1; n <= 16; n *= 2) {
+    if (forced && n != forced) continue;
+    const int chunk = (sh.S + n - 1) / n;
+    if (!forced && n > 1 && chunk < kMinTokens) continue;
+    const int smem = smem_bytes(sh.G, sh.D, chunk, n, !dense);
+    last_smem = smem;
+    if (smem > di.smem_optin) continue;
+    const int mc = max_active_clusters(kern, dev, n, smem, di.smem_optin);
+    if (mc <= 0) continue;
+    const long long waves = (rows + mc - 1) / mc;
+    const double per_wave = (double)rows * n / (double)waves;
+    if (per_wave > best * 1.0001) {
+      best = per_wave;
+      bp = Plan{n, chunk, smem};
+    }
+  }
+  if (bp.ncta == 0 && forced) {
+    setenv("LOKI_CLUSTER", "", 1);  // a forced size that cannot run: plan normally
+    loki_status s = plan_for(kern, di, sh, dense, p);
+    setenv("LOKI_CLUSTER", std::to_string(forced).c_str(), 1);
+    return s;
+  }
+  if (bp.ncta == 0)
+    return fail(LOKI_ERR_UNSUPPORTED,
+                "no launch shape fits: seq_len %d needs %d B of shared memory per CTA (limit %d) or an "
+                "unschedulable cluster",
+                sh.S, last_smem, di.smem_optin);
+  *p = bp;
   return LOKI_OK;
 }
 
@@ -229,12 +267,13 @@ template <typename T, int D, int G>
 std::atomic<int> DecodeKernels<T, D, G>::smem_dense[kMaxDevices];
 
 template <typename Kern, typename T>
-loki_status prepare_and_launch(Kern kern, std::atomic<int> *done_smem, const DecodeShape &sh, bool dense, Plan pl,
-                               int rows, DecodeArgs<T> args, int smem_limit, void *stream, Plan *used) {
+loki_status prepare_and_launch(Kern kern, std::atomic<int> *done_smem, const DevInfo &di, const DecodeShape &sh,
+                               bool dense, int rows, DecodeArgs<T> args, void *stream, Plan *used) {
   // the attribute covers every plan this device can take
-  loki_status s = prepare(kern, smem_limit, done_smem);
+  loki_status s = prepare(kern, di.smem_optin, done_smem);
   if (s != LOKI_OK) return s;
-  s = fit_cluster(kern, sh, dense, rows, &pl, smem_limit);
+  Plan pl;
+  s = plan_for(kern, di, sh, dense, &pl);
   if (s != LOKI_OK) return s;
   args.chunk = pl.chunk;
   if (used) *used = pl;
@@ -243,26 +282,25 @@ loki_status prepare_and_launch(Kern kern, std::atomic<int> *done_smem, const Dec
 }
 
 template <typename T, int D, int G>
-loki_status run_decode(bool dense, const DecodeShape &sh, const Plan &pl, int rows, const DecodeArgs<T> &args,
-                       int smem_limit, void *stream, Plan *used) {
+loki_status run_decode(bool dense, const DevInfo &di, const DecodeShape &sh, int rows, const DecodeArgs<T> &args,
+                       void *stream, Plan *used) {
   if (dense)
-    return prepare_and_launch(dense_decode_kernel<T, D, G>, DecodeKernels<T, D, G>::smem_dense, sh, true, pl, rows,
-                              args, smem_limit, stream, used);
-  return prepare_and_launch(loki_decode_kernel<T, D, G>, DecodeKernels<T, D, G>::smem_loki, sh, false, pl, rows,
-                            args, smem_limit, stream, used);
+    return prepare_and_launch(dense_decode_kernel<T, D, G>, DecodeKernels<T, D, G>::smem_dense, di, sh, true, rows,
+                              args, stream, used);
+  return prepare_and_launch(loki_decode_kernel<T, D, G>, DecodeKernels<T, D, G>::smem_loki, di, sh, false, rows,
+                            args, stream, used);
 }
 
 template <typename T, int D>
-loki_status run_decode_g(const DecodeShape &sh, bool dense, const Plan &pl, int rows, const DecodeArgs<T> &args,
-                         int smem_limit, void *stream, Plan *used) {
+loki_status run_decode_g(const DevInfo &di, const DecodeShape &sh, bool dense, int rows, const DecodeArgs<T> &args,
+                         void *stream, Plan *used) {
   switch (sh.G) {
-    case 1: return run_decode<T, D, 1>(dense, sh, pl, rows, args, smem_limit, stream, used);
-    case 2: return run_decode<T, D, 2>(dense, sh, pl, rows, args, smem_limit, stream, used);
-    case 4: return run_decode<T, D, 4>(dense, sh, pl, rows, args, smem_limit, stream, used);
-    case 8: return run_decode<T, D, 8>(dense, sh, pl, rows, args, smem_limit, stream, used);
+    case 1: return run_decode<T, D, 1>(dense, di, sh, rows, args, stream, used);
+    case 2: return run_decode<T, D, 2>(dense, di, sh, rows, args, stream, used);
+    case 4: return run_decode<T, D, 4>(dense, di, sh, rows, args, stream, used);
+    case 8: return run_decode<T, D, 8>(dense, di, sh, rows, args, stream, used);
   }
-  const int G = sh.G;
-  return fail(LOKI_ERR_UNSUPPORTED, "group size %d", G);
+  return fail(LOKI_ERR_UNSUPPORTED, "group size %d", sh.G);
 }
 
 template <typename T>
@@ -271,9 +309,6 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
                           Plan *used = nullptr) {
   DevInfo di;
   loki_status s = device_info(&di);
-  if (s != LOKI_OK) return s;
-  Plan pl;
-  s = plan(di, sh, dense, &pl);
   if (s != LOKI_OK) return s;
   constexpr int VEC = VecN<T>::value;
   DecodeArgs<T> a;
@@ -288,15 +323,15 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   a.seq_len = sh.S;
   a.d = d;
   a.k = k;
-  a.chunk = pl.chunk;
-  a.dpad = ((d + VEC - 1) / VEC) * VEC;
-  int need = a.dpad / VEC, lpt = 1;
-  while (lpt < need) lpt *= 2;
+  a.chunk = 0;  // set by the plan
+  a.nck = (d + VEC - 1) / VEC;
+  int lpt = 1;
+  while (lpt < a.nck) lpt *= 2;
   a.lpt = lpt;
   a.scale_log2 = resolve_scale(scale, sh.D);
   const int rows = sh.B * sh.Hkv;
-  if (sh.D == 64) return run_decode_g<T, 64>(sh, dense, pl, rows, a, di.smem_optin, stream, used);
-  return run_decode_g<T, 128>(sh, dense, pl, rows, a, di.smem_optin, stream, used);
+  if (sh.D == 64) return run_decode_g<T, 64>(di, sh, dense, rows, a, stream, used);
+  return run_decode_g<T, 128>(di, sh, dense, rows, a, stream, used);
 }
 
 template <typename T, int D>
@@ -323,18 +358,22 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   a.pos = pos;
   a.n_new = n_new;
   a.n_vec = c->batch * n_new;
-  // enough CTAs to cover the SMs twice, at least one 8-vector batch each
-  const long long want = (2LL * di.sms + c->n_kv_heads - 1) / c->n_kv_heads;
+  // enough CTAs to cover the SMs twice (heads x column blocks x chunks), at
+  // least one 8-vector batch each
+  const int col_blocks = D / kAppendCols;
+  const long long base = (long long)c->n_kv_heads * col_blocks;
+  const long long want = (2LL * di.sms + base - 1) / base;
   long long per = (a.n_vec + want - 1) / want;
   per = ((per + kAppendBatch - 1) / kAppendBatch) * kAppendBatch;
   if (per < kAppendBatch) per = kAppendBatch;
   a.per_cta = (int)per;
   const long long chunks = (a.n_vec + per - 1) / per;
-  if (chunks > 65535) return fail(LOKI_ERR_UNSUPPORTED, "append of %d vectors per head is too large", a.n_vec);
+  if (chunks > 65535 || c->n_kv_heads > 65535)
+    return fail(LOKI_ERR_UNSUPPORTED, "append of %d vectors per head is too large", a.n_vec);
   const int smem = append_smem_words(D) * 4;
   s = prepare(append_kernel<T, D>, smem, AppendKernel<T, D>::smem);
   if (s != LOKI_OK) return s;
-  dim3 grid((unsigned)c->n_kv_heads, (unsigned)chunks, 1);
+  dim3 grid((unsigned)c->n_kv_heads, (unsigned)col_blocks, (unsigned)chunks);
   append_kernel<T, D><<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "append_kernel launch");

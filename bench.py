@@ -317,8 +317,8 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     t_loki, t_dense, t_app, t_e2e = [float(x) for x in tt.tolist()]
-    cl, ct = L.loki_decode_launch_shape(cache, S, Hq)
-    dcl, dct = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
+    rot, ncl, nct, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
+    _, dcl, dct, _ = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
 
     if rank == 0:
         K = args.steps
@@ -338,17 +338,18 @@ def run_ours(args):
             "us_per_layer_step_per_gpu": loki_us,
             "hbm_gbs": ach,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                         "traffic": measured_traffic("loki_decode_kernel", w.name),
-                         "kernel": "loki_decode_kernel", "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+                         "traffic": measured_traffic("loki_decode_step", w.name),
+                         "kernel": "loki_rotate_kernel + loki_decode_kernel (programmatic dependent pair)",
+                         "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
                          "algorithmic_bytes_per_launch": lb},
             "dense": {"us": dense_us, "hbm_gbs": dach, "frac": dach / peak, "bytes_per_launch": db,
                       "launch": {"cluster_ctas": dcl, "ctas": dct}},
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
             "append_us": app_us,
-            "launch": {"cluster_ctas": cl, "ctas": ct, "threads_per_cta": 256},
+            "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256},
             "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gpu_launches": 3 * K,
+            "gpu_launches": 4 * K,
             "clocks": clocks,
             "wall_s_timed_region": wall,
             "per_step_loki_us": {"p50": float(np.percentile(per_step_loki, 50)) * 1000.0,

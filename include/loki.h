@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 1
+#define LOKI_VERSION 4
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -93,6 +93,14 @@ LOKI_API loki_status loki_append(const loki_cache *cache, int32_t pos, int32_t n
                         const void *k_new, const void *v_new, const float *P,
                         void *stream);
 
+/* loki_decode_workspace_size -- bytes of device workspace that
+ * loki_decode_attention needs for a cache of this shape with n_q_heads query
+ * heads: the rotated queries and the low-rank group queries of every (batch,
+ * KV head) row, B * Hkv * (G + 1) * D * 4 bytes plus alignment.  *bytes is a
+ * host pointer. */
+LOKI_API loki_status loki_decode_workspace_size(const loki_cache *cache, int32_t seq_len,
+                                       int32_t n_q_heads, size_t *bytes);
+
 /* loki_decode_attention -- one Loki decode step over tokens [0, seq_len).
  * Source: summary page, summary paragraph and section "Approach"; arXiv
  * record "Abstract".
@@ -104,17 +112,25 @@ LOKI_API loki_status loki_append(const loki_cache *cache, int32_t pos, int32_t n
  *   scale : softmax scale of the exact attention; <= 0 selects 1/sqrt(D).
  *   out   : [B, Hq, D] fp32 output (written).
  *   idx   : [B, Hkv, k] int32 selected token indices (written), ascending.
+ *   workspace, workspace_bytes : caller-owned device scratch of at least
+ *           loki_decode_workspace_size() bytes, 256-byte aligned.  Its contents
+ *           need no initialisation and are undefined after the call.  Calls
+ *           that may run at the same time (other streams) must not share a
+ *           workspace.
  * Per (b, g): q_hat_h = q_h . P_g (fp32, never rounded to the cache dtype);
  * score_i = sum over the G query heads h of group g of q_hat_h[:d] . k_hat_i[:d];
  * the k tokens with the largest scores are selected, ties going to the lower
  * index; out_h = softmax(scale * q_hat_h . k_hat_i over the selected i, full D)
- * weighted sum of v_i.  Requires seq_len <= S_cap, G in {1, 2, 4, 8}, and
- * seq_len small enough for the per-row scores to stay on chip (about 8e5
- * tokens); otherwise LOKI_ERR_UNSUPPORTED.  Needs no workspace. */
+ * weighted sum of v_i.  Requires seq_len <= S_cap and G in {1, 2, 4, 8};
+ * otherwise LOKI_ERR_INVALID_ARG or LOKI_ERR_UNSUPPORTED (also for seq_len
+ * above 393216 tokens, whose scores would not fit on chip).  Enqueues two
+ * kernels on the stream: the query rotation, then the decode kernel (scores,
+ * selection, attention) as its programmatic dependent. */
 LOKI_API loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len,
                                   int32_t n_q_heads, const void *q, const float *P,
                                   int32_t d, int32_t k, float scale, float *out,
-                                  int32_t *idx, void *stream);
+                                  int32_t *idx, void *workspace, size_t workspace_bytes,
+                                  void *stream);
 
 /* dense_decode_attention -- full softmax attention over every token
  * [0, seq_len) of the same rotated cache: the "Full Attention" baseline of the
@@ -126,13 +142,17 @@ LOKI_API loki_status dense_decode_attention(const loki_cache *cache, int32_t seq
                                    void *stream);
 
 /* Launch shape a decode call with these sizes would use, for logging and
- * tests: *cluster_ctas CTAs per (batch, KV head) row in one thread-block
- * cluster, *ctas the total grid.  `dense` selects the dense kernel.  Reads the
- * current device's attributes; launches nothing.  Output pointers are host
- * pointers. */
+ * tests.  shape: host array of 4 int32.
+ *   dense == 0 (loki_decode_attention): shape[0] CTAs of the query-rotation
+ *     kernel, shape[1] CTAs per (batch, KV head) row in one cluster of the
+ *     decode kernel, shape[2] CTAs of the decode kernel, shape[3] = 0.
+ *   dense != 0 (dense_decode_attention): shape[1] CTAs per row in one
+ *     cluster, shape[2] CTAs in all, shape[0] = shape[3] = 0.
+ * k is checked (1 <= k <= seq_len) for dense == 0 but does not change the
+ * shape.  Reads the current device's attributes; launches nothing. */
 LOKI_API loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len,
-                                     int32_t n_q_heads, int32_t dense,
-                                     int32_t *cluster_ctas, int32_t *ctas);
+                                     int32_t n_q_heads, int32_t k, int32_t dense,
+                                     int32_t *shape);
 
 /* Static description of a status code (never NULL). */
 LOKI_API const char *loki_status_string(loki_status s);

@@ -14,6 +14,7 @@ from .api import (
     loki_append,
     loki_decode_attention,
     loki_decode_launch_shape,
+    loki_decode_workspace_size,
     loki_status_string,
     loki_version,
 )
@@ -28,6 +29,7 @@ __all__ = [
     "loki_decode_attention",
     "dense_decode_attention",
     "loki_decode_launch_shape",
+    "loki_decode_workspace_size",
     "loki_status_string",
     "loki_version",
     "shard_batches",

@@ -68,6 +68,15 @@ class LokiCache:
     def desc(self) -> ctypes.POINTER(_lib.loki_cache):
         return ctypes.byref(self._desc)
 
+    def workspace(self, seq_len: int, n_q_heads: int) -> torch.Tensor:
+        """The decode workspace of this cache (scratch; no initialisation
+        needed), grown when a call needs more."""
+        need = loki_decode_workspace_size(self, seq_len, n_q_heads)
+        ws = getattr(self, "_ws", None)
+        if ws is None or ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws
+
 
 def loki_append(cache: LokiCache, pos: int, k_new: torch.Tensor, v_new: torch.Tensor, P: torch.Tensor,
                 stream: Optional[torch.cuda.Stream] = None) -> None:
@@ -82,12 +91,21 @@ def loki_append(cache: LokiCache, pos: int, k_new: torch.Tensor, v_new: torch.Te
                                        _stream_ptr(cache.device, stream)))
 
 
+def loki_decode_workspace_size(cache: LokiCache, seq_len: int, n_q_heads: int) -> int:
+    """Bytes of workspace a decode over seq_len tokens needs."""
+    n = ctypes.c_size_t(0)
+    _lib.check(_lib.load().loki_decode_workspace_size(cache.desc(), int(seq_len), int(n_q_heads), ctypes.byref(n)))
+    return int(n.value)
+
+
 def loki_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: torch.Tensor, d: int, k: int,
                           scale: float = 0.0, out: Optional[torch.Tensor] = None,
-                          idx: Optional[torch.Tensor] = None,
+                          idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                           stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """One Loki decode step.  q: [B, Hq, D] in the cache dtype.  Returns
-    (out [B, Hq, D] fp32, idx [B, Hkv, k] int32 ascending)."""
+    (out [B, Hq, D] fp32, idx [B, Hkv, k] int32 ascending).  `workspace`
+    (uint8 scratch on the cache's device, at least loki_decode_workspace_size
+    bytes) defaults to one the cache keeps."""
     B, Hq, D = q.shape if q.dim() == 3 else (-1, -1, -1)
     _need(q, "q", cache.dtype, (cache.batch, Hq, cache.head_dim), cache.device)
     _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
@@ -97,9 +115,13 @@ def loki_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: to
         idx = torch.empty((cache.batch, cache.n_kv_heads, int(k)), dtype=torch.int32, device=cache.device)
     _need(out, "out", torch.float32, (cache.batch, Hq, cache.head_dim), cache.device)
     _need(idx, "idx", torch.int32, (cache.batch, cache.n_kv_heads, int(k)), cache.device)
+    if workspace is None:
+        workspace = cache.workspace(seq_len, Hq)
+    if workspace.device != cache.device or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor on the cache's device")
     _lib.check(_lib.load().loki_decode_attention(cache.desc(), int(seq_len), int(Hq), _ptr(q), _ptr(P), int(d),
-                                                 int(k), float(scale), _ptr(out), _ptr(idx),
-                                                 _stream_ptr(cache.device, stream)))
+                                                 int(k), float(scale), _ptr(out), _ptr(idx), _ptr(workspace),
+                                                 int(workspace.numel()), _stream_ptr(cache.device, stream)))
     return out, idx
 
 
@@ -118,13 +140,16 @@ def dense_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: t
     return out
 
 
-def loki_decode_launch_shape(cache: LokiCache, seq_len: int, n_q_heads: int, dense: bool = False) -> Tuple[int, int]:
-    """(CTAs per (batch, KV head) row, total CTAs) of the decode launch."""
-    c, n = ctypes.c_int32(0), ctypes.c_int32(0)
+def loki_decode_launch_shape(cache: LokiCache, seq_len: int, n_q_heads: int, k: int = 1,
+                             dense: bool = False) -> Tuple[int, int, int, int]:
+    """Grid sizes of a decode call.  Loki: (rotation CTAs, decode CTAs per row
+    in one cluster, decode CTAs, 0).  Dense: (0, CTAs per row in one cluster,
+    CTAs, 0)."""
+    shape = (ctypes.c_int32 * 4)()
     with torch.cuda.device(cache.device):
-        _lib.check(_lib.load().loki_decode_launch_shape(cache.desc(), int(seq_len), int(n_q_heads), int(bool(dense)),
-                                                        ctypes.byref(c), ctypes.byref(n)))
-    return c.value, n.value
+        _lib.check(_lib.load().loki_decode_launch_shape(cache.desc(), int(seq_len), int(n_q_heads), int(k),
+                                                        int(bool(dense)), shape))
+    return tuple(int(x) for x in shape)
 
 
 def loki_status_string(status: int) -> str:

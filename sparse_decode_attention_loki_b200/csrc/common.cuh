@@ -130,6 +130,30 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Programmatic dependent launch.  griddep_wait(): block until every grid this
+// one depends on has completed and its memory operations are visible (returns
+// at once when the kernel was not launched as a dependent).
+// griddep_launch_dependents(): allow the dependent grid to be scheduled once
+// every CTA of this grid has executed it or exited.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 16-byte global load and store at L2 (not cached in L1): for data written by
+// other CTAs of the same grid and published through a fence + atomic.
+__device__ __forceinline__ uint4 ld_cg16(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void st_cg16(void *p, const uint4 &v) {
+  asm volatile("st.global.cg.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 // Split cluster barrier (arrive with release, wait with acquire).  Every thread
 // of every CTA in the cluster must execute each of them the same number of times.
 __device__ __forceinline__ void cluster_arrive() {

@@ -1,4 +1,4 @@
-// Loki decode-step kernels for sm_100a.
+// Building blocks of the Loki decode step and the dense decode kernel (sm_100a).
 //
 // Method ("Loki: Low-rank Keys for Efficient Sparse Attention", atlas.scime.ai
 // summary, section "Approach"): rotate the query into the PCA basis, rank every
@@ -6,32 +6,17 @@
 // compute exact softmax attention over them.  The dense kernel is the "Full
 // Attention" baseline (same page, "Experimental setup").
 //
-// B200 design.  One thread-block cluster of `ncta` CTAs owns one (batch, KV
-// head) row; CTA r owns the contiguous token range [r*chunk, (r+1)*chunk).
-// The whole decode step is one kernel:
-//   1. the first stages of the low-rank key stream are put in flight
-//      (cp.async into a shared-memory ring), then every CTA rotates the G
-//      queries of its KV group (q . P, fp32) and forms the group's low-rank
-//      query u = sum_h q_hat_h[:d] while those loads land;
-//   2. the CTA streams K_hat[i, :d] of its range through the ring and keeps one
-//      order-preserving uint32 key per token in shared memory -- scores never
-//      go to HBM;
-//   3. the cluster finds the k-th largest key by a radix select over 8-bit
-//      digits (at most 4 passes, usually 2-3): each CTA histograms its keys and
-//      stores the 256 counts into its slot in EVERY CTA of the cluster through
-//      distributed shared memory (16-byte DSMEM stores, double-buffered), so
-//      that after one cluster barrier every CTA derives the same digit, the
-//      per-CTA counts, and finally its own share of the ties and its offset;
-//   4. each CTA writes its selected token indices, ascending, at its offset in
-//      idx (ties at the threshold go to the lower index);
-//   5. the k selected tokens are split evenly over the cluster; each CTA
-//      gathers full K_hat and V rows through the ring and keeps an online
-//      softmax per query head (log2 domain, fp32);
-//   6. the CTAs' partial (max, sum, acc) states are merged through DSMEM with
-//      the log-sum-exp rule, and the output is written.
-// No workspace, no atomics in global memory, no software spin-waits: every
-// cross-CTA step is a hardware cluster barrier and every async copy is waited
-// for with cp.async.wait_group.
+// This file holds the pieces: the query rotation, the low-rank score stream,
+// the ordered write of a selection, the gather/stream attention loops (CUDA
+// cores, or warp-level tensor cores for query groups of 4+), the cluster
+// log-sum-exp combine and the dense decode kernel.  loki_step.cuh chains them
+// into the four kernels of one Loki step.
+//
+// Dense decode: one thread-block cluster of `ncta` CTAs owns one (batch, KV
+// head) row; CTA r streams the contiguous token range [r*chunk, (r+1)*chunk)
+// of K_hat and V through a per-warp cp.async ring with an online softmax per
+// query head, and the cluster merges the CTAs' (max, sum, acc) states through
+// distributed shared memory.  No workspace and no global atomics.
 #pragma once
 
 #include <type_traits>
@@ -68,8 +53,6 @@ constexpr int kStages = 4;
 constexpr int kWarpStageBytes = 2048;
 constexpr int kWarpRingBytes = kStages * kWarpStageBytes;
 constexpr int kRingWords = kWarps * kWarpRingBytes / 4;
-constexpr int kBins = 256;                 // 8-bit radix digits; one bin per thread
-static_assert(kThreads == kBins, "the select maps one histogram bin to each thread");
 
 __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 
@@ -77,15 +60,15 @@ __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 __host__ __device__ inline int rot_words(int G, int D) { return G * D + (kThreads / D) * G * D; }
 
 struct SmemLayout {
-  int qhat, u, pm, pl, pacc, ctl, lhist, slots, ring, keys, words;
+  int qhat, u, pm, pl, pacc, ctl, slots, ring, keys, words;
 };
 
-// Layout in 4-byte words, identical on host and device.  `slots` also serves
-// as the rotation scratch (before the CTA arrives on the first cluster
-// barrier no other CTA writes it) and, once the select is over, as the bf16
-// query tiles of the tensor-core attention; the ring also holds the per-warp
-// softmax states after the attention loop.
-__host__ __device__ inline SmemLayout decode_layout(int G, int D, int chunk, int ncta, bool loki) {
+// Layout in 4-byte words, identical on host and device.  `slots` serves as
+// the rotation scratch and then as the bf16 query tiles of the tensor-core
+// attention; the ring also holds the per-warp softmax states after the
+// attention loop.  `ids`: the attention kernel of the Loki step keeps its
+// share of the selected indices in the `keys` region (chunk words).
+__host__ __device__ inline SmemLayout decode_layout(int G, int D, int chunk, bool ids) {
   SmemLayout L;
   int o = 0;
   L.qhat = o;  o += G * D;
@@ -94,26 +77,19 @@ __host__ __device__ inline SmemLayout decode_layout(int G, int D, int chunk, int
   L.pl = o;    o += 16;
   L.pacc = o;  o += G * D;
   L.ctl = o;   o += 128;
-  L.lhist = o; o += loki ? kBins : 0;
   L.slots = o;
   {
-    const int s = loki ? 2 * ncta * kBins : 0;
     const int r = rot_words(G, D);
     const int q = 8 * D;  // bf16 query tiles of the tensor-core attention: 2 x 8 rows x D
-    const int m = s > r ? s : r;
-    o += round4(m > q ? m : q);
+    o += round4(r > q ? r : q);
   }
   L.ring = o;  o += kRingWords;
-  L.keys = o;  o += loki ? round4(chunk) : 0;
+  L.keys = o;  o += ids ? round4(chunk) : 0;
   L.words = o;
   return L;
 }
 
 // ctl word offsets (per CTA)
-constexpr int kCtlWtot = 0;       // [0..7]: warp totals for block scans
-constexpr int kCtlBucket = 8;     // [8..10]: bucket, count above it, count in it
-constexpr int kCtlGtAcc = 16;     // [16..31]: per-CTA count strictly above the prefix
-constexpr int kCtlIn = 32;        // [32..47]: per-CTA count in the bucket
 constexpr int kCtlWarpGt = 48;    // [48..55]
 constexpr int kCtlWarpEq = 56;    // [56..63]
 static_assert(kWarps == 8, "ctl layout assumes 8 warps");
@@ -178,22 +154,22 @@ __device__ __forceinline__ void rotate_queries(const DecodeArgs<T> &a, int b, in
 
 // ---------------------------------------------------------------------------
 // 2. low-rank score stream.  The CTA's tokens are cut into blocks of
-//    TS = kWarpStageBytes/(16*LPT) tokens; warp w streams blocks w, w+8, ...
-//    through its own ring slice.  Token t of a block keeps its LPT 16-byte
-//    chunks at byte (t*LPT + c)*16 of the stage; chunks c >= nck (beyond the
-//    first d dims) are neither copied nor used.  Each score becomes an
-//    order-preserving key in keys[], and the histogram of the keys' top byte
-//    (the first radix digit) is accumulated in lhist on the way.
-template <typename T, int D, int LPT>
+//    TS = SB/(16*LPT) tokens; warp w streams blocks w, w+8, ... through its
+//    own ring slice of NS stages of SB bytes.  Token t of a block keeps its
+//    LPT 16-byte chunks at byte (t*LPT + c)*16 of the stage; chunks c >= nck
+//    (beyond the first d dims) are neither copied nor used.  Each score
+//    becomes an order-preserving key in keys[].
+template <typename T, int D, int LPT, int SB = kWarpStageBytes, int NS = kStages>
 struct ScoreStream {
   static constexpr int VEC = VecN<T>::value;
-  static constexpr int TS = kWarpStageBytes / (16 * LPT);
-  static constexpr int TPW = 32 / LPT;  // tokens per warp instruction
+  static constexpr int TS = SB / (16 * LPT);  // tokens per warp stage
+  static constexpr int TPW = 32 / LPT;        // tokens per warp instruction
+  static_assert(TS >= TPW && TS % TPW == 0, "a stage must hold whole warp steps");
 
   __device__ __forceinline__ static void issue(const T *Krow, int t0, int len, int nck, int s,
                                                unsigned char *wring) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
+    unsigned char *st = wring + (s % NS) * SB;
     const int base = (s * kWarps + warp) * TS;
 #pragma unroll
     for (int it = 0; it < TS * LPT / 32; ++it) {
@@ -203,34 +179,41 @@ struct ScoreStream {
     }
   }
 
-  __device__ __forceinline__ static void consume(int len, int nck, int s, const unsigned char *wring,
-                                                 const float (&uv)[VEC], uint32_t *keys, uint32_t *lhist) {
+  // Score of token t of a stage: its nck chunks dotted with u, summed over the
+  // LPT lanes that share the token (every lane of the group gets the sum).
+  __device__ __forceinline__ static float dot_chunk(const unsigned char *st, int t, int c, int nck,
+                                                    const float (&uv)[VEC]) {
+    float sc = 0.f;
+    if (c < nck) {
+      const uint4 r = *reinterpret_cast<const uint4 *>(st + (t * LPT + c) * 16);
+      float f[VEC];
+      unpack16(r, f);
+#pragma unroll
+      for (int y = 0; y < VEC; ++y) sc = fmaf(uv[y], f[y], sc);
+    }
+#pragma unroll
+    for (int off = LPT / 2; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
+    return sc;
+  }
+
+  // keys[token] = score_key(score) for the tokens of stage s, and hist[key >>
+  // HSHIFT] += 1 for each of them.
+  template <int HSHIFT>
+  __device__ __forceinline__ static void consume_keys(int len, int nck, int s, const unsigned char *wring,
+                                                      const float (&uv)[VEC], uint32_t *keys, uint32_t *hist) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
+    const unsigned char *st = wring + (s % NS) * SB;
     const int c = lane % LPT;
     const int base = (s * kWarps + warp) * TS;
 #pragma unroll
     for (int step = 0; step < TS / TPW; ++step) {
       const int t = step * TPW + lane / LPT;
-      float sc = 0.f;
-      if (c < nck) {
-        const uint4 r = *reinterpret_cast<const uint4 *>(st + (t * LPT + c) * 16);
-        float f[VEC];
-        unpack16(r, f);
-#pragma unroll
-        for (int y = 0; y < VEC; ++y) sc = fmaf(uv[y], f[y], sc);
-      }
-#pragma unroll
-      for (int off = LPT / 2; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
-      const bool mine = c == 0 && base + t < len;
-      uint32_t bin = 0xffffffffu;
-      if (mine) {
+      const float sc = dot_chunk(st, t, c, nck, uv);
+      if (c == 0 && base + t < len) {
         const uint32_t key = score_key(sc);
         keys[base + t] = key;
-        bin = key >> 24;
+        atomicAdd(&hist[key >> HSHIFT], 1u);
       }
-      const uint32_t peers = __match_any_sync(kFull, bin);
-      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&lhist[bin], (uint32_t)__popc(peers));
     }
   }
 
@@ -241,35 +224,38 @@ struct ScoreStream {
   }
 };
 
-// Prologue: put the first kStages-1 stages of this warp in flight.
-template <typename T, int D, int LPT>
+// Prologue: put the first NS-1 stages of this warp in flight.
+template <typename T, int D, int LPT, int SB = kWarpStageBytes, int NS = kStages>
 __device__ __forceinline__ void score_prologue(const T *Krow, int t0, int len, int nck, unsigned char *ring) {
-  using SS = ScoreStream<T, D, LPT>;
-  unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+  using SS = ScoreStream<T, D, LPT, SB, NS>;
+  unsigned char *wring = ring + (threadIdx.x >> 5) * (SB * NS);
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
+  for (int s = 0; s < NS - 1; ++s) {
     SS::issue(Krow, t0, len, nck, s, wring);
     cp_async_commit();
   }
 }
 
-template <typename T, int D, int LPT>
-__device__ __forceinline__ void score_loop(const T *Krow, int t0, int len, int nck, unsigned char *ring,
-                                           const float *u, uint32_t *keys, uint32_t *lhist) {
-  using SS = ScoreStream<T, D, LPT>;
+// The key stream: leaves score_key(score) of every token of [t0, t0+len) in
+// keys[] and adds each key's top bits to hist[key >> HSHIFT].  Ends with
+// __syncthreads().
+template <typename T, int D, int LPT, int SB, int NS, int HSHIFT>
+__device__ __forceinline__ void score_keys_loop(const T *Krow, int t0, int len, int nck, unsigned char *ring,
+                                                const float *u, uint32_t *keys, uint32_t *hist) {
+  using SS = ScoreStream<T, D, LPT, SB, NS>;
   constexpr int VEC = VecN<T>::value;
-  unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+  unsigned char *wring = ring + (threadIdx.x >> 5) * (SB * NS);
   const int c = (threadIdx.x & 31) % LPT;
   float uv[VEC];
 #pragma unroll
   for (int y = 0; y < VEC; ++y) uv[y] = u[(c * VEC + y) % D];
   const int ns = SS::warp_stages(len);
   for (int s = 0; s < ns; ++s) {
-    cp_async_wait<kStages - 2>();
+    cp_async_wait<NS - 2>();
     __syncwarp();
-    SS::issue(Krow, t0, len, nck, s + kStages - 1, wring);
+    SS::issue(Krow, t0, len, nck, s + NS - 1, wring);
     cp_async_commit();
-    SS::consume(len, nck, s, wring, uv, keys, lhist);
+    SS::template consume_keys<HSHIFT>(len, nck, s, wring, uv, keys, hist);
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -290,88 +276,12 @@ __device__ __forceinline__ void score_loop(const T *Krow, int t0, int len, int n
   }
 
 // ---------------------------------------------------------------------------
-// 3. cluster radix select over 8-bit digits, most significant first.  Every
-//    CTA keeps the same (prefix, mask, remaining) and per-CTA counts; after it,
-//    this CTA's selected set is {key: key&mask > prefix} plus its first `take`
-//    keys (in token order) with key&mask == prefix, written from position
-//    `offset` of the row.  slots: [2][ncta][256] words; pass p stores this
-//    CTA's histogram into slot [p&1][rank] of every CTA.  On entry lhist holds
-//    the histogram of the keys' top byte (pass 0).  The caller zeroes
-//    ctl[kCtlGtAcc..kCtlIn+15] and performs cluster_arrive() before; pass 0
-//    performs the matching cluster_wait().
+// 3. the outcome of a radix select, as seen by one CTA: its selected set is
+//    {key : key & mask > prefix} plus its first `take` keys (in token order)
+//    with key & mask == prefix, written from position `offset` of the row.
 struct SelectState {
   uint32_t prefix, mask, take, offset;
 };
-
-__device__ __forceinline__ SelectState radix_select(cg::cluster_group &cluster, int ncta, int rank,
-                                                    const uint32_t *keys, int len, uint32_t k,
-                                                    uint32_t *lhist, uint32_t *slots, uint32_t *ctl) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t prefix = 0u, mask = 0u, remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    // the pass-0 histogram was accumulated by the score stream
-    if (pass > 0) lhist[tid] = 0u;
-    __syncthreads();
-    // warp-aggregated shared atomics: lanes with the same bin add once
-    for (int j0 = 0; pass > 0 && j0 < len; j0 += kThreads) {
-      const int j = j0 + tid;
-      uint32_t bin = 0xffffffffu;
-      if (j < len) {
-        const uint32_t key = keys[j];
-        if ((key & mask) == prefix) bin = (key >> shift) & (kBins - 1u);
-      }
-      const uint32_t peers = __match_any_sync(kFull, bin);
-      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&lhist[bin], (uint32_t)__popc(peers));
-    }
-    __syncthreads();
-    if (pass == 0) cluster_wait();  // every CTA of the cluster is running
-    uint32_t *buf = slots + (pass & 1) * ncta * kBins;
-    for (int q = tid; q < ncta * (kBins / 4); q += kThreads) {
-      const int dst = q / (kBins / 4), part = q % (kBins / 4);
-      uint4 *p = reinterpret_cast<uint4 *>(cluster.map_shared_rank(buf + rank * kBins, dst));
-      p[part] = reinterpret_cast<const uint4 *>(lhist)[part];
-    }
-    cluster.sync();
-    uint32_t tot = 0u;
-    for (int r = 0; r < ncta; ++r) tot += buf[r * kBins + tid];
-    const uint32_t above = block_excl_suffix_sum(tot, ctl + kCtlWtot);  // bins > tid
-    if (above < remaining && above + tot >= remaining) {
-      ctl[kCtlBucket + 0] = (uint32_t)tid;
-      ctl[kCtlBucket + 1] = above;
-      ctl[kCtlBucket + 2] = tot;
-    }
-    __syncthreads();
-    const uint32_t bucket = ctl[kCtlBucket + 0];
-    const uint32_t cnt_above = ctl[kCtlBucket + 1];
-    const uint32_t cnt_in = ctl[kCtlBucket + 2];
-    for (int r = warp; r < ncta; r += kWarps) {
-      uint32_t gt = 0u;
-      for (int x = lane; x < kBins; x += 32)
-        if ((uint32_t)x > bucket) gt += buf[r * kBins + x];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) gt += __shfl_xor_sync(kFull, gt, off);
-      if (lane == 0) {
-        ctl[kCtlGtAcc + r] += gt;
-        ctl[kCtlIn + r] = buf[r * kBins + bucket];
-      }
-    }
-    remaining -= cnt_above;
-    prefix |= bucket << shift;
-    mask |= (kBins - 1u) << shift;
-    __syncthreads();
-    if (cnt_in == remaining) break;  // the whole bucket is taken
-  }
-  // ties at the threshold are taken in token order: lower CTAs first
-  uint32_t eq_before = 0u, offset = 0u;
-  for (int r = 0; r < rank; ++r) {
-    const uint32_t want = remaining > eq_before ? remaining - eq_before : 0u;
-    offset += ctl[kCtlGtAcc + r] + min(ctl[kCtlIn + r], want);
-    eq_before += ctl[kCtlIn + r];
-  }
-  const uint32_t take = min(ctl[kCtlIn + rank], remaining > eq_before ? remaining - eq_before : 0u);
-  return SelectState{prefix, mask, take, offset};
-}
 
 // ---------------------------------------------------------------------------
 // 4. write this CTA's selected indices, ascending, from position st.offset of
@@ -876,64 +786,6 @@ __device__ __forceinline__ void cluster_combine(cg::cluster_group &cluster, int 
   }
 }
 
-// ---------------------------------------------------------------------------
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
-  extern __shared__ __align__(16) uint32_t smem[];
-  cg::cluster_group cluster = cg::this_cluster();
-  const int ncta = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int row = blockIdx.x / ncta;
-  const int b = row / a.n_kv_heads, g = row % a.n_kv_heads;
-  const SmemLayout L = decode_layout(G, D, a.chunk, ncta, true);
-  float *qhat = reinterpret_cast<float *>(smem + L.qhat);
-  float *u = reinterpret_cast<float *>(smem + L.u);
-  float *pm = reinterpret_cast<float *>(smem + L.pm);
-  float *pl = reinterpret_cast<float *>(smem + L.pl);
-  float *pacc = reinterpret_cast<float *>(smem + L.pacc);
-  uint32_t *ctl = smem + L.ctl;
-  uint32_t *lhist = smem + L.lhist;
-  uint32_t *slots = smem + L.slots;
-  unsigned char *ring = reinterpret_cast<unsigned char *>(smem + L.ring);
-  uint32_t *keys = smem + L.keys;
-
-  const int t0 = min(a.seq_len, rank * a.chunk);
-  const int len = min(a.seq_len, t0 + a.chunk) - t0;
-  const size_t row_off = (size_t)row * a.capacity * D;
-  const T *Krow = a.k_hat + row_off;
-  constexpr int MAXL = D / VecN<T>::value;
-
-  lhist[threadIdx.x] = 0u;  // ordered before the first atomic by the rotation's barriers
-  if (threadIdx.x < 32) ctl[kCtlGtAcc + threadIdx.x] = 0u;  // kCtlGtAcc and kCtlIn
-  rotate_queries<T, D, G>(a, b, g, qhat, u, reinterpret_cast<float *>(slots), true, [&] {
-    LOKI_LPT_DISPATCH(a.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.nck, ring)));
-  });
-  cluster_arrive();  // slots may now receive other CTAs' histograms
-  LOKI_LPT_DISPATCH(a.lpt, MAXL, (score_loop<T, D, L_>(Krow, t0, len, a.nck, ring, u, keys, lhist)));
-
-  const SelectState st = radix_select(cluster, ncta, rank, keys, len, (uint32_t)a.k, lhist, slots, ctl);
-  int32_t *idx_row = a.idx + (size_t)row * a.k;
-  write_selection(keys, len, t0, st, (uint32_t)a.k, ctl, idx_row);
-  cluster.sync();  // the whole row of idx is written and visible to the cluster
-
-  // this CTA's even share of the k selected rows; its indices are staged in
-  // shared memory (the score keys are dead now; the share is <= chunk), and
-  // clamped into the row so that no load can leave the cache even if they
-  // were wrong
-  const int s0 = (int)(((long long)rank * a.k) / ncta);
-  const int s1 = (int)(((long long)(rank + 1) * a.k) / ncta);
-  int32_t *ids = reinterpret_cast<int32_t *>(keys);
-  for (int i = threadIdx.x; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), a.seq_len - 1);
-  __syncthreads();
-  attend_prologue_any<T, D, G, true>(Krow, a.v + row_off, ids, 0, s1 - s0, ring);
-  attend_loop_any<T, D, G, true>(Krow, a.v + row_off, ids, 0, s1 - s0, qhat,
-                                 reinterpret_cast<unsigned char *>(slots), ring, pm, pl, pacc);
-  cluster.sync();
-  const int Hq = a.n_kv_heads * G;
-  cluster_combine<D, G>(cluster, ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);
-  cluster.sync();
-}
-
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
@@ -942,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kerne
   const int rank = (int)cluster.block_rank();
   const int row = blockIdx.x / ncta;
   const int b = row / a.n_kv_heads, g = row % a.n_kv_heads;
-  const SmemLayout L = decode_layout(G, D, a.chunk, ncta, false);
+  const SmemLayout L = decode_layout(G, D, a.chunk, false);
   float *qhat = reinterpret_cast<float *>(smem + L.qhat);
   float *u = reinterpret_cast<float *>(smem + L.u);
   float *pm = reinterpret_cast<float *>(smem + L.pm);

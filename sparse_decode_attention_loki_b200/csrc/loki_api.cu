@@ -13,6 +13,7 @@
 #include "loki.h"
 #include "append.cuh"
 #include "decode.cuh"
+#include "loki_step.cuh"
 
 namespace {
 
@@ -66,23 +67,6 @@ int env_int(const char *name, int dflt) {
   const char *s = std::getenv(name);
   if (!s || !*s) return dflt;
   return std::atoi(s);
-}
-
-// Raise a kernel's dynamic shared-memory limit (per device, remembered) and
-// allow 16-CTA clusters.
-template <typename Kern>
-loki_status prepare(Kern kern, int smem_bytes, std::atomic<int> *done_smem) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (done_smem[dev].load(std::memory_order_acquire) >= smem_bytes) return LOKI_OK;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(NonPortableClusterSizeAllowed)");
-  int prev = done_smem[dev].load();
-  while (prev < smem_bytes && !done_smem[dev].compare_exchange_weak(prev, smem_bytes)) {
-  }
-  return LOKI_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -142,29 +126,38 @@ float resolve_scale(float scale, int D) {
 }
 
 // ---------------------------------------------------------------------------
-// launch planning: CTAs per row (cluster size) and tokens per CTA
-struct Plan {
-  int ncta;
-  int chunk;
-  int smem;
-};
-
-int smem_bytes(int G, int D, int chunk, int ncta, bool loki) {
-  return decode_layout(G, D, chunk, ncta, loki).words * 4;
+// launches
+void set_cluster(cudaLaunchAttribute *attr, int ncta) {
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = (unsigned)ncta;
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+}
+void set_pdl(cudaLaunchAttribute *attr) {
+  attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr->val.programmaticStreamSerializationAllowed = 1;
 }
 
-void fill_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute *attr, const Plan &pl, int rows, void *stream) {
-  *cfg = cudaLaunchConfig_t{};
-  cfg->gridDim = dim3((unsigned)(rows * pl.ncta), 1, 1);
-  cfg->blockDim = dim3(kThreads, 1, 1);
-  cfg->dynamicSmemBytes = (size_t)pl.smem;
-  cfg->stream = static_cast<cudaStream_t>(stream);
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)pl.ncta;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg->attrs = attr;
-  cfg->numAttrs = 1;
+// Launch `kern` on `grid` CTAs of kThreads threads, as a cluster of `ncta`
+// CTAs when ncta > 0 and as a programmatic dependent of the previous kernel on
+// the stream when pdl is set.
+template <typename Kern, typename Args>
+loki_status launch_ex(Kern kern, long long grid, int smem, int ncta, bool pdl, const Args &args, void *stream,
+                      const char *what) {
+  if (grid < 1 || grid > 0x7fffffffLL) return fail(LOKI_ERR_UNSUPPORTED, "%s: grid of %lld CTAs", what, grid);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 0;
+  if (ncta > 0) set_cluster(&attr[cfg.numAttrs++], ncta);
+  if (pdl) set_pdl(&attr[cfg.numAttrs++]);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return LOKI_OK;
 }
 
 // Co-resident clusters of `ncta` CTAs for a kernel with `smem` bytes of
@@ -186,10 +179,14 @@ int max_active_clusters(Kern kern, int dev, int ncta, int smem, int smem_limit) 
     for (const OccEntry &e : g_occ)
       if (e.kern == (const void *)kern && e.dev == dev && e.ncta == ncta && e.smem_q == smem_q) return e.clusters;
   }
-  Plan pl{ncta, 0, smem_q};
-  cudaLaunchConfig_t cfg;
+  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  fill_config(&cfg, attr, pl, 1, nullptr);
+  cfg.gridDim = dim3((unsigned)ncta, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem_q;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  set_cluster(&attr[0], ncta);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -200,14 +197,28 @@ int max_active_clusters(Kern kern, int dev, int ncta, int smem, int smem_limit) 
   return n;
 }
 
-// Launch plan: CTAs per row (cluster size) and tokens per CTA.  Among cluster
-// sizes whose per-CTA share is at least kMinTokens tokens and whose shared
-// memory fits, take the one that keeps the most CTAs busy per wave of
-// co-resident clusters (rows*n / waves); ties go to the smaller cluster, which
-// spends less on the cross-CTA steps.  LOKI_CLUSTER (tuning only) forces n.
+// Per-kernel, per-device record of the dynamic shared memory already allowed.
+struct SmemGate {
+  std::atomic<int> bytes[kMaxDevices];
+};
+
+// ---------------------------------------------------------------------------
+// dense decode: one cluster of ncta CTAs per (batch, KV head) row
+struct Plan {
+  int ncta;
+  int chunk;
+  int smem;
+};
+
+// Among cluster sizes whose per-CTA share is at least kDenseMinTokens tokens
+// and whose shared memory fits, take the one that keeps the most CTAs busy per
+// wave of co-resident clusters (rows*n / waves); ties go to the smaller
+// cluster, which spends less on the cross-CTA merge.  LOKI_CLUSTER (tuning
+// only) forces n.
+constexpr int kDenseMinTokens = 256;
+
 template <typename Kern>
-loki_status plan_for(Kern kern, const DevInfo &di, const DecodeShape &sh, bool dense, Plan *p) {
-  constexpr int kMinTokens = 256;
+loki_status plan_dense(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan *p) {
   const int rows = sh.B * sh.Hkv;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -218,8 +229,8 @@ loki_status plan_for(Kern kern, const DevInfo &di, const DecodeShape &sh, bool d
   for (int n = 1; n <= 16; n *= 2) {
     if (forced && n != forced) continue;
     const int chunk = (sh.S + n - 1) / n;
-    if (!forced && n > 1 && chunk < kMinTokens) continue;
-    const int smem = smem_bytes(sh.G, sh.D, chunk, n, !dense);
+    if (!forced && n > 1 && chunk < kDenseMinTokens) continue;
+    const int smem = decode_layout(sh.G, sh.D, chunk, false).words * 4;
     last_smem = smem;
     if (smem > di.smem_optin) continue;
     const int mc = max_active_clusters(kern, dev, n, smem, di.smem_optin);
@@ -233,79 +244,164 @@ loki_status plan_for(Kern kern, const DevInfo &di, const DecodeShape &sh, bool d
   }
   if (bp.ncta == 0 && forced) {
     setenv("LOKI_CLUSTER", "", 1);  // a forced size that cannot run: plan normally
-    loki_status s = plan_for(kern, di, sh, dense, p);
+    loki_status s = plan_dense(kern, di, sh, p);
     setenv("LOKI_CLUSTER", std::to_string(forced).c_str(), 1);
     return s;
   }
   if (bp.ncta == 0)
     return fail(LOKI_ERR_UNSUPPORTED,
-                "no launch shape fits: seq_len %d needs %d B of shared memory per CTA (limit %d) or an "
-                "unschedulable cluster",
-                sh.S, last_smem, di.smem_optin);
+                "no dense launch shape fits: %d B of shared memory per CTA (limit %d) or an unschedulable cluster",
+                last_smem, di.smem_optin);
   *p = bp;
   return LOKI_OK;
 }
 
-template <typename Kern, typename Args>
-loki_status launch(Kern kern, const Plan &pl, int rows, const Args &args, void *stream) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  fill_config(&cfg, attr, pl, rows, stream);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
+// Raise a kernel's dynamic shared-memory limit to the device's opt-in maximum
+// (once per device and kernel: `gate` belongs to exactly one kernel) and allow
+// clusters of up to 16 CTAs.  Launches then pass their own smaller sizes.
+template <typename Kern>
+loki_status allow_smem(Kern kern, const DevInfo &di, SmemGate &gate, bool cluster) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (gate.bytes[dev].load(std::memory_order_acquire) >= di.smem_optin) return LOKI_OK;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.smem_optin);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
+  if (cluster) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(NonPortableClusterSizeAllowed)");
+  }
+  gate.bytes[dev].store(di.smem_optin, std::memory_order_release);
   return LOKI_OK;
 }
 
 template <typename T, int D, int G>
-struct DecodeKernels {
-  static std::atomic<int> smem_loki[kMaxDevices];
-  static std::atomic<int> smem_dense[kMaxDevices];
+struct DenseGate {
+  static SmemGate gate;
 };
 template <typename T, int D, int G>
-std::atomic<int> DecodeKernels<T, D, G>::smem_loki[kMaxDevices];
-template <typename T, int D, int G>
-std::atomic<int> DecodeKernels<T, D, G>::smem_dense[kMaxDevices];
+SmemGate DenseGate<T, D, G>::gate;
 
-template <typename Kern, typename T>
-loki_status prepare_and_launch(Kern kern, std::atomic<int> *done_smem, const DevInfo &di, const DecodeShape &sh,
-                               bool dense, int rows, DecodeArgs<T> args, void *stream, Plan *used) {
-  // the attribute covers every plan this device can take
-  loki_status s = prepare(kern, di.smem_optin, done_smem);
+template <typename T, int D, int G>
+loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a, void *stream, Plan *used) {
+  auto kern = dense_decode_kernel<T, D, G>;
+  loki_status s = allow_smem(kern, di, DenseGate<T, D, G>::gate, true);
   if (s != LOKI_OK) return s;
   Plan pl;
-  s = plan_for(kern, di, sh, dense, &pl);
+  s = plan_dense(kern, di, sh, &pl);
   if (s != LOKI_OK) return s;
-  args.chunk = pl.chunk;
-  if (used) *used = pl;
-  if (!stream && used) return LOKI_OK;  // shape query only
-  return launch(kern, pl, rows, args, stream);
+  if (used) {  // shape query only: launch nothing
+    *used = pl;
+    return LOKI_OK;
+  }
+  a.chunk = pl.chunk;
+  return launch_ex(kern, (long long)sh.B * sh.Hkv * pl.ncta, pl.smem, pl.ncta, false, a, stream,
+                   "dense_decode_kernel launch");
+}
+
+// ---------------------------------------------------------------------------
+// Loki step: rotate grid, then the decode grid as its programmatic dependent
+struct StepPlan {
+  int ncta, chunk, smem;
+};
+
+// CTAs per row (cluster size) of the decode kernel: the largest power of two
+// up to 16 that keeps the grid within one wave of co-resident CTAs, but never
+// fewer than the share of kMaxChunk tokens per CTA needs, and only sizes the
+// device can schedule.  LOKI_CLUSTER (a tuning override) forces the size.
+template <typename Kern>
+loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepPlan *p) {
+  const long long rows = (long long)sh.B * sh.Hkv;
+  const int S = sh.S;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int need = 1;
+  while (need < kMaxCluster && (S + need - 1) / need > kMaxChunk) need *= 2;
+  if ((S + need - 1) / need > kMaxChunk)
+    return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d exceeds %d tokens", S, kMaxChunk * kMaxCluster);
+  const int forced = env_int("LOKI_CLUSTER", 0);
+  StepPlan best{0, 0, 0};
+  for (int n = kMaxCluster; n >= need; n /= 2) {
+    if (forced && n != forced) continue;
+    const int chunk = round4((S + n - 1) / n);
+    const int smem = fused_smem(sh.G, sh.D, chunk).words * 4;
+    if (smem > di.smem_optin) continue;
+    const int mc = max_active_clusters(kern, dev, n, smem, di.smem_optin);
+    if (mc <= 0) continue;
+    best = StepPlan{n, chunk, smem};
+    if (forced || rows <= mc) break;  // one wave (or forced)
+  }
+  if (best.ncta == 0 && forced) {
+    setenv("LOKI_CLUSTER", "", 1);  // a forced size that cannot run: plan normally
+    loki_status s = plan_step(kern, di, sh, p);
+    setenv("LOKI_CLUSTER", std::to_string(forced).c_str(), 1);
+    return s;
+  }
+  if (best.ncta == 0)
+    return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d: no schedulable cluster fits the keys in shared memory", S);
+  *p = best;
+  return LOKI_OK;
 }
 
 template <typename T, int D, int G>
-loki_status run_decode(bool dense, const DevInfo &di, const DecodeShape &sh, int rows, const DecodeArgs<T> &args,
-                       void *stream, Plan *used) {
-  if (dense)
-    return prepare_and_launch(dense_decode_kernel<T, D, G>, DecodeKernels<T, D, G>::smem_dense, di, sh, true, rows,
-                              args, stream, used);
-  return prepare_and_launch(loki_decode_kernel<T, D, G>, DecodeKernels<T, D, G>::smem_loki, di, sh, false, rows,
-                            args, stream, used);
+struct StepGate {
+  static SmemGate gate;
+};
+template <typename T, int D, int G>
+SmemGate StepGate<T, D, G>::gate;
+
+template <typename T, int D, int G>
+loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da, void *ws, void *stream,
+                     StepPlan *used) {
+  auto kern = loki_decode_kernel<T, D, G>;
+  loki_status s = allow_smem(kern, di, StepGate<T, D, G>::gate, true);
+  if (s != LOKI_OK) return s;
+  StepPlan pl;
+  s = plan_step(kern, di, sh, &pl);
+  if (s != LOKI_OK) return s;
+  if (used) {  // shape query only: launch nothing
+    *used = pl;
+    return LOKI_OK;
+  }
+  const long long rows = (long long)sh.B * sh.Hkv;
+  const WsLayout W = ws_layout(rows, G, D);
+  unsigned char *w = static_cast<unsigned char *>(ws);
+  da.chunk = pl.chunk;
+  StepArgs<T> a;
+  a.da = da;
+  a.qhat = reinterpret_cast<float *>(w + W.qhat);
+  a.u = reinterpret_cast<float *>(w + W.u);
+  s = launch_ex(loki_rotate_kernel<T, D, G>, rows * (D / kRotCols), 0, 0, false, a, stream,
+                "loki_rotate_kernel launch");
+  if (s != LOKI_OK) return s;
+  return launch_ex(kern, rows * pl.ncta, pl.smem, pl.ncta, true, a, stream, "loki_decode_kernel launch");
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, int D, int G>
+loki_status dispatch(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
+                     void *stream, Plan *used) {
+  if (dense) return run_dense<T, D, G>(di, sh, a, stream, used);
+  StepPlan sp;
+  loki_status s = run_step<T, D, G>(di, sh, a, ws, stream, used ? &sp : nullptr);
+  if (s == LOKI_OK && used) *used = Plan{sp.ncta, sp.chunk, sp.smem};
+  return s;
 }
 
 template <typename T, int D>
-loki_status run_decode_g(const DevInfo &di, const DecodeShape &sh, bool dense, int rows, const DecodeArgs<T> &args,
-                         void *stream, Plan *used) {
+loki_status dispatch_g(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
+                       void *stream, Plan *used) {
   switch (sh.G) {
-    case 1: return run_decode<T, D, 1>(dense, di, sh, rows, args, stream, used);
-    case 2: return run_decode<T, D, 2>(dense, di, sh, rows, args, stream, used);
-    case 4: return run_decode<T, D, 4>(dense, di, sh, rows, args, stream, used);
-    case 8: return run_decode<T, D, 8>(dense, di, sh, rows, args, stream, used);
+    case 1: return dispatch<T, D, 1>(dense, di, sh, a, ws, stream, used);
+    case 2: return dispatch<T, D, 2>(dense, di, sh, a, ws, stream, used);
+    case 4: return dispatch<T, D, 4>(dense, di, sh, a, ws, stream, used);
+    case 8: return dispatch<T, D, 8>(dense, di, sh, a, ws, stream, used);
   }
   return fail(LOKI_ERR_UNSUPPORTED, "group size %d", sh.G);
 }
 
 template <typename T>
 loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense, const void *q, const float *P,
-                          int32_t d, int32_t k, float scale, float *out, int32_t *idx, void *stream,
+                          int32_t d, int32_t k, float scale, float *out, int32_t *idx, void *ws, void *stream,
                           Plan *used = nullptr) {
   DevInfo di;
   loki_status s = device_info(&di);
@@ -329,17 +425,16 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   while (lpt < a.nck) lpt *= 2;
   a.lpt = lpt;
   a.scale_log2 = resolve_scale(scale, sh.D);
-  const int rows = sh.B * sh.Hkv;
-  if (sh.D == 64) return run_decode_g<T, 64>(di, sh, dense, rows, a, stream, used);
-  return run_decode_g<T, 128>(di, sh, dense, rows, a, stream, used);
+  if (sh.D == 64) return dispatch_g<T, 64>(dense, di, sh, a, ws, stream, used);
+  return dispatch_g<T, 128>(dense, di, sh, a, ws, stream, used);
 }
 
 template <typename T, int D>
-struct AppendKernel {
-  static std::atomic<int> smem[kMaxDevices];
+struct AppendGate {
+  static SmemGate gate;
 };
 template <typename T, int D>
-std::atomic<int> AppendKernel<T, D>::smem[kMaxDevices];
+SmemGate AppendGate<T, D>::gate;
 
 template <typename T, int D>
 loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const void *k_new, const void *v_new,
@@ -371,7 +466,7 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   if (chunks > 65535 || c->n_kv_heads > 65535)
     return fail(LOKI_ERR_UNSUPPORTED, "append of %d vectors per head is too large", a.n_vec);
   const int smem = append_smem_words(D) * 4;
-  s = prepare(append_kernel<T, D>, smem, AppendKernel<T, D>::smem);
+  s = allow_smem(append_kernel<T, D>, di, AppendGate<T, D>::gate, false);
   if (s != LOKI_OK) return s;
   dim3 grid((unsigned)c->n_kv_heads, (unsigned)col_blocks, (unsigned)chunks);
   append_kernel<T, D><<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
@@ -402,9 +497,23 @@ loki_status loki_append(const loki_cache *cache, int32_t pos, int32_t n_new, con
                     : run_append<__nv_bfloat16, 128>(cache, pos, n_new, k_new, v_new, P, stream);
 }
 
+loki_status loki_decode_workspace_size(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads,
+                                       size_t *bytes) {
+  DecodeShape sh;
+  loki_status s = check_cache(cache, &sh);
+  if (s != LOKI_OK) return s;
+  if (!bytes) return fail(LOKI_ERR_INVALID_ARG, "bytes is NULL");
+  if (seq_len < 1 || seq_len > sh.Scap)
+    return fail(LOKI_ERR_INVALID_ARG, "seq_len %d outside [1, capacity=%d]", seq_len, sh.Scap);
+  if (n_q_heads < sh.Hkv || n_q_heads % sh.Hkv != 0)
+    return fail(LOKI_ERR_INVALID_ARG, "n_q_heads %d is not a positive multiple of n_kv_heads %d", n_q_heads, sh.Hkv);
+  *bytes = ws_layout((long long)sh.B * sh.Hkv, n_q_heads / sh.Hkv, sh.D).total;
+  return LOKI_OK;
+}
+
 loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, const void *q,
                                   const float *P, int32_t d, int32_t k, float scale, float *out, int32_t *idx,
-                                  void *stream) {
+                                  void *workspace, size_t workspace_bytes, void *stream) {
   DecodeShape sh;
   loki_status s = check_decode(cache, seq_len, n_q_heads, q, P, out, &sh);
   if (s != LOKI_OK) return s;
@@ -412,9 +521,15 @@ loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len, int3
   if (k < 1 || k > seq_len) return fail(LOKI_ERR_INVALID_ARG, "k=%d outside [1, seq_len=%d]", k, seq_len);
   if (!idx) return fail(LOKI_ERR_INVALID_ARG, "idx is NULL");
   if (!aligned(idx, 4)) return fail(LOKI_ERR_INVALID_ARG, "idx must be 4-byte aligned");
+  if (!workspace) return fail(LOKI_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(LOKI_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = ws_layout((long long)sh.B * sh.Hkv, sh.G, sh.D).total;
+  if (workspace_bytes < need)
+    return fail(LOKI_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes this call needs",
+                workspace_bytes, need);
   if (cache->dtype == LOKI_F32)
-    return decode_common<float>(cache, sh, false, q, P, d, k, scale, out, idx, stream);
-  return decode_common<__nv_bfloat16>(cache, sh, false, q, P, d, k, scale, out, idx, stream);
+    return decode_common<float>(cache, sh, false, q, P, d, k, scale, out, idx, workspace, stream);
+  return decode_common<__nv_bfloat16>(cache, sh, false, q, P, d, k, scale, out, idx, workspace, stream);
 }
 
 loki_status dense_decode_attention(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, const void *q,
@@ -423,32 +538,37 @@ loki_status dense_decode_attention(const loki_cache *cache, int32_t seq_len, int
   loki_status s = check_decode(cache, seq_len, n_q_heads, q, P, out, &sh);
   if (s != LOKI_OK) return s;
   if (cache->dtype == LOKI_F32)
-    return decode_common<float>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, stream);
-  return decode_common<__nv_bfloat16>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, stream);
+    return decode_common<float>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream);
+  return decode_common<__nv_bfloat16>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream);
 }
 
-loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, int32_t dense,
-                                     int32_t *cluster_ctas, int32_t *ctas) {
+loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, int32_t k,
+                                     int32_t dense, int32_t *shape) {
   DecodeShape sh;
   loki_status s = check_cache(cache, &sh);
   if (s != LOKI_OK) return s;
   if (seq_len < 1 || seq_len > sh.Scap) return fail(LOKI_ERR_INVALID_ARG, "seq_len %d outside [1, capacity]", seq_len);
   if (n_q_heads < sh.Hkv || n_q_heads % sh.Hkv != 0) return fail(LOKI_ERR_INVALID_ARG, "bad n_q_heads");
+  if (!dense && (k < 1 || k > seq_len)) return fail(LOKI_ERR_INVALID_ARG, "k=%d outside [1, seq_len=%d]", k, seq_len);
+  if (!shape) return fail(LOKI_ERR_INVALID_ARG, "shape is NULL");
   sh.S = seq_len;
   sh.Hq = n_q_heads;
   sh.G = n_q_heads / sh.Hkv;
-  if (!cluster_ctas || !ctas) return fail(LOKI_ERR_INVALID_ARG, "output pointers are NULL");
   if (sh.G != 1 && sh.G != 2 && sh.G != 4 && sh.G != 8)
     return fail(LOKI_ERR_UNSUPPORTED, "query group size %d not supported (1, 2, 4 or 8)", sh.G);
+  const long long rows = (long long)sh.B * sh.Hkv;
   Plan pl;
   if (cache->dtype == LOKI_F32)
-    s = decode_common<float>(cache, sh, dense != 0, nullptr, nullptr, 1, 1, 0.f, nullptr, nullptr, nullptr, &pl);
+    s = decode_common<float>(cache, sh, dense != 0, nullptr, nullptr, 1, 1, 0.f, nullptr, nullptr, nullptr, nullptr,
+                             &pl);
   else
     s = decode_common<__nv_bfloat16>(cache, sh, dense != 0, nullptr, nullptr, 1, 1, 0.f, nullptr, nullptr, nullptr,
-                                     &pl);
+                                     nullptr, &pl);
   if (s != LOKI_OK) return s;
-  *cluster_ctas = pl.ncta;
-  *ctas = pl.ncta * sh.B * sh.Hkv;
+  shape[0] = dense ? 0 : (int32_t)(rows * (sh.D / kRotCols));
+  shape[1] = pl.ncta;
+  shape[2] = (int32_t)(rows * pl.ncta);
+  shape[3] = 0;
   return LOKI_OK;
 }
 

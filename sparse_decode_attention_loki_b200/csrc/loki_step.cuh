@@ -1,0 +1,492 @@
+// One Loki decode step in two kernels ("Loki: Low-rank Keys for Efficient
+// Sparse Attention", atlas.scime.ai summary, section "Approach": PCA-project
+// queries and keys, rank tokens on the top-d principal dimensions, exact
+// attention over the top-k tokens).
+//
+//   rotate  D/32 CTAs per (batch, KV head) row: q_hat_h = q_h . P_g for the G
+//           query heads of the row (fp32, pre-scaled for the softmax) and the
+//           group's low-rank query u = sum_h q_hat_h[:d], into the workspace.
+//   decode  one thread-block cluster of ncta CTAs per row, about one wave of
+//           CTAs in all; CTA r owns tokens [r*chunk, (r+1)*chunk):
+//     1. the first stages of its low-rank key stream go in flight (cp.async
+//        ring) before it waits for the rotate grid (programmatic dependent
+//        launch), then it streams K_hat[i, :d], keeps one order-preserving
+//        uint32 key per token in shared memory and histograms the keys' top
+//        11 bits on the way;
+//     2. cluster radix select over 11/11/10-bit digits: each CTA adds the
+//        non-zero bins of its histogram into every CTA of the cluster through
+//        distributed shared memory, so after one cluster barrier every CTA
+//        knows the bucket of the k-th largest key; the keys in that bucket
+//        (the candidates) are refined the same way; the CTAs then exchange
+//        their counts above and at the threshold and write their indices in
+//        ascending order, ties at the threshold going to the lower index;
+//     3. the k selected rows are split evenly over the cluster: gather K_hat
+//        and V rows through the ring, online softmax per query head;
+//     4. the CTAs' (max, sum, acc) states are merged through distributed
+//        shared memory with the log-sum-exp rule into out.
+// Scores never leave the chip; the workspace holds only q_hat and u.
+#pragma once
+
+#include "decode.cuh"
+
+namespace loki {
+
+constexpr int kDig1Bits = 11;                   // first radix digit: key bits 31..21
+constexpr int kDig1Bins = 1 << kDig1Bits;       // 2048
+constexpr int kDig2Bits = 11;                   // second digit: bits 20..10
+constexpr int kDig3Bits = 10;                   // third digit: bits 9..0
+constexpr int kMaxCluster = 16;
+constexpr int kMaxChunk = 24576;                // tokens per decode CTA, at most
+constexpr int kCandCap = 4096;                  // candidate list per CTA (keys)
+
+// Workspace layout (bytes, each region 256-byte aligned).
+struct WsLayout {
+  size_t qhat, u, total;
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+__host__ __device__ inline WsLayout ws_layout(long long rows, int G, int D) {
+  WsLayout w;
+  size_t o = 0;
+  w.qhat = o; o = align256(o + (size_t)rows * G * D * 4);
+  w.u = o;    o = align256(o + (size_t)rows * D * 4);
+  w.total = o;
+  return w;
+}
+
+template <typename T>
+struct StepArgs {
+  DecodeArgs<T> da;  // cache, q, P, out, idx, sizes, d, k, scale; da.chunk = tokens per decode CTA
+  float *qhat;       // [rows, G, D], pre-scaled by scale * log2(e)
+  float *u;          // [rows, D], zero beyond d
+};
+
+// ---------------------------------------------------------------------------
+// rotate: CTA (row, cb) computes columns [32cb, 32cb + 32) of q_hat for the G
+// query heads of the row from a 32-column slice of P_g held in shared memory,
+// and those columns of u that lie below d.
+constexpr int kRotCols = 32;
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads) loki_rotate_kernel(const __grid_constant__ StepArgs<T> a) {
+  constexpr int NB = D / kRotCols;        // column blocks per row
+  constexpr int PARTS = kThreads / kRotCols;  // 8 partial sums per column
+  constexpr int RPP = D / PARTS;          // rows of P per part
+  __shared__ __align__(16) float Ps[D][kRotCols];
+  __shared__ float qs[G][D];
+  __shared__ float red[PARTS][G][kRotCols];
+  griddep_launch_dependents();
+  const int tid = threadIdx.x;
+  const int row = blockIdx.x / NB, cb = blockIdx.x - row * NB;
+  const int b = row / a.da.n_kv_heads, g = row - b * a.da.n_kv_heads;
+
+  // P_g[:, 32cb .. 32cb+32): eight float4 per row of P, all loads issued first
+  const float *Pg = a.da.P + (size_t)g * D * D + cb * kRotCols;
+  float4 pv[D / 32];
+#pragma unroll
+  for (int r = 0; r < D / 32; ++r) {
+    const int i = r * 32 + tid / 8;
+    pv[r] = __ldg(reinterpret_cast<const float4 *>(Pg + (size_t)i * D) + (tid % 8));
+  }
+  const int Hq = a.da.n_kv_heads * G;
+  const T *qg = a.da.q + ((size_t)b * Hq + (size_t)g * G) * D;
+  for (int e = tid; e < G * D; e += kThreads) qs[e / D][e % D] = to_f32(qg[e]);
+#pragma unroll
+  for (int r = 0; r < D / 32; ++r) reinterpret_cast<float4 *>(&Ps[r * 32 + tid / 8][0])[tid % 8] = pv[r];
+  __syncthreads();
+
+  const int j = tid % kRotCols, part = tid / kRotCols;
+  float acc[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 8
+  for (int i = part * RPP; i < (part + 1) * RPP; ++i) {
+    const float p = Ps[i][j];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = fmaf(qs[h][i], p, acc[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) red[part][h][j] = acc[h];
+  __syncthreads();
+
+  const int col = cb * kRotCols + j;
+  if (tid < G * kRotCols) {
+    const int h = tid / kRotCols;
+    float s = 0.f;
+#pragma unroll
+    for (int p = 0; p < PARTS; ++p) s += red[p][h][j];
+    a.qhat[((size_t)row * G + h) * D + col] = s * a.da.scale_log2;
+  }
+  if (tid < kRotCols) {
+    float s = 0.f;
+    if (col < a.da.d) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float t = 0.f;
+#pragma unroll
+        for (int p = 0; p < PARTS; ++p) t += red[p][h][j];
+        s += t;
+      }
+    }
+    a.u[(size_t)row * D + col] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode: shared-memory layout (4-byte words).  The select phase keeps its
+// histograms and candidate list in the ring (idle between the key stream and
+// the gather); the tensor-core query tiles reuse the first-digit histogram.
+struct FusedSmem {
+  int u, qhat, pm, pl, pacc, ctl, tbl, hist, ring, keys, words;
+};
+
+__host__ __device__ inline FusedSmem fused_smem(int G, int D, int chunk) {
+  FusedSmem L;
+  int o = 0;
+  L.u = o;    o += round4(D);
+  L.qhat = o; o += G * D;
+  L.pm = o;   o += 16;
+  L.pl = o;   o += 16;
+  L.pacc = o; o += G * D;
+  L.ctl = o;  o += 128;
+  L.tbl = o;  o += 2 * kMaxCluster;
+  L.hist = o; o += round4(kDig1Bins > 8 * D ? kDig1Bins : 8 * D);
+  L.ring = o; o += kRingWords;
+  L.keys = o; o += round4(chunk);
+  L.words = o;
+  return L;
+}
+
+// Skewed index of bin b in a shared-memory histogram: the consecutive bins a
+// thread scans fall into distinct banks across a warp.
+__host__ __device__ inline int hskew(int b) { return b + (b >> 5); }
+__host__ __device__ inline constexpr int skewed_words(int bins) { return bins + bins / 32; }
+
+// select buffers inside the ring (word offsets)
+constexpr int kRecv1 = 0;
+constexpr int kRecv2 = kRecv1 + skewed_words(1 << kDig1Bits);
+constexpr int kRecv3 = kRecv2 + skewed_words(1 << kDig2Bits);
+constexpr int kHloc = kRecv3 + skewed_words(1 << kDig3Bits);
+constexpr int kCand = kHloc + (1 << kDig2Bits);
+static_assert(kCand + kCandCap <= kRingWords, "select buffers must fit in the ring");
+
+// ctl words (write_selection uses 48..63)
+constexpr int kSelWtot = 0;     // [0..7] block-scan scratch
+constexpr int kSelBucket = 8;   // [8..10] bucket, count above it, count in it
+constexpr int kSelNcand = 12;
+
+// Among nb bins (skewed layout), find the one in which the count taken from
+// the top reaches `remaining` (1 <= remaining <= total).  Result in
+// ctl[kSelBucket..+2]: (bin, count in the bins above it, count in it).  Ends
+// with __syncthreads().
+__device__ __forceinline__ void find_bucket(const uint32_t *hist, int nb, uint32_t remaining, uint32_t *ctl) {
+  const int per = nb / kThreads;
+  const int lo = (int)threadIdx.x * per;
+  uint32_t mine = 0u;
+  for (int e = 0; e < per; ++e) mine += hist[hskew(lo + e)];
+  uint32_t above = block_excl_suffix_sum(mine, ctl + kSelWtot);
+  for (int e = per - 1; e >= 0; --e) {
+    const uint32_t c = hist[hskew(lo + e)];
+    if (above < remaining && above + c >= remaining) {
+      ctl[kSelBucket + 0] = (uint32_t)(lo + e);
+      ctl[kSelBucket + 1] = above;
+      ctl[kSelBucket + 2] = c;
+    }
+    above += c;
+  }
+  __syncthreads();
+}
+
+// Add the non-zero bins of this CTA's histogram (nb bins, plain layout) into
+// the skewed receive histogram of every CTA of the cluster.
+__device__ __forceinline__ void push_bins(cg::cluster_group &cluster, int ncta, const uint32_t *local, int nb,
+                                          uint32_t *recv) {
+  for (int e = threadIdx.x; e < nb; e += kThreads) {
+    const uint32_t c = local[e];
+    if (c)
+      for (int r = 0; r < ncta; ++r) atomicAdd(cluster.map_shared_rank(recv + hskew(e), r), c);
+  }
+}
+
+// Warp-inclusive scan of a 32-bit value.
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t t = __shfl_up_sync(kFull, v, off);
+    if (lane >= off) v += t;
+  }
+  return v;
+}
+
+// Keys of keys[0, len) with (key & mask) == prefix, appended to cand[] (order
+// not kept) while they fit in kCandCap; returns their count.  Four keys per
+// thread and step (keys is 16-byte aligned and padded to a multiple of 4).
+__device__ __forceinline__ int gather_candidates(const uint32_t *keys, int len, uint32_t prefix, uint32_t mask,
+                                                 uint32_t *cand, uint32_t *ctl) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid == 0) ctl[kSelNcand] = 0u;
+  __syncthreads();
+  const int n4 = (len + 3) >> 2;
+  for (int j40 = 0; j40 < n4; j40 += kThreads) {
+    const int j4 = j40 + tid;
+    uint32_t kk[4] = {0u, 0u, 0u, 0u};
+    uint32_t flags = 0u;
+    if (j4 < n4) {
+      const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+      kk[0] = v.x; kk[1] = v.y; kk[2] = v.z; kk[3] = v.w;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (4 * j4 + e < len && (kk[e] & mask) == prefix) flags |= 1u << e;
+    }
+    const uint32_t n = __popc(flags);
+    const uint32_t incl = warp_incl_scan(n);
+    uint32_t base = 0u;
+    if (lane == 31 && incl) base = atomicAdd(&ctl[kSelNcand], incl);
+    base = __shfl_sync(kFull, base, 31) + incl - n;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (flags & (1u << e)) {
+        if (base < (uint32_t)kCandCap) cand[base] = kk[e];
+        ++base;
+      }
+    }
+  }
+  __syncthreads();
+  return (int)ctl[kSelNcand];
+}
+
+// One cluster refinement pass: keys of set[0, n) with (key & mask) == prefix
+// add to bin (key >> shift) & (nb - 1); the cluster's sum lands in every CTA's
+// recv (zeroed before the cluster's first barrier) and each CTA finds the
+// bucket of rank `remaining` in it.
+__device__ __forceinline__ void refine_pass(cg::cluster_group &cluster, int ncta, const uint32_t *set, int n,
+                                            uint32_t prefix, uint32_t mask, int shift, int nb, uint32_t remaining,
+                                            uint32_t *hloc, uint32_t *recv, uint32_t *ctl) {
+  const int tid = threadIdx.x;
+  for (int e = tid; e < nb; e += kThreads) hloc[e] = 0u;
+  __syncthreads();
+  for (int i = tid; i < n; i += kThreads) {
+    const uint32_t key = set[i];
+    if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (uint32_t)(nb - 1)], 1u);
+  }
+  __syncthreads();
+  push_bins(cluster, ncta, hloc, nb, recv);
+  cluster.sync();
+  find_bucket(recv, nb, remaining, ctl);
+}
+
+// Write the CTA's selection, ascending: keys whose masked value is above
+// `prefix`, and the first `take` keys (in token order) whose masked value
+// equals it, from position `offset` of the row.  Warp w owns a contiguous
+// segment of the CTA's tokens (a multiple of 128); a counting sweep gives
+// each warp its offset, a second sweep compacts with warp scans, four keys
+// per lane and step.
+__device__ __forceinline__ void write_selection_vec(const uint32_t *keys, int len, int t0, const SelectState &st,
+                                                    uint32_t k, uint32_t *ctl, int32_t *idx_row) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (((len + kWarps - 1) / kWarps) + 127) & ~127;
+  const int sbeg = min(len, warp * seg), send = min(len, sbeg + seg);
+  uint32_t gt = 0u, eq = 0u;
+  for (int j0 = sbeg; j0 < send; j0 += 128) {
+    const int j = j0 + 4 * lane;
+    if (j < send) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(keys + j);
+      const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (j + e < send) {
+          const uint32_t km = kk[e] & st.mask;
+          gt += km > st.prefix;
+          eq += km == st.prefix;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    gt += __shfl_xor_sync(kFull, gt, off);
+    eq += __shfl_xor_sync(kFull, eq, off);
+  }
+  if (lane == 0) {
+    ctl[kCtlWarpGt + warp] = gt;
+    ctl[kCtlWarpEq + warp] = eq;
+  }
+  __syncthreads();
+  const uint32_t take = st.take;
+  uint32_t run_eq = 0u, run_sel = 0u;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t want = take > run_eq ? take - run_eq : 0u;
+    run_sel += ctl[kCtlWarpGt + w] + min(ctl[kCtlWarpEq + w], want);
+    run_eq += ctl[kCtlWarpEq + w];
+  }
+  int32_t *dst = idx_row + st.offset;
+  for (int j0 = sbeg; j0 < send; j0 += 128) {
+    const int j = j0 + 4 * lane;
+    uint32_t kk[4] = {0u, 0u, 0u, 0u};
+    if (j < send) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(keys + j);
+      kk[0] = v.x; kk[1] = v.y; kk[2] = v.z; kk[3] = v.w;
+    }
+    uint32_t ng = 0u, ne = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j + e < send) {
+        const uint32_t km = kk[e] & st.mask;
+        ng += km > st.prefix;
+        ne += km == st.prefix;
+      }
+    }
+    // warp scan of (ties << 16 | above): at most 128 of each per step
+    const uint32_t packed = (ne << 16) | ng;
+    const uint32_t incl = warp_incl_scan(packed);
+    const uint32_t excl = incl - packed;
+    const uint32_t tot = __shfl_sync(kFull, incl, 31);
+    uint32_t eq_rank = run_eq + (excl >> 16);  // tie rank of this lane's first tie in the CTA
+    uint32_t pos = run_sel + (excl & 0xffffu) + (min(take, eq_rank) - min(take, run_eq));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j + e < send) {
+        const uint32_t km = kk[e] & st.mask;
+        bool sel = km > st.prefix;
+        if (km == st.prefix) {
+          sel = eq_rank < take;
+          ++eq_rank;
+        }
+        if (sel) {
+          if (st.offset + pos < k) dst[pos] = t0 + j + e;  // bound: the row holds k entries
+          ++pos;
+        }
+      }
+    }
+    const uint32_t new_eq = run_eq + (tot >> 16);
+    run_sel += (tot & 0xffffu) + (min(take, new_eq) - min(take, run_eq));
+    run_eq = new_eq;
+  }
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel(const __grid_constant__ StepArgs<T> a) {
+  extern __shared__ __align__(16) uint32_t smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int ncta = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int row = blockIdx.x / ncta;
+  const int b = row / a.da.n_kv_heads, g = row - b * a.da.n_kv_heads;
+  const FusedSmem L = fused_smem(G, D, a.da.chunk);
+  float *u = reinterpret_cast<float *>(smem + L.u);
+  float *qhat = reinterpret_cast<float *>(smem + L.qhat);
+  float *pm = reinterpret_cast<float *>(smem + L.pm);
+  float *pl = reinterpret_cast<float *>(smem + L.pl);
+  float *pacc = reinterpret_cast<float *>(smem + L.pacc);
+  uint32_t *ctl = smem + L.ctl;
+  uint32_t *tbl = smem + L.tbl;
+  uint32_t *hist = smem + L.hist;
+  unsigned char *ring = reinterpret_cast<unsigned char *>(smem + L.ring);
+  uint32_t *rw = smem + L.ring;  // the ring as words, for the select buffers
+  uint32_t *keys = smem + L.keys;
+  const int tid = threadIdx.x;
+  const int S = a.da.seq_len;
+  const uint32_t k = (uint32_t)a.da.k;
+  const int t0 = min(S, rank * a.da.chunk);
+  const int len = min(S, t0 + a.da.chunk) - t0;
+  const size_t row_off = (size_t)row * a.da.capacity * D;
+  const T *Krow = a.da.k_hat + row_off;
+  const T *Vrow = a.da.v + row_off;
+  constexpr int MAXL = D / VecN<T>::value;
+
+  // 1. key stream: the first stages do not depend on the rotate grid
+  LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.da.nck, ring)));
+  for (int e = tid; e < kDig1Bins; e += kThreads) hist[e] = 0u;
+  griddep_wait();  // u and q_hat are written
+  for (int e = tid; e < D; e += kThreads) u[e] = __ldcg(a.u + (size_t)row * D + e);
+  for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
+  __syncthreads();
+  LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
+                    (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(Krow, t0, len, a.da.nck,
+                                                                                       ring, u, keys, hist)));
+
+  // 2. cluster radix select; the ring is idle until the gather
+  uint32_t *recv1 = rw + kRecv1, *recv2 = rw + kRecv2, *recv3 = rw + kRecv3;
+  uint32_t *hloc = rw + kHloc, *cand = rw + kCand;
+  for (int e = tid; e < kHloc; e += kThreads) rw[e] = 0u;  // recv1..recv3
+  cluster.sync();  // every CTA's receive histograms are zero
+  push_bins(cluster, ncta, hist, kDig1Bins, recv1);
+  cluster.sync();
+  find_bucket(recv1, kDig1Bins, k, ctl);
+  uint32_t remaining = k - ctl[kSelBucket + 1];
+  uint32_t prefix = ctl[kSelBucket + 0] << (32 - kDig1Bits);
+  uint32_t mask = ~0u << (32 - kDig1Bits);
+  if (ctl[kSelBucket + 2] != remaining) {  // uniform over the cluster
+    const int ncand = gather_candidates(keys, len, prefix, mask, cand, ctl);
+    const bool fits = ncand <= kCandCap;
+    const uint32_t *set = fits ? cand : keys;
+    const int nset = fits ? ncand : len;
+    constexpr int SH2 = 32 - kDig1Bits - kDig2Bits;
+    refine_pass(cluster, ncta, set, nset, prefix, mask, SH2, 1 << kDig2Bits, remaining, hloc, recv2, ctl);
+    remaining -= ctl[kSelBucket + 1];
+    prefix |= ctl[kSelBucket + 0] << SH2;
+    mask |= (uint32_t)((1 << kDig2Bits) - 1) << SH2;
+    if (ctl[kSelBucket + 2] != remaining) {  // uniform over the cluster
+      refine_pass(cluster, ncta, set, nset, prefix, mask, 0, 1 << kDig3Bits, remaining, hloc, recv3, ctl);
+      remaining -= ctl[kSelBucket + 1];
+      prefix |= ctl[kSelBucket + 0];
+      mask = ~0u;
+    }
+  }
+  // this CTA's counts above and at the threshold, into every CTA's table
+  uint32_t gt = 0u, eq = 0u;
+  for (int j4 = tid; j4 < (len + 3) >> 2; j4 += kThreads) {
+    const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (4 * j4 + e < len) {
+        const uint32_t km = kk[e] & mask;
+        gt += km > prefix;
+        eq += km == prefix;
+      }
+    }
+  }
+  gt = block_sum(gt, ctl + kSelWtot);
+  eq = block_sum(eq, ctl + kSelWtot);
+  if (tid < ncta) {
+    uint32_t *t = cluster.map_shared_rank(tbl, tid);
+    t[rank] = gt;
+    t[kMaxCluster + rank] = eq;
+  }
+  cluster.sync();
+  // ties at the threshold go to the lower index: lower CTAs first
+  uint32_t eq_before = 0u, offset = 0u;
+  for (int r = 0; r < rank; ++r) {
+    const uint32_t want = remaining > eq_before ? remaining - eq_before : 0u;
+    offset += tbl[r] + min(tbl[kMaxCluster + r], want);
+    eq_before += tbl[kMaxCluster + r];
+  }
+  const uint32_t take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
+  int32_t *idx_row = a.da.idx + (size_t)row * k;
+  write_selection_vec(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
+  cluster.sync();  // the whole row of idx is written and visible to the cluster
+
+  // 3. attention over this CTA's even share of the k selected rows; the
+  // indices are staged where the keys were (the share is at most chunk), and
+  // clamped into the row so that no load can leave the cache even if wrong
+  const int s0 = (int)(((long long)rank * k) / ncta);
+  const int s1 = (int)(((long long)(rank + 1) * k) / ncta);
+  int32_t *ids = reinterpret_cast<int32_t *>(keys);
+  for (int i = tid; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), S - 1);
+  __syncthreads();
+  attend_prologue_any<T, D, G, true>(Krow, Vrow, ids, 0, s1 - s0, ring);
+  attend_loop_any<T, D, G, true>(Krow, Vrow, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
+                                 pm, pl, pacc);
+
+  // 4. log-sum-exp merge of the cluster's states
+  cluster.sync();
+  const int Hq = a.da.n_kv_heads * G;
+  cluster_combine<D, G>(cluster, ncta, rank, pm, pl, pacc, a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
+  cluster.sync();
+}
+
+}  // namespace loki

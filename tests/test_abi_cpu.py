@@ -26,8 +26,9 @@ def lib():
 
 def test_header_declares_the_abi():
     names = _declared()
-    assert set(names) == {"loki_append", "loki_decode_attention", "dense_decode_attention",
-                          "loki_decode_launch_shape", "loki_status_string", "loki_last_error", "loki_version"}
+    assert set(names) == {"loki_append", "loki_decode_workspace_size", "loki_decode_attention",
+                          "dense_decode_attention", "loki_decode_launch_shape", "loki_status_string",
+                          "loki_last_error", "loki_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -48,7 +49,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 1
+    assert lib.loki_version() == 4
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -60,6 +61,8 @@ def _cache(dtype=1, B=1, H=2, D=128, cap=64, k=4096, v=8192):
 
 
 FAKE = 1 << 20   # aligned non-null address; never dereferenced because validation fails first
+WS = 1 << 24     # 256-byte aligned fake workspace address, with a size that passes the size check
+WSB = 1 << 40
 
 
 @pytest.mark.parametrize("cache_kw,seq,hq,d,k,status", [
@@ -79,20 +82,47 @@ FAKE = 1 << 20   # aligned non-null address; never dereferenced because validati
 ])
 def test_decode_validation(lib, cache_kw, seq, hq, d, k, status):
     c = _cache(**cache_kw)
-    r = lib.loki_decode_attention(ctypes.byref(c), seq, hq, FAKE, FAKE, d, k, 0.0, FAKE, FAKE, None)
+    r = lib.loki_decode_attention(ctypes.byref(c), seq, hq, FAKE, FAKE, d, k, 0.0, FAKE, FAKE, WS, WSB, None)
     assert r == status, lib.loki_last_error()
     assert lib.loki_last_error() != b""
 
 
 def test_decode_null_pointers(lib):
     c = _cache()
-    assert lib.loki_decode_attention(None, 10, 2, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE, None) == 1
+    assert lib.loki_decode_attention(None, 10, 2, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE, WS, WSB, None) == 1
     for args in [(None, FAKE, FAKE, FAKE), (FAKE, None, FAKE, FAKE), (FAKE, FAKE, None, FAKE), (FAKE, FAKE, FAKE, None)]:
         q, P, out, idx = args
-        assert lib.loki_decode_attention(ctypes.byref(c), 10, 2, q, P, 8, 4, 0.0, out, idx, None) == 1
-    assert lib.loki_decode_attention(ctypes.byref(c), 10, 2, FAKE + 8, FAKE, 8, 4, 0.0, FAKE, FAKE, None) == 1
+        assert lib.loki_decode_attention(ctypes.byref(c), 10, 2, q, P, 8, 4, 0.0, out, idx, WS, WSB, None) == 1
+    assert lib.loki_decode_attention(ctypes.byref(c), 10, 2, FAKE + 8, FAKE, 8, 4, 0.0, FAKE, FAKE, WS, WSB,
+                                     None) == 1
     assert lib.dense_decode_attention(ctypes.byref(c), 10, 2, None, FAKE, 0.0, FAKE, None) == 1
     assert lib.dense_decode_attention(ctypes.byref(c), 0, 2, FAKE, FAKE, 0.0, FAKE, None) == 1
+
+
+def _ws_bytes(rows, G, D):
+    """The workspace regions include/loki.h documents, each 256-byte aligned:
+    the rotated queries [rows, G, D] and the low-rank group queries [rows, D],
+    fp32."""
+    a = lambda x: (x + 255) // 256 * 256
+    return a(rows * G * D * 4) + a(rows * D * 4)
+
+
+def test_workspace_size_and_validation(lib):
+    c = _cache(B=3, H=2, cap=5000)
+    n = ctypes.c_size_t(0)
+    for S, hq in [(10, 2), (64, 4), (4999, 16), (5000, 2)]:
+        assert lib.loki_decode_workspace_size(ctypes.byref(c), S, hq, ctypes.byref(n)) == 0
+        assert n.value == _ws_bytes(6, hq // 2, 128)
+    assert lib.loki_decode_workspace_size(ctypes.byref(c), 5001, 2, ctypes.byref(n)) == 1
+    assert lib.loki_decode_workspace_size(ctypes.byref(c), 0, 2, ctypes.byref(n)) == 1
+    assert lib.loki_decode_workspace_size(ctypes.byref(c), 10, 3, ctypes.byref(n)) == 1
+    assert lib.loki_decode_workspace_size(ctypes.byref(c), 10, 2, None) == 1
+    need = _ws_bytes(6, 1, 128)
+    args = (ctypes.byref(c), 10, 2, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE)
+    assert lib.loki_decode_attention(*args, None, WSB, None) == 1          # no workspace
+    assert lib.loki_decode_attention(*args, WS + 16, WSB, None) == 1       # not 256-byte aligned
+    assert lib.loki_decode_attention(*args, WS, need - 1, None) == 1       # too small
+    assert b"smaller" in lib.loki_last_error()
 
 
 @pytest.mark.parametrize("pos,n_new,status", [(-1, 1, 1), (0, 0, 1), (60, 5, 1), (64, 1, 1)])

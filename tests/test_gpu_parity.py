@@ -206,6 +206,51 @@ def test_full_budget_equals_dense():
     assert np.all(idx == np.arange(700))
 
 
+# ----------------------------------------------------------------------------- workspace and score tiles
+def test_workspace_needs_no_initialisation_and_is_shared_across_shapes():
+    # one external workspace, filled with garbage first, shared by calls of
+    # different caches, lengths, d and k: every call must match the oracle
+    lib = L()
+    ws = torch.randint(0, 256, (32 << 20,), dtype=torch.uint8, device=DEV)
+    cases = [("bf16", 128, 4, 3001, 64, 375, 2, 2), ("bf16", 128, 1, 5000, 32, 1250, 4, 3),
+             ("f32", 64, 2, 700, 16, 99, 1, 2), ("bf16", 128, 4, 3001, 8, 2999, 2, 2),
+             ("bf16", 128, 8, 40000, 32, 5000, 1, 1)]
+    for dtype, D, G, S, d, k, Hkv, B in cases:
+        w = small_workload(dtype, D, G, S, Hkv=Hkv, B=B, seed=S + d)
+        inp = gen.decode_inputs(w, seq_len=S)
+        P32 = basis(w)
+        cache, K_hat, V, q, P = upload_case(w, inp, P32)
+        assert lib.loki_decode_workspace_size(cache, S, w.n_q_heads) <= ws.numel()
+        out, idx = lib.loki_decode_attention(cache, S, q, P, d, k, workspace=ws)
+        torch.cuda.synchronize()
+        ref = oracle.loki_decode(inp["q64"], K_hat, V, P32.astype(np.float64), S, d, k)
+        parity.check_decode(out.cpu().numpy(), idx.cpu().numpy(), ref, ref["q_hat"], K_hat, V,
+                            oracle.default_scale(D), dtype)
+
+
+@pytest.mark.parametrize("S,B,Hkv,G", [(20000, 1, 2, 1), (4096, 16, 8, 4), (257, 3, 2, 2), (70001, 1, 1, 4)])
+def test_cluster_shapes_and_ragged_chunks(S, B, Hkv, G):
+    # rows split over clusters of several CTAs with a ragged last chunk, grids
+    # of several waves, and a row longer than one CTA can hold
+    w = small_workload("bf16", 128, G, S, Hkv=Hkv, B=B, seed=S)
+    rot, ncta, ctas, zero = L().loki_decode_launch_shape(
+        L().LokiCache(B, Hkv, 128, S, dtype=torch.bfloat16, device=DEV), S, Hkv * G, max(1, S // 8))
+    assert rot == B * Hkv * 4 and ctas == B * Hkv * ncta and zero == 0
+    assert ncta in (1, 2, 4, 8, 16) and ncta * 24576 >= S
+    out, idx, ref, K_hat, V, *_ = run_decode(w, S, 32, max(1, S // 8))
+    parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(128), "bf16")
+
+
+def test_repeated_calls_are_identical():
+    w = small_workload("bf16", 128, 4, 3001)
+    out, idx, ref, K_hat, V, inp, P32, cache, q, P = run_decode(w, 3001, 64, 375)
+    for _ in range(3):
+        o2, i2 = L().loki_decode_attention(cache, 3001, q, P, 64, 375)
+        torch.cuda.synchronize()
+        assert np.array_equal(i2.cpu().numpy(), idx)
+        assert np.array_equal(o2.cpu().numpy(), out)
+
+
 # ----------------------------------------------------------------------------- dense, small shapes
 @pytest.mark.parametrize("ncta", [None, 1, 16])
 @pytest.mark.parametrize("dtype,D,G,S", [

@@ -132,6 +132,28 @@ LOKI_API loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_
                                   int32_t *idx, void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* loki_decode_attention_noalloc -- loki_decode_attention without a caller
+ * workspace, for callers that cannot allocate device memory on the decode
+ * path: for example a host runtime whose device memory plan is fixed at
+ * start-up, or one for which the implicit device synchronisation of
+ * cudaMalloc is not acceptable between decode steps.  The pages have no
+ * counterpart; this is an interface convenience of this library.
+ * Arguments and results are those of loki_decode_attention, minus the
+ * workspace.  The scratch is instead a fixed 4 MiB array in the library's
+ * device code, which every GPU that loads the library holds until the process
+ * exits; the call allocates and frees nothing.  A call whose
+ * loki_decode_workspace_size exceeds 4 MiB returns LOKI_ERR_UNSUPPORTED with a
+ * message, and enqueues nothing.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Every call on a device
+ * shares the one array and leaves its contents behind (nothing in it needs to
+ * start at zero): calls that may overlap on the GPU, from other streams or
+ * threads, race on it and must not be issued. */
+LOKI_API loki_status loki_decode_attention_noalloc(const loki_cache *cache, int32_t seq_len,
+                                          int32_t n_q_heads, const void *q, const float *P,
+                                          int32_t d, int32_t k, float scale, float *out,
+                                          int32_t *idx, void *stream);
+
 /* dense_decode_attention -- full softmax attention over every token
  * [0, seq_len) of the same rotated cache: the "Full Attention" baseline of the
  * summary page, section "Experimental setup".  Arguments as above; q is rotated

@@ -13,6 +13,7 @@ from .api import (
     dense_decode_attention,
     loki_append,
     loki_decode_attention,
+    loki_decode_attention_noalloc,
     loki_decode_launch_shape,
     loki_decode_workspace_size,
     loki_status_string,
@@ -27,6 +28,7 @@ __all__ = [
     "LokiCache",
     "loki_append",
     "loki_decode_attention",
+    "loki_decode_attention_noalloc",
     "dense_decode_attention",
     "loki_decode_launch_shape",
     "loki_decode_workspace_size",

@@ -125,6 +125,30 @@ def loki_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: to
     return out, idx
 
 
+def loki_decode_attention_noalloc(cache: LokiCache, seq_len: int, q: torch.Tensor, P: torch.Tensor, d: int, k: int,
+                                  scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                  idx: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """loki_decode_attention on the library's fixed device scratch instead of
+    a workspace, for callers that cannot allocate device memory on the decode
+    path.  Calls on one device share that scratch: they must not overlap on
+    the GPU.  Shapes beyond its 4 MiB raise LokiError (unsupported)."""
+    B, Hq, D = q.shape if q.dim() == 3 else (-1, -1, -1)
+    _need(q, "q", cache.dtype, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    if out is None:
+        out = torch.empty((cache.batch, Hq, cache.head_dim), dtype=torch.float32, device=cache.device)
+    if idx is None:
+        idx = torch.empty((cache.batch, cache.n_kv_heads, int(k)), dtype=torch.int32, device=cache.device)
+    _need(out, "out", torch.float32, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(idx, "idx", torch.int32, (cache.batch, cache.n_kv_heads, int(k)), cache.device)
+    with torch.cuda.device(cache.device):
+        _lib.check(_lib.load().loki_decode_attention_noalloc(cache.desc(), int(seq_len), int(Hq), _ptr(q), _ptr(P),
+                                                             int(d), int(k), float(scale), _ptr(out), _ptr(idx),
+                                                             _stream_ptr(cache.device, stream)))
+    return out, idx
+
+
 def dense_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: torch.Tensor, scale: float = 0.0,
                            out: Optional[torch.Tensor] = None,
                            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:

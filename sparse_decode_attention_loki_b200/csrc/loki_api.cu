@@ -475,6 +475,37 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   return LOKI_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch of loki_decode_attention_noalloc: a file-scope device array
+// that every device loading this library holds until the process exits.  In
+// host code its name is only a host-side stand-in; the device address comes
+// from cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+std::atomic<int> g_noalloc_ready[kMaxDevices];
+void *g_noalloc_addr[kMaxDevices];
+
+loki_status noalloc_scratch(void **addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LOKI_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+  if (!g_noalloc_ready[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ready[dev].load(std::memory_order_relaxed)) {
+      void *p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+      g_noalloc_addr[dev] = p;
+      g_noalloc_ready[dev].store(1, std::memory_order_release);
+    }
+  }
+  *addr = g_noalloc_addr[dev];
+  return LOKI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -530,6 +561,24 @@ loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len, int3
   if (cache->dtype == LOKI_F32)
     return decode_common<float>(cache, sh, false, q, P, d, k, scale, out, idx, workspace, stream);
   return decode_common<__nv_bfloat16>(cache, sh, false, q, P, d, k, scale, out, idx, workspace, stream);
+}
+
+loki_status loki_decode_attention_noalloc(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads,
+                                          const void *q, const float *P, int32_t d, int32_t k, float scale,
+                                          float *out, int32_t *idx, void *stream) {
+  size_t need = 0;
+  loki_status s = loki_decode_workspace_size(cache, seq_len, n_q_heads, &need);
+  if (s != LOKI_OK) return s;
+  if (need > kNoAllocScratchBytes)
+    return fail(LOKI_ERR_UNSUPPORTED,
+                "this call needs %zu bytes of scratch; the fixed scratch of loki_decode_attention_noalloc holds "
+                "%zu (use loki_decode_attention with a workspace)",
+                need, kNoAllocScratchBytes);
+  void *scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != LOKI_OK) return s;
+  return loki_decode_attention(cache, seq_len, n_q_heads, q, P, d, k, scale, out, idx, scratch,
+                               kNoAllocScratchBytes, stream);
 }
 
 loki_status dense_decode_attention(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, const void *q,

@@ -27,8 +27,8 @@ def lib():
 def test_header_declares_the_abi():
     names = _declared()
     assert set(names) == {"loki_append", "loki_decode_workspace_size", "loki_decode_attention",
-                          "dense_decode_attention", "loki_decode_launch_shape", "loki_status_string",
-                          "loki_last_error", "loki_version"}
+                          "loki_decode_attention_noalloc", "dense_decode_attention", "loki_decode_launch_shape",
+                          "loki_status_string", "loki_last_error", "loki_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):

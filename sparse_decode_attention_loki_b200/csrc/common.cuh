@@ -154,6 +154,27 @@ __device__ __forceinline__ void st_cg16(void *p, const uint4 &v) {
                : "memory");
 }
 
+// Distributed shared memory: the shared::cluster address of `local` (this
+// CTA's shared memory) in CTA `rank` of the cluster, and accesses through it.
+__device__ __forceinline__ uint32_t dsmem_addr(const void *local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"((uint32_t)__cvta_generic_to_shared(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void dsmem_red_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void dsmem_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // Split cluster barrier (arrive with release, wait with acquire).  Every thread
 // of every CTA in the cluster must execute each of them the same number of times.
 __device__ __forceinline__ void cluster_arrive() {

@@ -765,24 +765,48 @@ __device__ __forceinline__ void attend_loop_any(const T *Kb, const T *Vb, const 
 }
 
 // ---------------------------------------------------------------------------
-// 6. log-sum-exp combine of the cluster's partial states; CTA r writes the
-//    output elements r*256 + t (stride ncta*256).  Must follow a cluster
-//    barrier that orders every CTA's pm/pl/pacc writes.
+// 6. log-sum-exp combine of the cluster's partial states.  The ncta x G
+//    weights exp2(m_r,h - M_h) / L_h are formed once (scratch: 3*ncta*G + 2*G
+//    floats of this CTA's shared memory that nothing else uses now); then CTA r
+//    writes the output elements r*256 + t (stride ncta*256) as weighted sums
+//    of the CTAs' accumulators.  Must follow a cluster barrier that orders
+//    every CTA's pm/pl/pacc writes, and be followed by one before any CTA exits.
 template <int D, int G>
-__device__ __forceinline__ void cluster_combine(cg::cluster_group &cluster, int ncta, int rank,
-                                                const float *pm, const float *pl, const float *pacc,
-                                                float *out) {
-  for (int e = rank * kThreads + (int)threadIdx.x; e < G * D; e += ncta * kThreads) {
-    const int h = e / D;
+__device__ __forceinline__ void cluster_combine(int ncta, int rank, const float *pm, const float *pl,
+                                                const float *pacc, float *scratch, float *out) {
+  const int tid = threadIdx.x;
+  float *cm = scratch;               // [ncta][G] maxima, then weights
+  float *cl = cm + ncta * G;         // [ncta][G] sums
+  float *mh = cl + ncta * G;         // [G]
+  float *lh = mh + G;                // [G]
+  for (int e = tid; e < ncta * G; e += kThreads) {
+    const int r = e / G, h = e - r * G;
+    cm[e] = dsmem_ld_f32(dsmem_addr(pm + h, (uint32_t)r));
+    cl[e] = dsmem_ld_f32(dsmem_addr(pl + h, (uint32_t)r));
+  }
+  __syncthreads();
+  if (tid < G) {
     float M = -INFINITY;
-    for (int r = 0; r < ncta; ++r) M = fmaxf(M, *cluster.map_shared_rank(pm + h, r));
-    float A = 0.f, Ls = 0.f;
-    for (int r = 0; r < ncta; ++r) {
-      const float c = exp2f(*cluster.map_shared_rank(pm + h, r) - M);
-      A = fmaf(c, *cluster.map_shared_rank(pacc + e, r), A);
-      Ls = fmaf(c, *cluster.map_shared_rank(pl + h, r), Ls);
-    }
-    out[e] = A / Ls;
+    for (int r = 0; r < ncta; ++r) M = fmaxf(M, cm[r * G + tid]);
+    const float mref = (M == -INFINITY) ? 0.f : M;
+    float Ls = 0.f;
+    for (int r = 0; r < ncta; ++r) Ls = fmaf(exp2f(cm[r * G + tid] - mref), cl[r * G + tid], Ls);
+    mh[tid] = mref;
+    lh[tid] = Ls;
+  }
+  __syncthreads();
+  for (int e = tid; e < ncta * G; e += kThreads) cm[e] = exp2f(cm[e] - mh[e % G]) / lh[e % G];
+  __syncthreads();
+  for (int e = rank * kThreads + tid; e < G * D; e += ncta * kThreads) {
+    const int h = e / D;
+    float v[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) v[r] = r < ncta ? dsmem_ld_f32(dsmem_addr(pacc + e, (uint32_t)r)) : 0.f;
+    float A = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      if (r < ncta) A = fmaf(cm[r * G + h], v[r], A);
+    out[e] = A;
   }
 }
 
@@ -813,7 +837,8 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kerne
                                   reinterpret_cast<unsigned char *>(scratch), ring, pm, pl, pacc);
   cluster.sync();
   const int Hq = a.n_kv_heads * G;
-  cluster_combine<D, G>(cluster, ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);
+  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, reinterpret_cast<float *>(ring),
+                        a.out + ((size_t)b * Hq + (size_t)g * G) * D);
   cluster.sync();
 }
 

@@ -9,10 +9,10 @@
 //   decode  one thread-block cluster of ncta CTAs per row, about one wave of
 //           CTAs in all; CTA r owns tokens [r*chunk, (r+1)*chunk):
 //     1. the first stages of its low-rank key stream go in flight (cp.async
-//        ring) before it waits for the rotate grid (programmatic dependent
-//        launch), then it streams K_hat[i, :d], keeps one order-preserving
-//        uint32 key per token in shared memory and histograms the keys' top
-//        11 bits on the way;
+//        ring) while it forms u from q and P_g[:, :d] itself, then it
+//        streams K_hat[i, :d], keeps one order-preserving uint32 key per
+//        token in shared memory and histograms the keys' top 11 bits on the
+//        way;
 //     2. cluster radix select over 11/11/10-bit digits: each CTA adds the
 //        non-zero bins of its histogram into every CTA of the cluster through
 //        distributed shared memory, so after one cluster barrier every CTA
@@ -20,7 +20,8 @@
 //        (the candidates) are refined the same way; the CTAs then exchange
 //        their counts above and at the threshold and write their indices in
 //        ascending order, ties at the threshold going to the lower index;
-//     3. the k selected rows are split evenly over the cluster: gather K_hat
+//     3. (only now waiting for the rotate grid, a programmatic dependency)
+//        the k selected rows are split evenly over the cluster: gather K_hat
 //        and V rows through the ring, online softmax per query head;
 //     4. the CTAs' (max, sum, acc) states are merged through distributed
 //        shared memory with the log-sum-exp rule into out.
@@ -199,13 +200,19 @@ __device__ __forceinline__ void find_bucket(const uint32_t *hist, int nb, uint32
 }
 
 // Add the non-zero bins of this CTA's histogram (nb bins, plain layout) into
-// the skewed receive histogram of every CTA of the cluster.
-__device__ __forceinline__ void push_bins(cg::cluster_group &cluster, int ncta, const uint32_t *local, int nb,
-                                          uint32_t *recv) {
+// the skewed receive histogram of every CTA of the cluster (DSMEM reductions).
+__device__ __forceinline__ void push_bins(int ncta, const uint32_t *local, int nb, uint32_t *recv) {
+  uint32_t base[kMaxCluster];
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) base[r] = r < ncta ? dsmem_addr(recv, (uint32_t)r) : 0u;
   for (int e = threadIdx.x; e < nb; e += kThreads) {
     const uint32_t c = local[e];
-    if (c)
-      for (int r = 0; r < ncta; ++r) atomicAdd(cluster.map_shared_rank(recv + hskew(e), r), c);
+    if (c) {
+      const uint32_t off = 4u * (uint32_t)hskew(e);
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r)
+        if (r < ncta) dsmem_red_add(base[r] + off, c);
+    }
   }
 }
 
@@ -220,41 +227,39 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   return v;
 }
 
-// Keys of keys[0, len) with (key & mask) == prefix, appended to cand[] (order
-// not kept) while they fit in kCandCap; returns their count.  Four keys per
-// thread and step (keys is 16-byte aligned and padded to a multiple of 4).
+// Keys of keys[0, len) with (key & mask) == prefix, copied to cand[] while
+// they fit in kCandCap (in no particular order); returns their count.  A
+// counting sweep and a block scan give each thread its output offset, a second
+// sweep writes; four keys per thread and step (keys is 16-byte aligned and
+// padded to a multiple of 4).
 __device__ __forceinline__ int gather_candidates(const uint32_t *keys, int len, uint32_t prefix, uint32_t mask,
                                                  uint32_t *cand, uint32_t *ctl) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  if (tid == 0) ctl[kSelNcand] = 0u;
-  __syncthreads();
+  const int tid = threadIdx.x;
   const int n4 = (len + 3) >> 2;
-  for (int j40 = 0; j40 < n4; j40 += kThreads) {
-    const int j4 = j40 + tid;
-    uint32_t kk[4] = {0u, 0u, 0u, 0u};
-    uint32_t flags = 0u;
-    if (j4 < n4) {
-      const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
-      kk[0] = v.x; kk[1] = v.y; kk[2] = v.z; kk[3] = v.w;
+  uint32_t mine = 0u;
+  for (int j4 = tid; j4 < n4; j4 += kThreads) {
+    const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (4 * j4 + e < len && (kk[e] & mask) == prefix) flags |= 1u << e;
-    }
-    const uint32_t n = __popc(flags);
-    const uint32_t incl = warp_incl_scan(n);
-    uint32_t base = 0u;
-    if (lane == 31 && incl) base = atomicAdd(&ctl[kSelNcand], incl);
-    base = __shfl_sync(kFull, base, 31) + incl - n;
+    for (int e = 0; e < 4; ++e) mine += (4 * j4 + e < len && (kk[e] & mask) == prefix) ? 1u : 0u;
+  }
+  // exclusive prefix over threads: total after thread t = suffix sum of the rest
+  const uint32_t after = block_excl_suffix_sum(mine, ctl + kSelWtot);
+  const uint32_t total = block_sum(mine, ctl + kSelWtot);
+  uint32_t pos = total - after - mine;
+  for (int j4 = tid; j4 < n4; j4 += kThreads) {
+    const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (flags & (1u << e)) {
-        if (base < (uint32_t)kCandCap) cand[base] = kk[e];
-        ++base;
+      if (4 * j4 + e < len && (kk[e] & mask) == prefix) {
+        if (pos < (uint32_t)kCandCap) cand[pos] = kk[e];
+        ++pos;
       }
     }
   }
   __syncthreads();
-  return (int)ctl[kSelNcand];
+  return (int)total;
 }
 
 // One cluster refinement pass: keys of set[0, n) with (key & mask) == prefix
@@ -272,7 +277,7 @@ __device__ __forceinline__ void refine_pass(cg::cluster_group &cluster, int ncta
     if ((key & mask) == prefix) atomicAdd(&hloc[(key >> shift) & (uint32_t)(nb - 1)], 1u);
   }
   __syncthreads();
-  push_bins(cluster, ncta, hloc, nb, recv);
+  push_bins(ncta, hloc, nb, recv);
   cluster.sync();
   find_bucket(recv, nb, remaining, ctl);
 }
@@ -366,6 +371,67 @@ __device__ __forceinline__ void write_selection_vec(const uint32_t *keys, int le
   }
 }
 
+// u[j] = sum_i qs[i] * P_g[i][j] for j < d (zero beyond), qs = the sum of the
+// G queries of the row (fp32): by linearity equal to sum_h q_hat_h[:d].
+// Its loads of P and q are issued first; `after_loads()` runs while they are
+// in flight.  Thread (c4 = tid % C4P, part = tid / C4P) holds the float4 of columns
+// [4c4, 4c4+4) of the rows of its part (C4P = ceil(d/4) rounded up to a
+// power of two); all its loads of P are issued before the first use, then the
+// parts are added in a fixed order in shared memory.  qs: D floats, red:
+// 4*kThreads floats of scratch.  Ends with __syncthreads().
+template <typename T, int D, int G, typename F>
+__device__ __forceinline__ void lowrank_query(const DecodeArgs<T> &a, int b, int g, float *qs, float *red, float *u,
+                                              F &&after_loads) {
+  constexpr int RMAX = D / 8;  // rows per part when C4P = 32 (the most)
+  const int tid = threadIdx.x;
+  const int c4n = (a.d + 3) >> 2;
+  int C4P = 1;
+  while (C4P < c4n) C4P <<= 1;
+  const int parts = kThreads / C4P;                 // >= 8
+  const int rpp = parts >= D ? 1 : D / parts;       // rows per part, <= RMAX
+  const int c4 = tid % C4P, part = tid / C4P;
+  const bool active = c4 < c4n && part * rpp < D;  // parts beyond D rows stay idle
+  const float *Pg = a.P + (size_t)g * D * D + 4 * c4;
+  float4 pv[RMAX];
+#pragma unroll
+  for (int x = 0; x < RMAX; ++x)
+    pv[x] = (active && x < rpp) ? __ldg(reinterpret_cast<const float4 *>(Pg + (size_t)(part * rpp + x) * D))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+  const T *qg = a.q + ((size_t)b * a.n_kv_heads * G + (size_t)g * G) * D;
+  float qv[G];
+  const int iq = tid < D ? tid : 0;
+#pragma unroll
+  for (int h = 0; h < G; ++h) qv[h] = to_f32(qg[(size_t)h * D + iq]);
+  after_loads();  // the caller's own loads go in flight behind these
+  if (tid < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) s += qv[h];
+    qs[tid] = s;
+  }
+  __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int x = 0; x < RMAX; ++x) {
+    if (active && x < rpp) {
+      const float qv = qs[part * rpp + x];
+      acc.x = fmaf(qv, pv[x].x, acc.x);
+      acc.y = fmaf(qv, pv[x].y, acc.y);
+      acc.z = fmaf(qv, pv[x].z, acc.z);
+      acc.w = fmaf(qv, pv[x].w, acc.w);
+    }
+  }
+  reinterpret_cast<float4 *>(red)[tid] = acc;  // red[(part * C4P + c4) * 4 + y]
+  __syncthreads();
+  for (int jj = tid; jj < D; jj += kThreads) {
+    float s = 0.f;
+    if (jj < a.d)
+      for (int p = 0; p < parts && p * rpp < D; ++p) s += red[(p * C4P + (jj >> 2)) * 4 + (jj & 3)];
+    u[jj] = s;
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel(const __grid_constant__ StepArgs<T> a) {
@@ -397,12 +463,12 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   const T *Vrow = a.da.v + row_off;
   constexpr int MAXL = D / VecN<T>::value;
 
-  // 1. key stream: the first stages do not depend on the rotate grid
-  LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.da.nck, ring)));
+  // 1. key stream; the low-rank group query is formed while its first stages
+  // are in flight (neither depends on the rotate grid)
+  lowrank_query<T, D, G>(a.da, b, g, qhat, reinterpret_cast<float *>(hist), u, [&] {
+    LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.da.nck, ring)));
+  });
   for (int e = tid; e < kDig1Bins; e += kThreads) hist[e] = 0u;
-  griddep_wait();  // u and q_hat are written
-  for (int e = tid; e < D; e += kThreads) u[e] = __ldcg(a.u + (size_t)row * D + e);
-  for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
   __syncthreads();
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
                     (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(Krow, t0, len, a.da.nck,
@@ -413,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   uint32_t *hloc = rw + kHloc, *cand = rw + kCand;
   for (int e = tid; e < kHloc; e += kThreads) rw[e] = 0u;  // recv1..recv3
   cluster.sync();  // every CTA's receive histograms are zero
-  push_bins(cluster, ncta, hist, kDig1Bins, recv1);
+  push_bins(ncta, hist, kDig1Bins, recv1);
   cluster.sync();
   find_bucket(recv1, kDig1Bins, k, ctl);
   uint32_t remaining = k - ctl[kSelBucket + 1];
@@ -453,9 +519,8 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   gt = block_sum(gt, ctl + kSelWtot);
   eq = block_sum(eq, ctl + kSelWtot);
   if (tid < ncta) {
-    uint32_t *t = cluster.map_shared_rank(tbl, tid);
-    t[rank] = gt;
-    t[kMaxCluster + rank] = eq;
+    dsmem_st(dsmem_addr(tbl + rank, (uint32_t)tid), gt);
+    dsmem_st(dsmem_addr(tbl + kMaxCluster + rank, (uint32_t)tid), eq);
   }
   cluster.sync();
   // ties at the threshold go to the lower index: lower CTAs first
@@ -470,6 +535,8 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   write_selection_vec(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
   cluster.sync();  // the whole row of idx is written and visible to the cluster
 
+  griddep_wait();  // q_hat is written
+  for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
   // 3. attention over this CTA's even share of the k selected rows; the
   // indices are staged where the keys were (the share is at most chunk), and
   // clamped into the row so that no load can leave the cache even if wrong
@@ -485,7 +552,8 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   // 4. log-sum-exp merge of the cluster's states
   cluster.sync();
   const int Hq = a.da.n_kv_heads * G;
-  cluster_combine<D, G>(cluster, ncta, rank, pm, pl, pacc, a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
+  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, reinterpret_cast<float *>(ring),
+                        a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
   cluster.sync();
 }
 

@@ -765,48 +765,39 @@ __device__ __forceinline__ void attend_loop_any(const T *Kb, const T *Vb, const 
 }
 
 // ---------------------------------------------------------------------------
-// 6. log-sum-exp combine of the cluster's partial states.  The ncta x G
-//    weights exp2(m_r,h - M_h) / L_h are formed once (scratch: 3*ncta*G + 2*G
-//    floats of this CTA's shared memory that nothing else uses now); then CTA r
-//    writes the output elements r*256 + t (stride ncta*256) as weighted sums
-//    of the CTAs' accumulators.  Must follow a cluster barrier that orders
-//    every CTA's pm/pl/pacc writes, and be followed by one before any CTA exits.
+// 6. log-sum-exp combine of the cluster's partial states: CTA r writes the
+//    output elements r*256 + t (stride ncta*256); each reads the (max, sum,
+//    acc) of its head from every CTA through distributed shared memory, all
+//    loads issued before the first use.  Must follow a cluster barrier that
+//    orders every CTA's pm/pl/pacc writes, and be followed by one before any
+//    CTA exits.
 template <int D, int G>
 __device__ __forceinline__ void cluster_combine(int ncta, int rank, const float *pm, const float *pl,
-                                                const float *pacc, float *scratch, float *out) {
-  const int tid = threadIdx.x;
-  float *cm = scratch;               // [ncta][G] maxima, then weights
-  float *cl = cm + ncta * G;         // [ncta][G] sums
-  float *mh = cl + ncta * G;         // [G]
-  float *lh = mh + G;                // [G]
-  for (int e = tid; e < ncta * G; e += kThreads) {
-    const int r = e / G, h = e - r * G;
-    cm[e] = dsmem_ld_f32(dsmem_addr(pm + h, (uint32_t)r));
-    cl[e] = dsmem_ld_f32(dsmem_addr(pl + h, (uint32_t)r));
-  }
-  __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int r = 0; r < ncta; ++r) M = fmaxf(M, cm[r * G + tid]);
-    const float mref = (M == -INFINITY) ? 0.f : M;
-    float Ls = 0.f;
-    for (int r = 0; r < ncta; ++r) Ls = fmaf(exp2f(cm[r * G + tid] - mref), cl[r * G + tid], Ls);
-    mh[tid] = mref;
-    lh[tid] = Ls;
-  }
-  __syncthreads();
-  for (int e = tid; e < ncta * G; e += kThreads) cm[e] = exp2f(cm[e] - mh[e % G]) / lh[e % G];
-  __syncthreads();
-  for (int e = rank * kThreads + tid; e < G * D; e += ncta * kThreads) {
+                                                const float *pacc, float *out) {
+  constexpr int R = 16;  // the largest cluster
+  for (int e = rank * kThreads + (int)threadIdx.x; e < G * D; e += ncta * kThreads) {
     const int h = e / D;
-    float v[16];
+    float m[R], l[R], v[R];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) v[r] = r < ncta ? dsmem_ld_f32(dsmem_addr(pacc + e, (uint32_t)r)) : 0.f;
-    float A = 0.f;
+    for (int r = 0; r < R; ++r) {
+      m[r] = r < ncta ? dsmem_ld_f32(dsmem_addr(pm + h, (uint32_t)r)) : -INFINITY;
+      l[r] = r < ncta ? dsmem_ld_f32(dsmem_addr(pl + h, (uint32_t)r)) : 0.f;
+      v[r] = r < ncta ? dsmem_ld_f32(dsmem_addr(pacc + e, (uint32_t)r)) : 0.f;
+    }
+    float M = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < ncta) A = fmaf(cm[r * G + h], v[r], A);
-    out[e] = A;
+    for (int r = 0; r < R; ++r) M = fmaxf(M, m[r]);
+    const float mref = (M == -INFINITY) ? 0.f : M;
+    float A = 0.f, Ls = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r < ncta) {
+        const float c = exp2f(m[r] - mref);
+        A = fmaf(c, v[r], A);
+        Ls = fmaf(c, l[r], Ls);
+      }
+    }
+    out[e] = A / Ls;
   }
 }
 
@@ -837,8 +828,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kerne
                                   reinterpret_cast<unsigned char *>(scratch), ring, pm, pl, pacc);
   cluster.sync();
   const int Hq = a.n_kv_heads * G;
-  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, reinterpret_cast<float *>(ring),
-                        a.out + ((size_t)b * Hq + (size_t)g * G) * D);
+  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);
   cluster.sync();
 }
 

@@ -304,10 +304,14 @@ struct StepPlan {
   int ncta, chunk, smem;
 };
 
-// CTAs per row (cluster size) of the decode kernel: the largest power of two
-// up to 16 that keeps the grid within one wave of co-resident CTAs, but never
-// fewer than the share of kMaxChunk tokens per CTA needs, and only sizes the
-// device can schedule.  LOKI_CLUSTER (a tuning override) forces the size.
+// CTAs per row (cluster size) of the decode kernel.  Start from the fewest
+// CTAs whose share is at most kTargetChunk tokens (two CTAs then fit on an SM;
+// more only when a share would exceed kMaxChunk), and take the first power of
+// two up to 16 whose grid covers at least 80% of the device's co-resident
+// CTAs, else the largest schedulable one: fewer, longer CTAs spend less on
+// the cross-CTA steps.  LOKI_CLUSTER (a tuning override) forces the size.
+constexpr int kTargetChunk = 8192;
+
 template <typename Kern>
 loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepPlan *p) {
   const long long rows = (long long)sh.B * sh.Hkv;
@@ -315,20 +319,23 @@ loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepP
   int dev = 0;
   cudaGetDevice(&dev);
   int need = 1;
-  while (need < kMaxCluster && (S + need - 1) / need > kMaxChunk) need *= 2;
-  if ((S + need - 1) / need > kMaxChunk)
+  while (need < kMaxCluster && (S + need - 1) / need > kTargetChunk) need *= 2;
+  while (need > 1 && (S + need - 1) / need > kMaxChunk) need *= 2;
+  if ((S + kMaxCluster - 1) / kMaxCluster > kMaxChunk)
     return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d exceeds %d tokens", S, kMaxChunk * kMaxCluster);
+  if (need > kMaxCluster) need = kMaxCluster;
   const int forced = env_int("LOKI_CLUSTER", 0);
   StepPlan best{0, 0, 0};
-  for (int n = kMaxCluster; n >= need; n /= 2) {
-    if (forced && n != forced) continue;
+  for (int n = 1; n <= kMaxCluster; n *= 2) {
+    if (forced ? n != forced : n < need) continue;
     const int chunk = round4((S + n - 1) / n);
+    if (chunk > kMaxChunk) continue;
     const int smem = fused_smem(sh.G, sh.D, chunk).words * 4;
     if (smem > di.smem_optin) continue;
     const int mc = max_active_clusters(kern, dev, n, smem, di.smem_optin);
     if (mc <= 0) continue;
     best = StepPlan{n, chunk, smem};
-    if (forced || rows <= mc) break;  // one wave (or forced)
+    if (forced || rows * 5 >= 4LL * mc) break;  // covers 80% of a wave
   }
   if (best.ncta == 0 && forced) {
     setenv("LOKI_CLUSTER", "", 1);  // a forced size that cannot run: plan normally

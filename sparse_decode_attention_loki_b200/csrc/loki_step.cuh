@@ -552,8 +552,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   // 4. log-sum-exp merge of the cluster's states
   cluster.sync();
   const int Hq = a.da.n_kv_heads * G;
-  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, reinterpret_cast<float *>(ring),
-                        a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
+  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
   cluster.sync();
 }
 

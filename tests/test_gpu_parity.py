@@ -183,14 +183,17 @@ def test_exact_ties_take_lowest_index(ncta):
     parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(D), "bf16")
 
 
-@pytest.mark.parametrize("ncta", [None, 16])
-def test_zero_query_selects_first_k(ncta):
-    w = small_workload("bf16", 128, 4, 1234)
-    inp = gen.decode_inputs(w, seq_len=1234)
+@pytest.mark.parametrize("S,ncta", [(1234, None), (1234, 16), (15000, None), (15000, 1), (20000, 16)])
+def test_zero_query_selects_first_k(S, ncta):
+    # every score is equal: the selection is decided by the tie rule alone;
+    # the longer rows put more candidate keys in one CTA than its exchange
+    # slot holds, which takes the distributed refinement path
+    w = small_workload("bf16", 128, 4, S)
+    inp = gen.decode_inputs(w, seq_len=S)
     inp["q"] = torch.zeros_like(inp["q"])
     inp["q64"] = np.zeros_like(inp["q64"])
-    k = 77
-    out, idx, ref, K_hat, V, *_ = run_decode(w, 1234, 32, k, ncta=ncta, inp=inp)
+    k = 77 if S < 10000 else 3001
+    out, idx, ref, K_hat, V, *_ = run_decode(w, S, 32, k, ncta=ncta, inp=inp)
     assert np.all(idx == np.arange(k, dtype=np.int32))
     for h in range(w.n_q_heads):
         np.testing.assert_allclose(out[:, h], V[:, h // 4, :k].mean(axis=1), atol=5e-3)

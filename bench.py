@@ -309,6 +309,32 @@ def run_ours(args):
         for i in range(n):
             t_e2e += e2e_ev[i][0].elapsed_time(e2e_ev[i][1])
         done += n
+    # ---------------- Exact-TopK baseline (d = D) and the agreement of the two selections
+    idx_exact = torch.empty_like(idx)
+    for i in range(args.warmup):
+        L.loki_decode_attention(cache, S, qs[i % NSET], P, D, w.k, out=out, idx=idx_exact)
+    torch.cuda.synchronize()
+    ex_steps = min(args.steps, 500)
+    ex_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CH, ex_steps))]
+    t_exact = 0.0
+    done = 0
+    while done < ex_steps:
+        n = min(CH, ex_steps - done)
+        for i in range(n):
+            flush.fill_(float(i & 7))
+            ex_ev[i][0].record(stream)
+            L.loki_decode_attention(cache, S, qs[(done + i) % NSET], P, D, w.k, out=out, idx=idx_exact)
+            ex_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_exact += ex_ev[i][0].elapsed_time(ex_ev[i][1])
+        done += n
+    jac = []
+    for j in range(NSET):
+        L.loki_decode_attention(cache, S, qs[j], P, w.d, w.k, out=out, idx=idx)
+        L.loki_decode_attention(cache, S, qs[j], P, D, w.k, out=out, idx=idx_exact)
+        jac.append(L.topk_jaccard(idx, idx_exact))
+    jaccard = torch.stack(jac)
     h2d = q_host[0].numel() * q_host[0].element_size()
     d2h = out_host.numel() * 4 + idx_host.numel() * 4
 
@@ -346,10 +372,13 @@ def run_ours(args):
                       "launch": {"cluster_ctas": dcl, "ctas": dct}},
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
             "append_us": app_us,
+            "exact_topk": {"us": t_exact * 1000.0 / ex_steps, "d": D, "k": w.k, "steps": ex_steps,
+                           "jaccard_vs_loki": {"mean": float(jaccard.mean()), "min": float(jaccard.min()),
+                                               "rows": int(jaccard.numel())}},
             "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256},
             "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gpu_launches": 4 * K,
+            "gpu_launches": 4 * K,  # timed loop: append, rotate, decode, dense
             "clocks": clocks,
             "wall_s_timed_region": wall,
             "per_step_loki_us": {"p50": float(np.percentile(per_step_loki, 50)) * 1000.0,

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 4
+#define LOKI_VERSION 5
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -162,6 +162,22 @@ LOKI_API loki_status dense_decode_attention(const loki_cache *cache, int32_t seq
                                    int32_t n_q_heads, const void *q,
                                    const float *P, float scale, float *out,
                                    void *stream);
+
+/* loki_topk_jaccard -- agreement of two top-k selections: for every row r,
+ * jaccard[r] = |A_r n B_r| / |A_r u B_r| of the index sets A_r = idx_a[r, :k]
+ * and B_r = idx_b[r, :k].  This is the selection-agreement measure the summary
+ * page reports between Loki and the exact top-k (sections "Key results" and
+ * "Experimental setup"); the exact top-k is loki_decode_attention with
+ * d = D (the ranking on all principal dimensions equals the ranking on the
+ * unrotated keys, since P is orthonormal).
+ *   idx_a, idx_b : [rows, k] int32 device arrays; each row holds k distinct
+ *                  indices in ascending order (as loki_decode_attention
+ *                  writes them).  Rows that are not ascending give an
+ *                  unspecified value, never an out-of-bounds access.
+ *   jaccard      : [rows] float device array (written).
+ * Requires rows >= 1 and k >= 1.  One kernel on `stream`. */
+LOKI_API loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_b, int32_t rows,
+                              int32_t k, float *jaccard, void *stream);
 
 /* Launch shape a decode call with these sizes would use, for logging and
  * tests.  shape: host array of 4 int32.

@@ -14,4 +14,5 @@ from .loki_oracle import (  # noqa: F401
     default_scale,
     loki_decode,
     dense_decode,
+    topk_jaccard,
 )

@@ -205,6 +205,22 @@ def sparse_attention(q_hat, K_hat, V_cache, idx, scale: float, return_weights: b
     return (out, weights) if return_weights else out
 
 
+def topk_jaccard(idx_a, idx_b) -> np.ndarray:
+    """Agreement of two top-k selections, the measure the summary page reports
+    between Loki and exact attention ("Key results", "Experimental setup"):
+    |A n B| / |A u B| of the index sets of every row.  [..., k] -> [...]."""
+    a = np.asarray(idx_a)
+    b = np.asarray(idx_b)
+    k = a.shape[-1]
+    fa = a.reshape(-1, k)
+    fb = b.reshape(-1, b.shape[-1])
+    out = np.empty(fa.shape[0])
+    for r in range(fa.shape[0]):
+        sa, sb = set(fa[r].tolist()), set(fb[r].tolist())
+        out[r] = len(sa & sb) / len(sa | sb)
+    return out.reshape(a.shape[:-1])
+
+
 def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)
 

@@ -18,6 +18,7 @@ from .api import (
     loki_decode_workspace_size,
     loki_status_string,
     loki_version,
+    topk_jaccard,
 )
 from .sharding import shard_batches
 
@@ -34,5 +35,6 @@ __all__ = [
     "loki_decode_workspace_size",
     "loki_status_string",
     "loki_version",
+    "topk_jaccard",
     "shard_batches",
 ]

@@ -164,6 +164,26 @@ def dense_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: t
     return out
 
 
+def topk_jaccard(idx_a: torch.Tensor, idx_b: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Per-row Jaccard similarity of two selections [..., k] int32 (ascending
+    rows, as loki_decode_attention returns them).  Returns float32 [...]: the
+    agreement of Loki's selection with the exact top-k when idx_b comes from a
+    call with d = D."""
+    if idx_a.shape != idx_b.shape or idx_a.dim() < 1:
+        raise ValueError(f"selections must have equal shapes, got {tuple(idx_a.shape)} and {tuple(idx_b.shape)}")
+    k = int(idx_a.shape[-1])
+    rows = idx_a.numel() // k if k else 0
+    dev = idx_a.device
+    for t, nm in ((idx_a, "idx_a"), (idx_b, "idx_b")):
+        if t.dtype != torch.int32 or t.device != dev or not t.is_contiguous() or dev.type != "cuda":
+            raise ValueError(f"{nm} must be a contiguous int32 CUDA tensor on {dev}")
+    out = torch.empty(idx_a.shape[:-1], dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _lib.check(_lib.load().loki_topk_jaccard(_ptr(idx_a), _ptr(idx_b), int(rows), k, _ptr(out),
+                                                 _stream_ptr(dev, stream)))
+    return out
+
+
 def loki_decode_launch_shape(cache: LokiCache, seq_len: int, n_q_heads: int, k: int = 1,
                              dense: bool = False) -> Tuple[int, int, int, int]:
     """Grid sizes of a decode call.  Loki: (rotation CTAs, decode CTAs per row

@@ -14,6 +14,7 @@
 #include "append.cuh"
 #include "decode.cuh"
 #include "loki_step.cuh"
+#include "topk_stats.cuh"
 
 namespace {
 
@@ -586,6 +587,23 @@ loki_status loki_decode_attention_noalloc(const loki_cache *cache, int32_t seq_l
   if (s != LOKI_OK) return s;
   return loki_decode_attention(cache, seq_len, n_q_heads, q, P, d, k, scale, out, idx, scratch,
                                kNoAllocScratchBytes, stream);
+}
+
+loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_b, int32_t rows, int32_t k, float *jaccard,
+                              void *stream) {
+  if (rows < 1 || k < 1) return fail(LOKI_ERR_INVALID_ARG, "rows=%d and k=%d must be >= 1", rows, k);
+  if (!idx_a || !idx_b || !jaccard) return fail(LOKI_ERR_INVALID_ARG, "idx_a, idx_b or jaccard is NULL");
+  if (!aligned(idx_a, 4) || !aligned(idx_b, 4) || !aligned(jaccard, 4))
+    return fail(LOKI_ERR_INVALID_ARG, "idx_a, idx_b and jaccard must be 4-byte aligned");
+  JaccardArgs a;
+  a.a = idx_a;
+  a.b = idx_b;
+  a.out = jaccard;
+  a.k = k;
+  topk_jaccard_kernel<<<(unsigned)rows, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "topk_jaccard_kernel launch");
+  return LOKI_OK;
 }
 
 loki_status dense_decode_attention(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, const void *q,

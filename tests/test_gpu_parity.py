@@ -254,6 +254,39 @@ def test_repeated_calls_are_identical():
         assert np.array_equal(o2.cpu().numpy(), out)
 
 
+# ----------------------------------------------------------------------------- Exact-TopK baseline and agreement
+@pytest.mark.parametrize("rows,S,k", [(1, 10, 1), (5, 300, 7), (3, 5000, 1000), (2, 40000, 4096), (4, 8, 8)])
+def test_jaccard_kernel_matches_oracle(rows, S, k):
+    rng = np.random.default_rng(rows * 1000 + k)
+    a = np.stack([np.sort(rng.choice(S, k, replace=False)) for _ in range(rows)]).astype(np.int32)
+    b = np.stack([np.sort(rng.choice(S, k, replace=False)) for _ in range(rows)]).astype(np.int32)
+    b[0] = a[0]  # identical sets
+    if rows > 1 and 2 * k <= S:  # disjoint sets
+        b[1] = np.sort(rng.choice(np.setdiff1d(np.arange(S), a[1]), k, replace=False))
+    got = L().topk_jaccard(torch.from_numpy(a).to(DEV), torch.from_numpy(b).to(DEV)).cpu().numpy()
+    # c / (2k - c) of two integers, correctly rounded to fp32 on both sides
+    np.testing.assert_array_equal(got, oracle.topk_jaccard(a, b).astype(np.float32))
+
+
+@pytest.mark.parametrize("dtype,G", [("bf16", 4), ("f32", 1)])
+def test_exact_topk_baseline_and_agreement(dtype, G):
+    # the Exact-TopK baseline is the decode with d = D; the agreement of Loki's
+    # selection with it is the Jaccard similarity of the two index sets
+    S, k = 3001, 375
+    w = small_workload(dtype, 128, G, S)
+    inp = gen.decode_inputs(w, seq_len=S)
+    P32 = basis(w)
+    o1, i1, ref1, K_hat, V, *_ = run_decode(w, S, 32, k, inp=inp, P32=P32)
+    o2, i2, ref2, *_ = run_decode(w, S, 128, k, inp=inp, P32=P32)
+    parity.check_decode(o1, i1, ref1, ref1["q_hat"], K_hat, V, oracle.default_scale(128), dtype)
+    parity.check_decode(o2, i2, ref2, ref2["q_hat"], K_hat, V, oracle.default_scale(128), dtype)
+    got = L().topk_jaccard(torch.from_numpy(i1).to(DEV), torch.from_numpy(i2).to(DEV)).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle.topk_jaccard(i1, i2).astype(np.float32))
+    if np.array_equal(i1, ref1["idx"]) and np.array_equal(i2, ref2["idx"]):
+        np.testing.assert_array_equal(got, oracle.topk_jaccard(ref1["idx"], ref2["idx"]).astype(np.float32))
+    assert np.all(got > 0.0) and np.all(got <= 1.0)
+
+
 # ----------------------------------------------------------------------------- dense, small shapes
 @pytest.mark.parametrize("ncta", [None, 1, 16])
 @pytest.mark.parametrize("dtype,D,G,S", [

@@ -408,3 +408,40 @@ def test_oracle_matches_stored_tiny_output():
     assert r["idx"].tolist() == ref["idx"]
     np.testing.assert_allclose(r["out"], np.array(ref["out"]), rtol=0, atol=1e-9)
     np.testing.assert_allclose(dense, np.array(ref["dense_out"]), rtol=0, atol=1e-9)
+
+
+# ----------------------------------------------------------------------------- top-k agreement
+def test_jaccard_closed_forms():
+    a = np.array([[1, 2, 3, 4], [0, 1, 2, 3], [5, 6, 7, 8]])
+    b = np.array([[3, 4, 5, 6], [0, 1, 2, 3], [1, 2, 3, 4]])
+    # |{3,4}| / |{1..6}|, identical sets, disjoint sets
+    np.testing.assert_allclose(oracle.topk_jaccard(a, b), [2 / 6, 1.0, 0.0], rtol=0, atol=1e-15)
+
+
+def test_jaccard_brute_force():
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        S, k = int(rng.integers(1, 40)), 0
+        k = int(rng.integers(1, S + 1))
+        a = np.sort(rng.choice(S, k, replace=False))
+        b = np.sort(rng.choice(S, k, replace=False))
+        inter = sum(1 for x in a if x in b)
+        union = len(np.union1d(a, b))
+        assert oracle.topk_jaccard(a[None], b[None])[0] == inter / union
+        assert inter / union == inter / (2 * k - inter)
+
+
+def test_exact_topk_is_the_full_dimension_selection():
+    # d = D ranks on q_hat . k_hat = q . k (P orthonormal): the exact top-k
+    rng = np.random.default_rng(4)
+    B, Hkv, G, D, S, k = 1, 2, 2, 16, 50, 9
+    X = rng.standard_normal((256, D))
+    P, _ = oracle.pca_basis(X)
+    keys = rng.standard_normal((B, Hkv, S, D))
+    q = rng.standard_normal((B, Hkv * G, D))
+    K_hat = oracle.rotate_keys(keys, np.stack([P, P]), "f64")
+    ref = oracle.loki_decode(q, K_hat, np.zeros_like(K_hat), np.stack([P, P]), S, D, k)
+    for g in range(Hkv):
+        s = sum(keys[0, g] @ q[0, h] for h in range(g * G, (g + 1) * G))
+        exact = np.sort(np.argsort(-s, kind="stable")[:k])
+        assert oracle.topk_jaccard(ref["idx"][0, g][None], exact[None])[0] == 1.0

@@ -115,6 +115,12 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, u
 }
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// Skewed index of bin b in a shared-memory histogram (one spare word per 32
+// bins): the consecutive bins one thread scans fall into distinct banks
+// across a warp.
+__host__ __device__ inline int hskew(int b) { return b + (b >> 5); }
+__host__ __device__ inline constexpr int skewed_words(int bins) { return bins + bins / 32; }
+
 // Order-preserving map fp32 -> uint32: a > b  <=>  key(a) > key(b) for finite
 // a, b.  -0 and +0 map to the same key so that equal scores tie (and the lower
 // index wins) regardless of the sign of zero.

@@ -196,8 +196,8 @@ struct ScoreStream {
     return sc;
   }
 
-  // keys[token] = score_key(score) for the tokens of stage s, and hist[key >>
-  // HSHIFT] += 1 for each of them.
+  // keys[token] = score_key(score) for the tokens of stage s, and bin
+  // key >> HSHIFT of the skewed histogram hist (see hskew) += 1 for each.
   template <int HSHIFT>
   __device__ __forceinline__ static void consume_keys(int len, int nck, int s, const unsigned char *wring,
                                                       const float (&uv)[VEC], uint32_t *keys, uint32_t *hist) {
@@ -212,7 +212,7 @@ struct ScoreStream {
       if (c == 0 && base + t < len) {
         const uint32_t key = score_key(sc);
         keys[base + t] = key;
-        atomicAdd(&hist[key >> HSHIFT], 1u);
+        atomicAdd(&hist[hskew((int)(key >> HSHIFT))], 1u);
       }
     }
   }
@@ -237,8 +237,8 @@ __device__ __forceinline__ void score_prologue(const T *Krow, int t0, int len, i
 }
 
 // The key stream: leaves score_key(score) of every token of [t0, t0+len) in
-// keys[] and adds each key's top bits to hist[key >> HSHIFT].  Ends with
-// __syncthreads().
+// keys[] and counts each key's top bits in the skewed histogram hist.  Ends
+// with __syncthreads().
 template <typename T, int D, int LPT, int SB, int NS, int HSHIFT>
 __device__ __forceinline__ void score_keys_loop(const T *Krow, int t0, int len, int nck, unsigned char *ring,
                                                 const float *u, uint32_t *keys, uint32_t *hist) {

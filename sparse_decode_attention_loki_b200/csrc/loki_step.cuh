@@ -13,13 +13,17 @@
 //        streams K_hat[i, :d], keeps one order-preserving uint32 key per
 //        token in shared memory and histograms the keys' top 11 bits on the
 //        way;
-//     2. cluster radix select over 11/11/10-bit digits: each CTA adds the
-//        non-zero bins of its histogram into every CTA of the cluster through
-//        distributed shared memory, so after one cluster barrier every CTA
-//        knows the bucket of the k-th largest key; the keys in that bucket
-//        (the candidates) are refined the same way; the CTAs then exchange
-//        their counts above and at the threshold and write their indices in
-//        ascending order, ties at the threshold going to the lower index;
+//     2. cluster radix select over 11/11/10-bit digits: every CTA adds the
+//        non-zero bins of its histogram into the leader CTA's (distributed
+//        shared memory reductions), the leader finds the bucket of the k-th
+//        largest key and tells every CTA; each CTA sends the leader its keys in
+//        that bucket (the candidates, a few percent) and its count above it;
+//        the leader finishes the threshold on the candidates, derives every
+//        CTA's share of the selection (ties at the threshold go to the lower
+//        index) and hands each CTA its (threshold, ties to take, offset); each
+//        CTA writes its indices in ascending order (should a CTA's candidates
+//        overflow its slot at the leader, the cluster refines with distributed
+//        histogram passes instead);
 //     3. (only now waiting for the rotate grid, a programmatic dependency)
 //        the k selected rows are split evenly over the cluster: gather K_hat
 //        and V rows through the ring, online softmax per query head;
@@ -38,7 +42,6 @@ constexpr int kDig2Bits = 11;                   // second digit: bits 20..10
 constexpr int kDig3Bits = 10;                   // third digit: bits 9..0
 constexpr int kMaxCluster = 16;
 constexpr int kMaxChunk = 24576;                // tokens per decode CTA, at most
-constexpr int kCandCap = 4096;                  // candidate list per CTA (keys)
 
 // Workspace layout (bytes, each region 256-byte aligned).
 struct WsLayout {
@@ -152,30 +155,31 @@ __host__ __device__ inline FusedSmem fused_smem(int G, int D, int chunk) {
   L.pacc = o; o += G * D;
   L.ctl = o;  o += 128;
   L.tbl = o;  o += 2 * kMaxCluster;
-  L.hist = o; o += round4(kDig1Bins > 8 * D ? kDig1Bins : 8 * D);
+  L.hist = o; o += round4(skewed_words(kDig1Bins) > 8 * D ? skewed_words(kDig1Bins) : 8 * D);
   L.ring = o; o += kRingWords;
   L.keys = o; o += round4(chunk);
   L.words = o;
   return L;
 }
 
-// Skewed index of bin b in a shared-memory histogram: the consecutive bins a
-// thread scans fall into distinct banks across a warp.
-__host__ __device__ inline int hskew(int b) { return b + (b >> 5); }
-__host__ __device__ inline constexpr int skewed_words(int bins) { return bins + bins / 32; }
 
-// select buffers inside the ring (word offsets)
-constexpr int kRecv1 = 0;
-constexpr int kRecv2 = kRecv1 + skewed_words(1 << kDig1Bits);
+// select buffers inside the ring (word offsets).  The leader (rank 0) keeps
+// the candidate slots of every CTA and its own refinement histogram; the
+// distributed fallback reuses the same words once the slots are dead.
+constexpr int kHref = 0;                                       // leader's refinement histogram
+constexpr int kHdr = kHref + skewed_words(1 << kDig2Bits);     // [kMaxCluster][2]: candidates, count above
+constexpr int kSlots = kHdr + 2 * kMaxCluster;                 // candidate keys, one slot per CTA
+constexpr int kRecv2 = 0;
 constexpr int kRecv3 = kRecv2 + skewed_words(1 << kDig2Bits);
 constexpr int kHloc = kRecv3 + skewed_words(1 << kDig3Bits);
-constexpr int kCand = kHloc + (1 << kDig2Bits);
-static_assert(kCand + kCandCap <= kRingWords, "select buffers must fit in the ring");
+static_assert(kHloc + (1 << kDig2Bits) <= kRingWords, "select buffers must fit in the ring");
+static_assert(kSlots + kMaxCluster * 256 <= kRingWords, "candidate slots must fit in the ring");
 
 // ctl words (write_selection uses 48..63)
 constexpr int kSelWtot = 0;     // [0..7] block-scan scratch
-constexpr int kSelBucket = 8;   // [8..10] bucket, count above it, count in it
-constexpr int kSelNcand = 12;
+constexpr int kSelBucket = 8;   // [8..10] bucket, count above it, count in it (this CTA's search)
+constexpr int kSelFirst = 16;   // [16..18] the leader's first-digit result
+constexpr int kSelOut = 20;     // [20..24] from the leader: prefix, mask, take, offset, fallback
 
 // Among nb bins (skewed layout), find the one in which the count taken from
 // the top reaches `remaining` (1 <= remaining <= total).  Result in
@@ -216,6 +220,15 @@ __device__ __forceinline__ void push_bins(int ncta, const uint32_t *local, int n
   }
 }
 
+// Add the non-zero bins of this CTA's skewed histogram into the skewed
+// histogram at `dst` (a shared::cluster address, another CTA's).
+__device__ __forceinline__ void push_skewed(const uint32_t *local, int nb, uint32_t dst) {
+  for (int e = threadIdx.x; e < nb; e += kThreads) {
+    const uint32_t c = local[hskew(e)];
+    if (c) dsmem_red_add(dst + 4u * (uint32_t)hskew(e), c);
+  }
+}
+
 // Warp-inclusive scan of a 32-bit value.
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   const int lane = threadIdx.x & 31;
@@ -225,41 +238,6 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
     if (lane >= off) v += t;
   }
   return v;
-}
-
-// Keys of keys[0, len) with (key & mask) == prefix, copied to cand[] while
-// they fit in kCandCap (in no particular order); returns their count.  A
-// counting sweep and a block scan give each thread its output offset, a second
-// sweep writes; four keys per thread and step (keys is 16-byte aligned and
-// padded to a multiple of 4).
-__device__ __forceinline__ int gather_candidates(const uint32_t *keys, int len, uint32_t prefix, uint32_t mask,
-                                                 uint32_t *cand, uint32_t *ctl) {
-  const int tid = threadIdx.x;
-  const int n4 = (len + 3) >> 2;
-  uint32_t mine = 0u;
-  for (int j4 = tid; j4 < n4; j4 += kThreads) {
-    const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
-    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) mine += (4 * j4 + e < len && (kk[e] & mask) == prefix) ? 1u : 0u;
-  }
-  // exclusive prefix over threads: total after thread t = suffix sum of the rest
-  const uint32_t after = block_excl_suffix_sum(mine, ctl + kSelWtot);
-  const uint32_t total = block_sum(mine, ctl + kSelWtot);
-  uint32_t pos = total - after - mine;
-  for (int j4 = tid; j4 < n4; j4 += kThreads) {
-    const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
-    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (4 * j4 + e < len && (kk[e] & mask) == prefix) {
-        if (pos < (uint32_t)kCandCap) cand[pos] = kk[e];
-        ++pos;
-      }
-    }
-  }
-  __syncthreads();
-  return (int)total;
 }
 
 // One cluster refinement pass: keys of set[0, n) with (key & mask) == prefix
@@ -453,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   unsigned char *ring = reinterpret_cast<unsigned char *>(smem + L.ring);
   uint32_t *rw = smem + L.ring;  // the ring as words, for the select buffers
   uint32_t *keys = smem + L.keys;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.da.seq_len;
   const uint32_t k = (uint32_t)a.da.k;
   const int t0 = min(S, rank * a.da.chunk);
@@ -468,69 +446,205 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   lowrank_query<T, D, G>(a.da, b, g, qhat, reinterpret_cast<float *>(hist), u, [&] {
     LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.da.nck, ring)));
   });
-  for (int e = tid; e < kDig1Bins; e += kThreads) hist[e] = 0u;
+  for (int e = tid; e < skewed_words(kDig1Bins); e += kThreads) hist[e] = 0u;
   __syncthreads();
+  cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
                     (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(Krow, t0, len, a.da.nck,
                                                                                        ring, u, keys, hist)));
 
   // 2. cluster radix select; the ring is idle until the gather
-  uint32_t *recv1 = rw + kRecv1, *recv2 = rw + kRecv2, *recv3 = rw + kRecv3;
-  uint32_t *hloc = rw + kHloc, *cand = rw + kCand;
-  for (int e = tid; e < kHloc; e += kThreads) rw[e] = 0u;  // recv1..recv3
-  cluster.sync();  // every CTA's receive histograms are zero
-  push_bins(ncta, hist, kDig1Bins, recv1);
+  const bool leader = rank == 0;
+  cluster_wait();  // every CTA, the leader in particular, zeroed its histogram before its stream
+  if (!leader) push_skewed(hist, kDig1Bins, dsmem_addr(hist, 0u));
+  cluster.sync();  // the leader's histogram holds the cluster's sum
+  if (leader) {
+    find_bucket(hist, kDig1Bins, k, ctl);
+    if (tid < ncta) {
+      const uint32_t dst = dsmem_addr(ctl + kSelFirst, (uint32_t)tid);
+      dsmem_st(dst, ctl[kSelBucket + 0]);
+      dsmem_st(dst + 4u, ctl[kSelBucket + 1]);
+      dsmem_st(dst + 8u, ctl[kSelBucket + 2]);
+    }
+  }
   cluster.sync();
-  find_bucket(recv1, kDig1Bins, k, ctl);
-  uint32_t remaining = k - ctl[kSelBucket + 1];
-  uint32_t prefix = ctl[kSelBucket + 0] << (32 - kDig1Bits);
+  uint32_t remaining = k - ctl[kSelFirst + 1];
+  const bool refine = ctl[kSelFirst + 2] != remaining;  // else the whole bucket is taken
+  uint32_t prefix = ctl[kSelFirst + 0] << (32 - kDig1Bits);
   uint32_t mask = ~0u << (32 - kDig1Bits);
-  if (ctl[kSelBucket + 2] != remaining) {  // uniform over the cluster
-    const int ncand = gather_candidates(keys, len, prefix, mask, cand, ctl);
-    const bool fits = ncand <= kCandCap;
-    const uint32_t *set = fits ? cand : keys;
-    const int nset = fits ? ncand : len;
+  const int cap = ((kRingWords - kSlots) / ncta) & ~3;  // candidate slot per CTA, at the leader
+  uint32_t *href = rw + kHref, *hdr = rw + kHdr;
+
+  // this CTA's candidates (its keys in the bucket) into its slot at the
+  // leader, with its count of candidates and of keys above the bucket
+  {
+    const int n4 = (len + 3) >> 2;
+    uint32_t mine = 0u, above = 0u;
+    for (int j4 = tid; j4 < n4; j4 += kThreads) {
+      const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+      const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (4 * j4 + e < len) {
+          const uint32_t km = kk[e] & mask;
+          mine += km == prefix;
+          above += km > prefix;
+        }
+      }
+    }
+    const uint32_t after = block_excl_suffix_sum(mine, ctl + kSelWtot);
+    const uint32_t total = block_sum(mine, ctl + kSelWtot);
+    above = block_sum(above, ctl + kSelWtot);
+    if (refine && total <= (uint32_t)cap) {
+      const uint32_t slot = dsmem_addr(rw + kSlots + rank * cap, 0u);
+      uint32_t pos = total - after - mine;
+      for (int j4 = tid; j4 < n4; j4 += kThreads) {
+        const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+        const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (4 * j4 + e < len && (kk[e] & mask) == prefix) {
+            dsmem_st(slot + 4u * pos, kk[e]);
+            ++pos;
+          }
+        }
+      }
+    }
+    if (tid == 0) {
+      const uint32_t h = dsmem_addr(hdr + 2 * rank, 0u);
+      dsmem_st(h, total);
+      dsmem_st(h + 4u, above);
+    }
+  }
+  cluster.sync();  // the leader holds every CTA's candidates and counts
+
+  // the leader finishes the threshold on the union of the candidates, then
+  // gives every CTA its (prefix, mask, take, offset)
+  if (leader) {
+    bool overflow = false;
+    for (int r = 0; r < ncta; ++r) overflow |= hdr[2 * r] > (uint32_t)cap;
+    uint32_t pre = prefix, msk = mask, rem = remaining;
+    if (refine && !overflow) {
+      constexpr int SH2 = 32 - kDig1Bits - kDig2Bits;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? SH2 : 0;
+        const int nb = pass == 0 ? (1 << kDig2Bits) : (1 << kDig3Bits);
+        for (int e = tid; e < skewed_words(1 << kDig2Bits); e += kThreads) href[e] = 0u;
+        __syncthreads();
+        for (int r = 0; r < ncta; ++r) {
+          const uint32_t *sl = rw + kSlots + r * cap;
+          for (int i = tid; i < (int)hdr[2 * r]; i += kThreads) {
+            const uint32_t key = sl[i];
+            if ((key & msk) == pre) atomicAdd(&href[hskew((int)((key >> shift) & (uint32_t)(nb - 1)))], 1u);
+          }
+        }
+        __syncthreads();
+        find_bucket(href, nb, rem, ctl);
+        rem -= ctl[kSelBucket + 1];
+        const uint32_t inb = ctl[kSelBucket + 2];
+        pre |= ctl[kSelBucket + 0] << shift;
+        msk |= (uint32_t)(nb - 1) << shift;
+        __syncthreads();  // ctl read before it is reused
+        if (inb == rem) break;
+      }
+      // every CTA's counts above and at the threshold (warp w: CTAs w, w+8)
+      for (int r = warp; r < ncta; r += kWarps) {
+        const uint32_t *sl = rw + kSlots + r * cap;
+        uint32_t gtc = 0u, eqc = 0u;
+        for (int i = lane; i < (int)hdr[2 * r]; i += 32) {
+          const uint32_t km = sl[i] & msk;
+          gtc += km > pre;
+          eqc += km == pre;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          gtc += __shfl_xor_sync(kFull, gtc, off);
+          eqc += __shfl_xor_sync(kFull, eqc, off);
+        }
+        if (lane == 0) {
+          tbl[r] = gtc + hdr[2 * r + 1];
+          tbl[kMaxCluster + r] = eqc;
+        }
+      }
+    } else if (!refine) {
+      if (tid < ncta) {
+        tbl[tid] = hdr[2 * tid + 1];
+        tbl[kMaxCluster + tid] = hdr[2 * tid];
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      // ties at the threshold go to the lower index: lower CTAs first
+      const uint32_t fallback = (refine && overflow) ? 1u : 0u;
+      uint32_t eq_before = 0u, off = 0u;
+      for (int r = 0; r < ncta; ++r) {
+        const uint32_t eqr = tbl[kMaxCluster + r];
+        const uint32_t take_r = fallback ? 0u : min(eqr, rem > eq_before ? rem - eq_before : 0u);
+        const uint32_t dst = dsmem_addr(ctl + kSelOut, (uint32_t)r);
+        dsmem_st(dst, pre);
+        dsmem_st(dst + 4u, msk);
+        dsmem_st(dst + 8u, take_r);
+        dsmem_st(dst + 12u, off);
+        dsmem_st(dst + 16u, fallback);
+        off += tbl[r] + take_r;
+        eq_before += eqr;
+      }
+    }
+  }
+  cluster.sync();
+  uint32_t take, offset;
+  if (ctl[kSelOut + 4] == 0u) {
+    prefix = ctl[kSelOut + 0];
+    mask = ctl[kSelOut + 1];
+    take = ctl[kSelOut + 2];
+    offset = ctl[kSelOut + 3];
+  } else {
+    // a candidate slot overflowed (uniform over the cluster): distributed
+    // refinement passes over every CTA's own keys
+    uint32_t *recv2 = rw + kRecv2, *recv3 = rw + kRecv3, *hloc = rw + kHloc;
+    for (int e = tid; e < kHloc - kRecv2; e += kThreads) recv2[e] = 0u;  // recv2 and recv3
+    cluster.sync();  // every CTA's receive histograms are zero
     constexpr int SH2 = 32 - kDig1Bits - kDig2Bits;
-    refine_pass(cluster, ncta, set, nset, prefix, mask, SH2, 1 << kDig2Bits, remaining, hloc, recv2, ctl);
+    refine_pass(cluster, ncta, keys, len, prefix, mask, SH2, 1 << kDig2Bits, remaining, hloc, recv2, ctl);
     remaining -= ctl[kSelBucket + 1];
     prefix |= ctl[kSelBucket + 0] << SH2;
     mask |= (uint32_t)((1 << kDig2Bits) - 1) << SH2;
     if (ctl[kSelBucket + 2] != remaining) {  // uniform over the cluster
-      refine_pass(cluster, ncta, set, nset, prefix, mask, 0, 1 << kDig3Bits, remaining, hloc, recv3, ctl);
+      refine_pass(cluster, ncta, keys, len, prefix, mask, 0, 1 << kDig3Bits, remaining, hloc, recv3, ctl);
       remaining -= ctl[kSelBucket + 1];
       prefix |= ctl[kSelBucket + 0];
       mask = ~0u;
     }
-  }
-  // this CTA's counts above and at the threshold, into every CTA's table
-  uint32_t gt = 0u, eq = 0u;
-  for (int j4 = tid; j4 < (len + 3) >> 2; j4 += kThreads) {
-    const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
-    const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+    uint32_t gt = 0u, eq = 0u;
+    for (int j4 = tid; j4 < (len + 3) >> 2; j4 += kThreads) {
+      const uint4 v = reinterpret_cast<const uint4 *>(keys)[j4];
+      const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (4 * j4 + e < len) {
-        const uint32_t km = kk[e] & mask;
-        gt += km > prefix;
-        eq += km == prefix;
+      for (int e = 0; e < 4; ++e) {
+        if (4 * j4 + e < len) {
+          const uint32_t km = kk[e] & mask;
+          gt += km > prefix;
+          eq += km == prefix;
+        }
       }
     }
+    gt = block_sum(gt, ctl + kSelWtot);
+    eq = block_sum(eq, ctl + kSelWtot);
+    if (tid < ncta) {
+      dsmem_st(dsmem_addr(tbl + rank, (uint32_t)tid), gt);
+      dsmem_st(dsmem_addr(tbl + kMaxCluster + rank, (uint32_t)tid), eq);
+    }
+    cluster.sync();
+    // ties at the threshold go to the lower index: lower CTAs first
+    uint32_t eq_before = 0u;
+    offset = 0u;
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t want = remaining > eq_before ? remaining - eq_before : 0u;
+      offset += tbl[r] + min(tbl[kMaxCluster + r], want);
+      eq_before += tbl[kMaxCluster + r];
+    }
+    take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
   }
-  gt = block_sum(gt, ctl + kSelWtot);
-  eq = block_sum(eq, ctl + kSelWtot);
-  if (tid < ncta) {
-    dsmem_st(dsmem_addr(tbl + rank, (uint32_t)tid), gt);
-    dsmem_st(dsmem_addr(tbl + kMaxCluster + rank, (uint32_t)tid), eq);
-  }
-  cluster.sync();
-  // ties at the threshold go to the lower index: lower CTAs first
-  uint32_t eq_before = 0u, offset = 0u;
-  for (int r = 0; r < rank; ++r) {
-    const uint32_t want = remaining > eq_before ? remaining - eq_before : 0u;
-    offset += tbl[r] + min(tbl[kMaxCluster + r], want);
-    eq_before += tbl[kMaxCluster + r];
-  }
-  const uint32_t take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
   int32_t *idx_row = a.da.idx + (size_t)row * k;
   write_selection_vec(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
   cluster.sync();  // the whole row of idx is written and visible to the cluster

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 5
+#define LOKI_VERSION 6
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -88,6 +88,9 @@ typedef struct {
  * Computes k_hat[b][g][pos+t][j] = round_to_dtype( sum_i k_new[b][g][t][i] *
  * P[g][i][j] ) with fp32 accumulation and round-to-nearest-even, and copies
  * v_new unchanged.  Entries outside [pos, pos + n_new) are not touched.
+ * bf16 caches with B * n_new >= 256 take the tensor-core path: P is split into
+ * three bf16 terms (summing to P within 2^-27 relative) and the 3*D products
+ * are accumulated in fp32 by tcgen05.mma before the single rounding.
  * Requires 0 <= pos, 1 <= n_new, pos + n_new <= S_cap. */
 LOKI_API loki_status loki_append(const loki_cache *cache, int32_t pos, int32_t n_new,
                         const void *k_new, const void *v_new, const float *P,
@@ -162,6 +165,13 @@ LOKI_API loki_status dense_decode_attention(const loki_cache *cache, int32_t seq
                                    int32_t n_q_heads, const void *q,
                                    const float *P, float scale, float *out,
                                    void *stream);
+
+/* loki_device_error_count -- the number of bounded device-side waits that
+ * have timed out in this process on the current device since the library was
+ * loaded (a kernel that times out records it here, releases what it holds and
+ * returns; its outputs are then incomplete).  Synchronous: copies a counter
+ * from device memory.  *count is a host pointer. */
+LOKI_API loki_status loki_device_error_count(uint32_t *count);
 
 /* loki_topk_jaccard -- agreement of two top-k selections: for every row r,
  * jaccard[r] = |A_r n B_r| / |A_r u B_r| of the index sets A_r = idx_a[r, :k]

@@ -45,6 +45,7 @@ SIGNATURES = {
                                              _vp]),
     "dense_decode_attention": (_i32, [_cache_p, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _vp]),
     "loki_topk_jaccard": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp]),
+    "loki_device_error_count": (_i32, [ctypes.POINTER(ctypes.c_uint32)]),
     "loki_decode_launch_shape": (_i32, [_cache_p, _i32, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
     "loki_status_string": (ctypes.c_char_p, [_i32]),
     "loki_last_error": (ctypes.c_char_p, []),

@@ -12,6 +12,7 @@
 
 #include "loki.h"
 #include "append.cuh"
+#include "append_tc.cuh"
 #include "decode.cuh"
 #include "loki_step.cuh"
 #include "topk_stats.cuh"
@@ -437,6 +438,13 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   return dispatch_g<T, 128>(dense, di, sh, a, ws, stream, used);
 }
 
+template <int D>
+struct AppendTcGate {
+  static SmemGate gate;
+};
+template <int D>
+SmemGate AppendTcGate<D>::gate;
+
 template <typename T, int D>
 struct AppendGate {
   static SmemGate gate;
@@ -461,6 +469,23 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   a.pos = pos;
   a.n_new = n_new;
   a.n_vec = c->batch * n_new;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (a.n_vec >= kTcMinVectors) {
+      // a bulk append: the rotation is a GEMM per head, on the tensor cores
+      auto kern = append_tc_kernel<D>;
+      s = allow_smem(kern, di, AppendTcGate<D>::gate, false);
+      if (s != LOKI_OK) return s;
+      // persistent: one CTA per SM over the (head, tile) units
+      const long long units = (long long)c->n_kv_heads * ((a.n_vec + kTcM - 1) / kTcM);
+      if (units > INT32_MAX) return fail(LOKI_ERR_UNSUPPORTED, "bulk append of %d vectors per head is too large", a.n_vec);
+      a.per_cta = 0;
+      dim3 grid((unsigned)(units < di.sms ? units : di.sms), 1, 1);
+      kern<<<grid, kTcThreads, TcLayout<D>::kBytes, static_cast<cudaStream_t>(stream)>>>(a);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "append_tc_kernel launch");
+      return LOKI_OK;
+    }
+  }
   // enough CTAs to cover the SMs twice (heads x column blocks x chunks), at
   // least one 8-vector batch each
   const int col_blocks = D / kAppendCols;
@@ -587,6 +612,13 @@ loki_status loki_decode_attention_noalloc(const loki_cache *cache, int32_t seq_l
   if (s != LOKI_OK) return s;
   return loki_decode_attention(cache, seq_len, n_q_heads, q, P, d, k, scale, out, idx, scratch,
                                kNoAllocScratchBytes, stream);
+}
+
+loki_status loki_device_error_count(uint32_t *count) {
+  if (!count) return fail(LOKI_ERR_INVALID_ARG, "count is NULL");
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_loki_device_errors, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(device error count)");
+  return LOKI_OK;
 }
 
 loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_b, int32_t rows, int32_t k, float *jaccard,

@@ -108,7 +108,7 @@ def gamma(n: int) -> float:
     return n * u / (1 - n * u)
 
 
-def check_append(gpu_khat, keys64, P64, dtype: str) -> dict:
+def check_append(gpu_khat, keys64, P64, dtype: str, tensor_core: bool = False) -> dict:
     """GPU rotated keys vs exact fp64 rotation.  The GPU accumulates the D
     products in fp32 and rounds once to the cache dtype.  With
     bound = gamma_D * sum_i |k_i P_ij| (the fp32 dot-product error bound), the
@@ -116,10 +116,18 @@ def check_append(gpu_khat, keys64, P64, dtype: str) -> dict:
       fp32 cache: |gpu - exact| <= bound;
       bf16 cache: gpu = RNE_bf16(y) lies in [RNE(exact - bound), RNE(exact + bound)]
       (RNE is monotone); where it differs from RNE(exact) that is explained by
-      fp32 accumulation alone."""
+      fp32 accumulation alone.
+    tensor_core: the bulk path of bf16 caches splits P into three bf16 terms
+    (their sum is P to 2^-27 relative) and accumulates the 3*D exact products
+    in fp32 on the tensor cores, whose accumulation is not assumed to round to
+    nearest: bound = 2 * gamma_{3D} * sum_i |k_i P_ij| (+ the split residual)."""
     D = keys64.shape[-1]
     exact = np.einsum("bgti,gij->bgtj", keys64, P64)
-    bound = gamma(D) * np.einsum("bgti,gij->bgtj", np.abs(keys64), np.abs(P64)) + 1e-300
+    mag = np.einsum("bgti,gij->bgtj", np.abs(keys64), np.abs(P64))
+    if tensor_core:
+        bound = (2.0 * gamma(3 * D) + 2.0 ** -26) * mag + 1e-300
+    else:
+        bound = gamma(D) * mag + 1e-300
     g = np.asarray(gpu_khat, dtype=np.float64)
     if dtype == "f32":
         err = np.abs(g - exact)

@@ -28,7 +28,8 @@ def test_header_declares_the_abi():
     names = _declared()
     assert set(names) == {"loki_append", "loki_decode_workspace_size", "loki_decode_attention",
                           "loki_decode_attention_noalloc", "dense_decode_attention", "loki_decode_launch_shape",
-                          "loki_topk_jaccard", "loki_status_string", "loki_last_error", "loki_version"}
+                          "loki_topk_jaccard", "loki_device_error_count", "loki_status_string", "loki_last_error",
+                          "loki_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -49,7 +50,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 5
+    assert lib.loki_version() == 6
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -123,6 +124,10 @@ def test_workspace_size_and_validation(lib):
     assert lib.loki_decode_attention(*args, WS + 16, WSB, None) == 1       # not 256-byte aligned
     assert lib.loki_decode_attention(*args, WS, need - 1, None) == 1       # too small
     assert b"smaller" in lib.loki_last_error()
+
+
+def test_device_error_count_validation(lib):
+    assert lib.loki_device_error_count(None) == 1
 
 
 def test_jaccard_validation(lib):

@@ -7,6 +7,7 @@ both sides score exactly the same K_hat; the GPU append kernel is checked on its
 own against the exact rotation.
 """
 import contextlib
+import ctypes
 import os
 
 import numpy as np
@@ -84,13 +85,20 @@ def run_decode(w, S, d, k, ncta=None, scale=0.0, inp=None, P32=None, capacity=No
 
 
 # ----------------------------------------------------------------------------- append
+TC_MIN_VECTORS = 256   # bf16 appends of at least this many vectors per KV head run on the tensor cores
+
+
 @pytest.mark.parametrize("dtype,D,n_new,pos,B,Hkv", [
     ("bf16", 128, 1, 0, 2, 3),
     ("bf16", 128, 37, 5, 3, 2),
-    ("bf16", 128, 300, 100, 2, 2),
+    ("bf16", 128, 300, 100, 2, 2),     # tensor cores: 600 vectors, 5 tiles (ragged)
+    ("bf16", 128, 150, 3, 3, 5),       # tensor cores: 450 vectors
+    ("bf16", 128, 2048, 0, 1, 2),      # tensor cores: 16 full tiles
     ("bf16", 64, 9, 3, 1, 4),
+    ("bf16", 64, 257, 11, 1, 3),       # tensor cores, D = 64
     ("f32", 64, 1, 7, 2, 2),
     ("f32", 128, 41, 0, 2, 3),
+    ("f32", 128, 700, 2, 1, 2),        # fp32 caches stay on the CUDA cores
 ])
 def test_append_matches_exact_rotation(dtype, D, n_new, pos, B, Hkv):
     w = small_workload(dtype, D, 1, n_new, Hkv=Hkv, B=B)
@@ -105,13 +113,32 @@ def test_append_matches_exact_rotation(dtype, D, n_new, pos, B, Hkv):
     torch.cuda.synchronize()
     kh = cache.k_hat.to(torch.float64).cpu().numpy()
     vv = cache.v.to(torch.float64).cpu().numpy()
-    st = parity.check_append(kh[:, :, pos:pos + n_new], inp["keys64"], P32.astype(np.float64), dtype)
+    tc = dtype == "bf16" and B * n_new >= TC_MIN_VECTORS
+    st = parity.check_append(kh[:, :, pos:pos + n_new], inp["keys64"], P32.astype(np.float64), dtype,
+                             tensor_core=tc)
+    if tc:
+        n = ctypes.c_uint32(0)
+        L()._lib.check(L().load_library().loki_device_error_count(ctypes.byref(n)))
+        assert n.value == 0, "a bounded wait of the tensor-core append timed out"
     if dtype == "bf16":
         assert st["mismatch"] <= 0.05 * st["n"]   # sanity: most values round exactly like the oracle
     np.testing.assert_array_equal(vv[:, :, pos:pos + n_new], inp["values64"])
     # nothing outside [pos, pos + n_new) is touched
     assert np.all(kh[:, :, :pos] == 7.0) and np.all(kh[:, :, pos + n_new:] == 7.0)
     assert np.all(vv[:, :, :pos] == -3.0) and np.all(vv[:, :, pos + n_new:] == -3.0)
+
+
+def test_bulk_append_identity_basis_is_a_copy():
+    # the tensor-core path with P = I: the split terms are 1, 0, 0 and the
+    # products exact, so the cache must hold the keys bit for bit
+    w = small_workload("bf16", 128, 1, 1000)
+    inp = gen.decode_inputs(w, seq_len=1000)
+    P = torch.eye(128, dtype=torch.float32).expand(2, 128, 128).contiguous().to(DEV)
+    cache = L().LokiCache(2, 2, 128, 1000, dtype=torch.bfloat16, device=DEV)
+    L().loki_append(cache, 0, inp["keys"].to(DEV), inp["values"].to(DEV), P)
+    torch.cuda.synchronize()
+    assert torch.equal(cache.k_hat.cpu(), inp["keys"])
+    assert torch.equal(cache.v.cpu(), inp["values"])
 
 
 def test_append_identity_basis_is_a_copy():

@@ -185,6 +185,30 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def time_prefill(L, cache, k_pre, v_pre, P, stream, dev, reps: int = 5):
+    """Device time of the bulk append of the prompt (rewriting the same cache
+    rows), L2 flushed before each repetition; median over reps."""
+    import torch
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    ts = []
+    for i in range(reps + 2):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        L.loki_append(cache, 0, k_pre, v_pre, P)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1) * 1000.0)
+    us = float(np.median(ts))
+    nbytes = 4 * k_pre.numel() * k_pre.element_size()  # keys in, rotated keys out, values in, values out
+    return {"us": us, "vectors_per_kv_head": int(k_pre.shape[0] * k_pre.shape[2]), "bytes": nbytes,
+            "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "reps": reps,
+            "kernel": "append_tc_kernel" if (k_pre.dtype == torch.bfloat16
+                                             and k_pre.shape[0] * k_pre.shape[2] >= 256) else "append_kernel"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -217,7 +241,10 @@ def run_ours(args):
             k_pre[:, h] = gen.device_keys(gen.make_key_model(w, h), B, S - 1, g_dev, dev, td)
         v_pre = torch.randn((B, Hkv, S - 1, D), generator=g_dev, device=dev).to(td)
         L.loki_append(cache, 0, k_pre, v_pre, P)
+        prefill = time_prefill(L, cache, k_pre, v_pre, P, stream, dev)
         del k_pre, v_pre
+    else:
+        prefill = None
     NSET = 4
     qs = [torch.randn((B, Hq, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
     kn = [torch.randn((B, Hkv, 1, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
@@ -372,6 +399,7 @@ def run_ours(args):
                       "launch": {"cluster_ctas": dcl, "ctas": dct}},
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
             "append_us": app_us,
+            "prefill_append": None if prefill is None else dict(prefill, frac=prefill["hbm_gbs"] / peak),
             "exact_topk": {"us": t_exact * 1000.0 / ex_steps, "d": D, "k": w.k, "steps": ex_steps,
                            "jaccard_vs_loki": {"mean": float(jaccard.mean()), "min": float(jaccard.min()),
                                                "rows": int(jaccard.numel())}},

@@ -209,6 +209,26 @@ def time_prefill(L, cache, k_pre, v_pre, P, stream, dev, reps: int = 5):
                                              and k_pre.shape[0] * k_pre.shape[2] >= 256) else "append_kernel"}
 
 
+def time_pca(L, calib, dev, stream, reps: int = 3):
+    """Device time of the GPU calibration (loki_pca_calibrate) of every KV
+    head's basis from its calibration keys; median over reps."""
+    import torch
+    keys = torch.as_tensor(np.stack(calib).astype(np.float32)).to(dev)
+    H, N, D = keys.shape
+    ws = torch.empty(L.loki_pca_workspace_size(H, D), dtype=torch.uint8, device=dev)
+    L.loki_pca_calibrate(keys, workspace=ws)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        L.loki_pca_calibrate(keys, workspace=ws)
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1000.0)
+    return {"us": float(np.median(ts)), "heads": int(H), "keys_per_head": int(N), "reps": reps,
+            "kernels": "pca_mean_kernel, pca_cov_kernel, pca_jacobi_kernel"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -231,7 +251,9 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     # offline calibration (host) and cache prefill: S-1 tokens; each step appends token S-1
-    P = pca_bases([gen.calibration_keys(w, g) for g in range(Hkv)]).to(dev)
+    calib = [gen.calibration_keys(w, g) for g in range(Hkv)]
+    P = pca_bases(calib).to(dev)
+    pca = time_pca(L, calib, dev, stream)
     cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev)
     g_dev = torch.Generator(device=dev)
     g_dev.manual_seed(w.seed * 131 + rank)
@@ -400,6 +422,7 @@ def run_ours(args):
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
             "append_us": app_us,
             "prefill_append": None if prefill is None else dict(prefill, frac=prefill["hbm_gbs"] / peak),
+            "pca_calibrate": pca,
             "exact_topk": {"us": t_exact * 1000.0 / ex_steps, "d": D, "k": w.k, "steps": ex_steps,
                            "jaccard_vs_loki": {"mean": float(jaccard.mean()), "min": float(jaccard.min()),
                                                "rows": int(jaccard.numel())}},

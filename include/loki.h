@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 6
+#define LOKI_VERSION 7
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -188,6 +188,37 @@ LOKI_API loki_status loki_device_error_count(uint32_t *count);
  * Requires rows >= 1 and k >= 1.  One kernel on `stream`. */
 LOKI_API loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_b, int32_t rows,
                               int32_t k, float *jaccard, void *stream);
+
+/* loki_pca_workspace_size -- bytes of device workspace loki_pca_calibrate
+ * needs for n_heads heads of dimension head_dim (64 or 128): the per-head
+ * means and covariances in fp64.  *bytes is a host pointer. */
+LOKI_API loki_status loki_pca_workspace_size(int32_t n_heads, int32_t head_dim, size_t *bytes);
+
+/* loki_pca_calibrate -- the offline PCA calibration of the key basis, on the
+ * GPU (summary page, summary paragraph: the PCA transform is calibrated
+ * offline; section "Approach": queries and keys are projected with it).  For
+ * every head g, from its N calibration keys x_n:
+ *   C_g = (1/N) sum_n (x_n - mean)(x_n - mean)^T          (fp64)
+ *   P_g[:, j] = the unit eigenvector of C_g with the j-th largest eigenvalue,
+ *               its sign chosen so that its entry of largest magnitude is
+ *               positive (the first such entry on a tie), rounded to fp32.
+ * Equal eigenvalues are ordered by an unspecified but deterministic rule;
+ * for them only the span of their eigenvectors is defined.
+ *   keys      : [n_heads, n_keys, head_dim] in dtype (LOKI_F32 or LOKI_BF16),
+ *               16-byte aligned, read only.
+ *   P         : [n_heads, head_dim, head_dim] fp32, 16-byte aligned (written);
+ *               the layout loki_append and the decode calls take.
+ *   eigvals   : [n_heads, head_dim] fp64 in descending order (written), or
+ *               NULL.
+ *   workspace : device scratch of at least loki_pca_workspace_size bytes,
+ *               256-byte aligned; no initial contents needed.
+ * Three kernels on `stream`: means, covariance tiles, and a cyclic Jacobi
+ * eigensolver (one CTA per head, at most 30 sweeps).  This is a calibration
+ * step, not part of the decode path; it has no counterpart in the pages'
+ * kernels, which take P as given. */
+LOKI_API loki_status loki_pca_calibrate(const void *keys, int32_t dtype, int32_t n_heads,
+                               int32_t n_keys, int32_t head_dim, float *P, double *eigvals,
+                               void *workspace, size_t workspace_bytes, void *stream);
 
 /* Launch shape a decode call with these sizes would use, for logging and
  * tests.  shape: host array of 4 int32.

@@ -16,6 +16,8 @@ from .api import (
     loki_decode_attention_noalloc,
     loki_decode_launch_shape,
     loki_decode_workspace_size,
+    loki_pca_calibrate,
+    loki_pca_workspace_size,
     loki_status_string,
     loki_version,
     topk_jaccard,
@@ -33,6 +35,8 @@ __all__ = [
     "dense_decode_attention",
     "loki_decode_launch_shape",
     "loki_decode_workspace_size",
+    "loki_pca_calibrate",
+    "loki_pca_workspace_size",
     "loki_status_string",
     "loki_version",
     "topk_jaccard",

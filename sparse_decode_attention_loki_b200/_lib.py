@@ -47,6 +47,8 @@ SIGNATURES = {
     "loki_topk_jaccard": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp]),
     "loki_device_error_count": (_i32, [ctypes.POINTER(ctypes.c_uint32)]),
     "loki_decode_launch_shape": (_i32, [_cache_p, _i32, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
+    "loki_pca_workspace_size": (_i32, [_i32, _i32, ctypes.POINTER(ctypes.c_size_t)]),
+    "loki_pca_calibrate": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "loki_status_string": (ctypes.c_char_p, [_i32]),
     "loki_last_error": (ctypes.c_char_p, []),
     "loki_version": (_i32, []),

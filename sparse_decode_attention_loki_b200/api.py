@@ -184,6 +184,38 @@ def topk_jaccard(idx_a: torch.Tensor, idx_b: torch.Tensor, stream: Optional[torc
     return out
 
 
+def loki_pca_workspace_size(n_heads: int, head_dim: int) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check(_lib.load().loki_pca_workspace_size(int(n_heads), int(head_dim), ctypes.byref(n)))
+    return int(n.value)
+
+
+def loki_pca_calibrate(keys: torch.Tensor, stream: Optional[torch.cuda.Stream] = None,
+                       workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """PCA basis of each head from its calibration keys, on the GPU.
+
+    keys: [H, N, D] fp32 or bf16 CUDA tensor.  Returns (P [H, D, D] fp32,
+    eigenvalues [H, D] fp64, descending); column j of P[g] is the j-th
+    principal direction, its largest-magnitude entry positive."""
+    if keys.dim() != 3 or keys.device.type != "cuda" or not keys.is_contiguous():
+        raise ValueError("keys must be a contiguous [H, N, D] CUDA tensor")
+    if keys.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"keys dtype {keys.dtype} (float32 or bfloat16)")
+    H, N, D = (int(x) for x in keys.shape)
+    dev = keys.device
+    need = loki_pca_workspace_size(H, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    P = torch.empty((H, D, D), dtype=torch.float32, device=dev)
+    w = torch.empty((H, D), dtype=torch.float64, device=dev)
+    dt = _lib.LOKI_F32 if keys.dtype == torch.float32 else _lib.LOKI_BF16
+    with torch.cuda.device(dev):
+        _lib.check(_lib.load().loki_pca_calibrate(_ptr(keys), dt, H, N, D, _ptr(P), _ptr(w), _ptr(workspace),
+                                                  workspace.numel() * workspace.element_size(),
+                                                  _stream_ptr(dev, stream)))
+    return P, w
+
+
 def loki_decode_launch_shape(cache: LokiCache, seq_len: int, n_q_heads: int, k: int = 1,
                              dense: bool = False) -> Tuple[int, int, int, int]:
     """Grid sizes of a decode call.  Loki: (rotation CTAs, decode CTAs per row

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libloki.so")
 
 SOURCES = ["loki_api.cu"]
-HEADERS = ["common.cuh", "decode.cuh", "append.cuh", "append_tc.cuh", "loki_step.cuh", "topk_stats.cuh"]
+HEADERS = ["common.cuh", "decode.cuh", "append.cuh", "append_tc.cuh", "loki_step.cuh", "pca.cuh", "topk_stats.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -15,6 +15,7 @@
 #include "append_tc.cuh"
 #include "decode.cuh"
 #include "loki_step.cuh"
+#include "pca.cuh"
 #include "topk_stats.cuh"
 
 namespace {
@@ -539,6 +540,60 @@ loki_status noalloc_scratch(void **addr) {
   return LOKI_OK;
 }
 
+// PCA workspace: per-head means [H, D] then covariances [H, D, D], fp64,
+// each region 256-byte aligned.
+struct PcaWs {
+  size_t mean, cov, total;
+};
+PcaWs pca_ws(long long heads, int D) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  PcaWs w;
+  w.mean = 0;
+  w.cov = up((size_t)heads * D * sizeof(double));
+  w.total = w.cov + up((size_t)heads * D * D * sizeof(double));
+  return w;
+}
+
+template <int D>
+struct PcaGate {
+  static SmemGate gate;
+};
+template <int D>
+SmemGate PcaGate<D>::gate;
+
+template <typename T, int D>
+loki_status run_pca(const T *keys, int32_t H, int32_t N, float *P, double *eigvals, void *ws, void *stream) {
+  DevInfo di;
+  loki_status s = device_info(&di);
+  if (s != LOKI_OK) return s;
+  const PcaWs w = pca_ws(H, D);
+  PcaArgs<T> a;
+  a.keys = keys;
+  a.n_heads = H;
+  a.n_keys = N;
+  a.mean = reinterpret_cast<double *>(static_cast<unsigned char *>(ws) + w.mean);
+  a.cov = reinterpret_cast<double *>(static_cast<unsigned char *>(ws) + w.cov);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  constexpr int NT = D / kPcaTile;
+  pca_mean_kernel<T, D><<<dim3((unsigned)H, NT), 256, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pca_mean_kernel launch");
+  pca_cov_kernel<T, D><<<dim3((unsigned)H, NT * (NT + 1) / 2), 256, 0, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pca_cov_kernel launch");
+  auto kern = pca_jacobi_kernel<D>;
+  s = allow_smem(kern, di, PcaGate<D>::gate, false);
+  if (s != LOKI_OK) return s;
+  PcaEigArgs ea;
+  ea.cov = a.cov;
+  ea.P = P;
+  ea.eigvals = eigvals;
+  kern<<<(unsigned)H, kPcaThreads, PcaSmem<D>::kBytes, st>>>(ea);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pca_jacobi_kernel launch");
+  return LOKI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -676,6 +731,40 @@ loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, i
   shape[2] = (int32_t)(rows * pl.ncta);
   shape[3] = 0;
   return LOKI_OK;
+}
+
+loki_status loki_pca_workspace_size(int32_t n_heads, int32_t head_dim, size_t *bytes) {
+  if (!bytes) return fail(LOKI_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_heads < 1 || n_heads > 65535) return fail(LOKI_ERR_INVALID_ARG, "n_heads=%d outside [1, 65535]", n_heads);
+  if (head_dim != 64 && head_dim != 128) return fail(LOKI_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", head_dim);
+  *bytes = pca_ws(n_heads, head_dim).total;
+  return LOKI_OK;
+}
+
+loki_status loki_pca_calibrate(const void *keys, int32_t dtype, int32_t n_heads, int32_t n_keys, int32_t head_dim,
+                               float *P, double *eigvals, void *workspace, size_t workspace_bytes, void *stream) {
+  size_t need = 0;
+  loki_status s = loki_pca_workspace_size(n_heads, head_dim, &need);
+  if (s != LOKI_OK) return s;
+  if (dtype != LOKI_F32 && dtype != LOKI_BF16) return fail(LOKI_ERR_INVALID_ARG, "dtype %d", dtype);
+  if (n_keys < 1) return fail(LOKI_ERR_INVALID_ARG, "n_keys=%d must be >= 1", n_keys);
+  if ((long long)n_keys * head_dim > INT32_MAX) return fail(LOKI_ERR_UNSUPPORTED, "n_keys=%d too large", n_keys);
+  if (!keys || !P || !workspace) return fail(LOKI_ERR_INVALID_ARG, "keys, P or workspace is NULL");
+  if (!aligned(keys, 16) || !aligned(P, 16) || (eigvals && !aligned(eigvals, 8)))
+    return fail(LOKI_ERR_INVALID_ARG, "keys and P must be 16-byte aligned, eigvals 8-byte aligned");
+  if (!aligned(workspace, 256)) return fail(LOKI_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(LOKI_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes this call needs",
+                workspace_bytes, need);
+  if (dtype == LOKI_F32)
+    return head_dim == 64 ? run_pca<float, 64>(static_cast<const float *>(keys), n_heads, n_keys, P, eigvals,
+                                               workspace, stream)
+                          : run_pca<float, 128>(static_cast<const float *>(keys), n_heads, n_keys, P, eigvals,
+                                                workspace, stream);
+  return head_dim == 64 ? run_pca<__nv_bfloat16, 64>(static_cast<const __nv_bfloat16 *>(keys), n_heads, n_keys, P,
+                                                     eigvals, workspace, stream)
+                        : run_pca<__nv_bfloat16, 128>(static_cast<const __nv_bfloat16 *>(keys), n_heads, n_keys, P,
+                                                      eigvals, workspace, stream);
 }
 
 const char *loki_status_string(loki_status s) {

@@ -28,8 +28,8 @@ def test_header_declares_the_abi():
     names = _declared()
     assert set(names) == {"loki_append", "loki_decode_workspace_size", "loki_decode_attention",
                           "loki_decode_attention_noalloc", "dense_decode_attention", "loki_decode_launch_shape",
-                          "loki_topk_jaccard", "loki_device_error_count", "loki_status_string", "loki_last_error",
-                          "loki_version"}
+                          "loki_topk_jaccard", "loki_device_error_count", "loki_pca_workspace_size",
+                          "loki_pca_calibrate", "loki_status_string", "loki_last_error", "loki_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -50,7 +50,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 6
+    assert lib.loki_version() == 7
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -136,6 +136,41 @@ def test_jaccard_validation(lib):
     assert lib.loki_topk_jaccard(None, FAKE, 3, 4, FAKE, None) == 1
     assert lib.loki_topk_jaccard(FAKE, FAKE + 2, 3, 4, FAKE, None) == 1
     assert lib.loki_topk_jaccard(FAKE, FAKE, 3, 4, None, None) == 1
+
+
+def _pca_ws_bytes(H, D):
+    """Means [H, D] then covariances [H, D, D], fp64, each region padded to 256 bytes."""
+    a = lambda x: (x + 255) // 256 * 256
+    return a(H * D * 8) + a(H * D * D * 8)
+
+
+def test_pca_workspace_size_and_validation(lib):
+    n = ctypes.c_size_t(0)
+    for H, D in [(1, 64), (8, 128), (32, 128), (3, 64)]:
+        assert lib.loki_pca_workspace_size(H, D, ctypes.byref(n)) == 0
+        assert n.value == _pca_ws_bytes(H, D)
+    assert lib.loki_pca_workspace_size(0, 128, ctypes.byref(n)) == 1
+    assert lib.loki_pca_workspace_size(2, 96, ctypes.byref(n)) == 2
+    assert lib.loki_pca_workspace_size(2, 128, None) == 1
+    need = _pca_ws_bytes(2, 128)
+    ok = (FAKE, 0, 2, 100, 128, FAKE, FAKE, WS, need, None)
+    def call(**kw):
+        names = ["keys", "dtype", "H", "N", "D", "P", "w", "ws", "wsb", "stream"]
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return lib.loki_pca_calibrate(*[args[k] for k in names])
+    assert call(dtype=2) == 1
+    assert call(N=0) == 1
+    assert call(D=32) == 2
+    assert call(H=0) == 1
+    assert call(keys=None) == 1
+    assert call(P=None) == 1
+    assert call(ws=None) == 1
+    assert call(keys=FAKE + 8) == 1      # not 16-byte aligned
+    assert call(w=FAKE + 4) == 1         # eigenvalues not 8-byte aligned
+    assert call(ws=WS + 64) == 1         # workspace not 256-byte aligned
+    assert call(wsb=need - 1) == 1
+    assert b"smaller" in lib.loki_last_error()
 
 
 @pytest.mark.parametrize("pos,n_new,status", [(-1, 1, 1), (0, 0, 1), (60, 5, 1), (64, 1, 1)])

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 7
+#define LOKI_VERSION 8
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -188,6 +188,89 @@ LOKI_API loki_status loki_device_error_count(uint32_t *count);
  * Requires rows >= 1 and k >= 1.  One kernel on `stream`. */
 LOKI_API loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_b, int32_t rows,
                               int32_t k, float *jaccard, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Paged caches and per-sequence lengths
+ * ------------------------------------------------------------------------
+ * The pages name the missing integration with paged serving kernels as a
+ * limitation (summary page, section "Limitations": not yet integrated with
+ * FlashAttention; PagedAttention is among its references).  These calls run
+ * the same Loki step on a paged cache whose sequences have their own lengths;
+ * the per-row computation is exactly that of loki_decode_attention on the
+ * sequence's tokens 0 .. seq_lens[b]-1 in order.
+ *
+ * A paged rotated-key cache: fixed-size pages from one pool.
+ *   k_hat : [num_pages, Hkv, page_size, D] rotated keys in `dtype`, 16-byte
+ *           aligned; v : the same layout, values.
+ * page_size is a power of two, 1 .. 65536 tokens. */
+typedef struct {
+  int32_t dtype;       /* loki_dtype                                          */
+  int32_t n_kv_heads;  /* Hkv >= 1                                            */
+  int32_t head_dim;    /* D: 64 or 128                                        */
+  int32_t page_size;   /* tokens per page, a power of two                     */
+  int32_t num_pages;   /* pages in each pool, >= 1                            */
+  void *k_hat;
+  void *v;
+} loki_paged_cache;
+
+/* The sequences of a batch in a paged cache.
+ *   block_table : [batch, pages_per_seq] int32 device array: token t of
+ *                 sequence b sits at slot t % page_size of page
+ *                 block_table[b][t / page_size].  Ids outside
+ *                 [0, num_pages) are clamped into it (never an out-of-bounds
+ *                 access; the result is then unspecified).
+ *   seq_lens    : [batch] int32 device array, tokens attended per sequence,
+ *                 each in [1, max_seq_len] (values outside are clamped), or
+ *                 NULL for max_seq_len everywhere.  Ignored by
+ *                 loki_paged_append.
+ *   max_seq_len : the largest length, 1 <= max_seq_len <= pages_per_seq *
+ *                 page_size; launch shapes are planned for it. */
+typedef struct {
+  int32_t batch;          /* B >= 1                                           */
+  int32_t pages_per_seq;  /* columns of block_table, >= 1                     */
+  int32_t max_seq_len;
+  const int32_t *block_table;
+  const int32_t *seq_lens;
+} loki_seq_table;
+
+/* loki_paged_append -- loki_append for a paged cache: new vector t of
+ * sequence b (k_new[b, :, t, :] rotated by P, v_new[b, :, t, :] as is) goes to
+ * token pos[b] + t of sequence b.  pos: [batch] int32 device array.  Tokens
+ * whose position is negative or beyond the sequence's pages_per_seq *
+ * page_size are not written.  Same arithmetic and kernels as loki_append
+ * (tensor cores for bf16 appends of at least 256 vectors per KV head). */
+LOKI_API loki_status loki_paged_append(const loki_paged_cache *cache, const loki_seq_table *seqs,
+                              const int32_t *pos, int32_t n_new, const void *k_new,
+                              const void *v_new, const float *P, void *stream);
+
+/* Workspace bytes of loki_paged_decode_attention (same rule as
+ * loki_decode_workspace_size for B = seqs->batch). */
+LOKI_API loki_status loki_paged_decode_workspace_size(const loki_paged_cache *cache,
+                                             const loki_seq_table *seqs, int32_t n_q_heads,
+                                             size_t *bytes);
+
+/* loki_paged_decode_attention -- the Loki step of loki_decode_attention on a
+ * paged cache with per-sequence lengths.
+ *   ks    : [batch] int32 device array: tokens kept for sequence b, clamped
+ *           into [1, min(seq_lens[b], k_max)]; or NULL for
+ *           min(seq_lens[b], k_max) everywhere.
+ *   k_max : 1 <= k_max <= max_seq_len; the length of each idx row.
+ *   idx   : [B, Hkv, k_max] int32 (written): row (b, g) holds the k_b
+ *           selected positions in ascending order, then -1 up to k_max.
+ * Everything else as loki_decode_attention (out [B, Hq, D] fp32, workspace of
+ * loki_paged_decode_workspace_size bytes, two kernels on `stream`). */
+LOKI_API loki_status loki_paged_decode_attention(const loki_paged_cache *cache,
+                                        const loki_seq_table *seqs, int32_t n_q_heads,
+                                        const void *q, const float *P, int32_t d,
+                                        const int32_t *ks, int32_t k_max, float scale,
+                                        float *out, int32_t *idx, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/* dense_decode_attention on a paged cache with per-sequence lengths. */
+LOKI_API loki_status dense_paged_decode_attention(const loki_paged_cache *cache,
+                                         const loki_seq_table *seqs, int32_t n_q_heads,
+                                         const void *q, const float *P, float scale,
+                                         float *out, void *stream);
 
 /* loki_pca_workspace_size -- bytes of device workspace loki_pca_calibrate
  * needs for n_heads heads of dimension head_dim (64 or 128): the per-head

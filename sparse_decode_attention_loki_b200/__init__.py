@@ -10,12 +10,17 @@ C ABI of include/loki.h (libloki.so); this package is its Python binding.
 from ._lib import LIB_PATH, LokiError, load as load_library
 from .api import (
     LokiCache,
+    PagedLokiCache,
+    SeqTable,
     dense_decode_attention,
+    dense_paged_decode_attention,
     loki_append,
     loki_decode_attention,
     loki_decode_attention_noalloc,
     loki_decode_launch_shape,
     loki_decode_workspace_size,
+    loki_paged_append,
+    loki_paged_decode_attention,
     loki_pca_calibrate,
     loki_pca_workspace_size,
     loki_status_string,
@@ -29,6 +34,11 @@ __all__ = [
     "LokiError",
     "load_library",
     "LokiCache",
+    "PagedLokiCache",
+    "SeqTable",
+    "loki_paged_append",
+    "loki_paged_decode_attention",
+    "dense_paged_decode_attention",
     "loki_append",
     "loki_decode_attention",
     "loki_decode_attention_noalloc",

@@ -31,9 +31,33 @@ class loki_cache(ctypes.Structure):
     ]
 
 
+class loki_paged_cache(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("k_hat", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+    ]
+
+
+class loki_seq_table(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("pages_per_seq", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32),
+        ("block_table", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+    ]
+
+
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
 _cache_p = ctypes.POINTER(loki_cache)
+_pcache_p = ctypes.POINTER(loki_paged_cache)
+_seqs_p = ctypes.POINTER(loki_seq_table)
 
 # name -> (restype, argtypes); every entry point of include/loki.h
 SIGNATURES = {
@@ -47,6 +71,11 @@ SIGNATURES = {
     "loki_topk_jaccard": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp]),
     "loki_device_error_count": (_i32, [ctypes.POINTER(ctypes.c_uint32)]),
     "loki_decode_launch_shape": (_i32, [_cache_p, _i32, _i32, _i32, _i32, ctypes.POINTER(_i32)]),
+    "loki_paged_append": (_i32, [_pcache_p, _seqs_p, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "loki_paged_decode_workspace_size": (_i32, [_pcache_p, _seqs_p, _i32, ctypes.POINTER(ctypes.c_size_t)]),
+    "loki_paged_decode_attention": (_i32, [_pcache_p, _seqs_p, _i32, _vp, _vp, _i32, _vp, _i32, ctypes.c_float, _vp,
+                                           _vp, _vp, ctypes.c_size_t, _vp]),
+    "dense_paged_decode_attention": (_i32, [_pcache_p, _seqs_p, _i32, _vp, _vp, ctypes.c_float, _vp, _vp]),
     "loki_pca_workspace_size": (_i32, [_i32, _i32, ctypes.POINTER(ctypes.c_size_t)]),
     "loki_pca_calibrate": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "loki_status_string": (ctypes.c_char_p, [_i32]),

@@ -184,6 +184,120 @@ def topk_jaccard(idx_a: torch.Tensor, idx_b: torch.Tensor, stream: Optional[torc
     return out
 
 
+class PagedLokiCache:
+    """A paged rotated-key cache: pools k_hat and v of shape
+    [num_pages, Hkv, page_size, D] shared by the sequences of a batch through a
+    page table (see SeqTable)."""
+
+    def __init__(self, num_pages: int, n_kv_heads: int, head_dim: int, page_size: int,
+                 dtype: torch.dtype = torch.bfloat16, device=None,
+                 k_hat: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None):
+        if dtype not in _DTYPES:
+            raise ValueError(f"cache dtype must be float32 or bfloat16, got {dtype}")
+        device = torch.device(device if device is not None else "cuda")
+        if device.type != "cuda":
+            raise ValueError("the cache must live in CUDA device memory")
+        if device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        shape = (num_pages, n_kv_heads, page_size, head_dim)
+        self.k_hat = k_hat if k_hat is not None else torch.empty(shape, dtype=dtype, device=device)
+        self.v = v if v is not None else torch.empty(shape, dtype=dtype, device=device)
+        _need(self.k_hat, "k_hat", dtype, shape, device)
+        _need(self.v, "v", dtype, shape, device)
+        self.num_pages, self.n_kv_heads, self.head_dim, self.page_size = num_pages, n_kv_heads, head_dim, page_size
+        self.dtype = dtype
+        self.device = device
+        self._desc = _lib.loki_paged_cache(_DTYPES[dtype], n_kv_heads, head_dim, page_size, num_pages,
+                                           self.k_hat.data_ptr(), self.v.data_ptr())
+
+    def desc(self):
+        return ctypes.byref(self._desc)
+
+
+class SeqTable:
+    """The sequences of a batch in a paged cache: block_table [B, pages_per_seq]
+    int32 page ids and seq_lens [B] int32 (or None: max_seq_len everywhere),
+    both on the cache's device."""
+
+    def __init__(self, block_table: torch.Tensor, seq_lens: Optional[torch.Tensor], max_seq_len: int):
+        if block_table.dim() != 2 or block_table.dtype != torch.int32 or not block_table.is_contiguous():
+            raise ValueError("block_table must be a contiguous [B, pages_per_seq] int32 tensor")
+        B = int(block_table.shape[0])
+        if seq_lens is not None:
+            _need(seq_lens, "seq_lens", torch.int32, (B,), block_table.device)
+        self.block_table, self.seq_lens, self.max_seq_len = block_table, seq_lens, int(max_seq_len)
+        self.batch, self.pages_per_seq = B, int(block_table.shape[1])
+        self._desc = _lib.loki_seq_table(B, self.pages_per_seq, self.max_seq_len, block_table.data_ptr(),
+                                         seq_lens.data_ptr() if seq_lens is not None else None)
+
+    def desc(self):
+        return ctypes.byref(self._desc)
+
+
+def loki_paged_append(cache: PagedLokiCache, seqs: SeqTable, pos: torch.Tensor, k_new: torch.Tensor,
+                      v_new: torch.Tensor, P: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Rotate k_new [B, Hkv, n_new, D] by P and write it with v_new at tokens
+    pos[b] .. pos[b] + n_new - 1 of each sequence b (pos: [B] int32)."""
+    n_new = k_new.shape[2] if k_new.dim() == 4 else -1
+    shp = (seqs.batch, cache.n_kv_heads, n_new, cache.head_dim)
+    _need(k_new, "k_new", cache.dtype, shp, cache.device)
+    _need(v_new, "v_new", cache.dtype, shp, cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    _need(pos, "pos", torch.int32, (seqs.batch,), cache.device)
+    _lib.check(_lib.load().loki_paged_append(cache.desc(), seqs.desc(), _ptr(pos), int(n_new), _ptr(k_new),
+                                             _ptr(v_new), _ptr(P), _stream_ptr(cache.device, stream)))
+
+
+def loki_paged_decode_attention(cache: PagedLokiCache, seqs: SeqTable, q: torch.Tensor, P: torch.Tensor, d: int,
+                                k_max: int, ks: Optional[torch.Tensor] = None, scale: float = 0.0,
+                                out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                                workspace: Optional[torch.Tensor] = None,
+                                stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The Loki step on a paged cache with per-sequence lengths.  Returns
+    (out [B, Hq, D] fp32, idx [B, Hkv, k_max] int32, -1 past each row's k)."""
+    B, Hkv, D = seqs.batch, cache.n_kv_heads, cache.head_dim
+    if q.dim() != 3 or q.shape[0] != B or q.shape[2] != D:
+        raise ValueError(f"q must be [B={B}, Hq, D={D}], got {tuple(q.shape)}")
+    Hq = int(q.shape[1])
+    _need(q, "q", cache.dtype, (B, Hq, D), cache.device)
+    _need(P, "P", torch.float32, (Hkv, D, D), cache.device)
+    if ks is not None:
+        _need(ks, "ks", torch.int32, (B,), cache.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=cache.device)
+    if idx is None:
+        idx = torch.empty((B, Hkv, int(k_max)), dtype=torch.int32, device=cache.device)
+    _need(out, "out", torch.float32, (B, Hq, D), cache.device)
+    _need(idx, "idx", torch.int32, (B, Hkv, int(k_max)), cache.device)
+    n = ctypes.c_size_t(0)
+    lib = _lib.load()
+    _lib.check(lib.loki_paged_decode_workspace_size(cache.desc(), seqs.desc(), Hq, ctypes.byref(n)))
+    if workspace is None or workspace.numel() * workspace.element_size() < n.value:
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=cache.device)
+    _lib.check(lib.loki_paged_decode_attention(cache.desc(), seqs.desc(), Hq, _ptr(q), _ptr(P), int(d),
+                                               _ptr(ks) if ks is not None else None, int(k_max), float(scale),
+                                               _ptr(out), _ptr(idx), _ptr(workspace),
+                                               workspace.numel() * workspace.element_size(),
+                                               _stream_ptr(cache.device, stream)))
+    return out, idx
+
+
+def dense_paged_decode_attention(cache: PagedLokiCache, seqs: SeqTable, q: torch.Tensor, P: torch.Tensor,
+                                 scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Full attention over each sequence's seq_lens[b] tokens of a paged cache."""
+    B, D = seqs.batch, cache.head_dim
+    Hq = int(q.shape[1]) if q.dim() == 3 else -1
+    _need(q, "q", cache.dtype, (B, Hq, D), cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, D, D), cache.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=cache.device)
+    _need(out, "out", torch.float32, (B, Hq, D), cache.device)
+    _lib.check(_lib.load().dense_paged_decode_attention(cache.desc(), seqs.desc(), Hq, _ptr(q), _ptr(P),
+                                                        float(scale), _ptr(out), _stream_ptr(cache.device, stream)))
+    return out
+
+
 def loki_pca_workspace_size(n_heads: int, head_dim: int) -> int:
     n = ctypes.c_size_t(0)
     _lib.check(_lib.load().loki_pca_workspace_size(int(n_heads), int(head_dim), ctypes.byref(n)))

@@ -30,14 +30,37 @@ struct AppendArgs {
   int32_t n_new;
   int32_t n_vec;     // B * n_new vectors per KV head
   int32_t per_cta;   // vectors per CTA (multiple of kAppendBatch)
+  // paged cache (PAGED instantiations): pools [num_pages, Hkv, page, D], new
+  // vector t of sequence b goes to token pos_arr[b] + t of its page table
+  const int32_t *pos_arr;  // [B]
+  const int32_t *table;    // [B, pages_per_seq]
+  int32_t pages_per_seq;
+  int32_t page_shift;      // page size = 1 << page_shift tokens
+  int32_t num_pages;
 };
+
+// Element offset in the cache of new vector t of sequence b, head g; -1 when
+// a paged sequence's position falls outside its page table (not written).
+// Page ids are clamped into the pool.
+template <typename T, int D, bool PAGED>
+__device__ __forceinline__ long long append_dst(const AppendArgs<T> &a, int b, int g, int t) {
+  if constexpr (!PAGED) {
+    return (((long long)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * D;
+  } else {
+    const int tok = __ldg(a.pos_arr + b) + t;
+    if (tok < 0 || (tok >> a.page_shift) >= a.pages_per_seq) return -1;
+    const int p =
+        min(max(__ldg(a.table + (size_t)b * a.pages_per_seq + (tok >> a.page_shift)), 0), a.num_pages - 1);
+    return ((((long long)p * a.n_kv_heads + g) << a.page_shift) + (tok & ((1 << a.page_shift) - 1))) * D;
+  }
+}
 
 constexpr int kAppendBatch = kWarps;   // vectors per batch: one per warp
 constexpr int kAppendCols = 32;        // output columns per CTA: one per lane
 
 __host__ __device__ inline int append_smem_words(int D) { return D * kAppendCols + kAppendBatch * D; }
 
-template <typename T, int D>
+template <typename T, int D, bool PAGED>
 __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendArgs<T> a) {
   extern __shared__ __align__(16) float asmem[];
   float *Ps = asmem;                   // [D][32]: columns cb*32 .. cb*32+31 of P_g
@@ -82,7 +105,8 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
     const int f = f0 + warp;
     if (f < f_end) {
       const int b = f / a.n_new, t = f % a.n_new;
-      from_f32(acc, a.k_hat + (((size_t)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * D + j);
+      const long long off = append_dst<T, D, PAGED>(a, b, g, t);
+      if (off >= 0) from_f32(acc, a.k_hat + off + j);
     }
   }
 
@@ -96,9 +120,8 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
     const int b = f / a.n_new, t = f % a.n_new;
     const uint4 *src = reinterpret_cast<const uint4 *>(
         a.v_new + (((size_t)b * a.n_kv_heads + g) * a.n_new + t) * D) + c;
-    uint4 *dst = reinterpret_cast<uint4 *>(
-        a.v + (((size_t)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * D) + c;
-    *dst = __ldg(src);
+    const long long off = append_dst<T, D, PAGED>(a, b, g, t);
+    if (off >= 0) reinterpret_cast<uint4 *>(a.v + off)[c] = __ldg(src);
   }
 }
 

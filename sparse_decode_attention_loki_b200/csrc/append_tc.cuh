@@ -149,7 +149,7 @@ __device__ __forceinline__ void tile_row(int n_new, int b0, int t0, int r, int &
   }
 }
 
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_constant__ AppendArgs<__nv_bfloat16> a) {
   using Lay = TcLayout<D>;
   constexpr int CH = D / 8;                 // 16-byte chunks per vector
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_c
   // offsets (in elements) of vector (b, t) of head g in the new-vector
   // arrays and in the cache
   auto src_off = [&](int g, int b, int t) { return (((size_t)b * a.n_kv_heads + g) * a.n_new + t) * D; };
-  auto dst_off = [&](int g, int b, int t) { return (((size_t)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * D; };
+  auto dst_off = [&](int g, int b, int t) { return append_dst<__nv_bfloat16, D, PAGED>(a, b, g, t); };
 
   // keys of unit u into stage `st` (rows past n_vec are zero); always one
   // commit group, empty when u is past the range
@@ -233,7 +233,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_c
       const int b0 = f0 / a.n_new;
       int b, t;
       tile_row(a.n_new, b0, f0 - b0 * a.n_new, r, b, t);
-      dst = a.k_hat + dst_off(g, b, t) + col0;
+      const long long off = dst_off(g, b, t);
+      if (off >= 0) dst = a.k_hat + off + col0;
     }
 #pragma unroll
     for (int cb = 0; cb < QC / 16; ++cb) {
@@ -330,7 +331,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_c
       if (f0 + r < a.n_vec) {
         int b, t;
         tile_row(a.n_new, b0, t0, r, b, t);
-        reinterpret_cast<uint4 *>(a.v + dst_off(g, b, t))[cch] = vv[x];
+        const long long off = dst_off(g, b, t);
+        if (off >= 0) reinterpret_cast<uint4 *>(a.v + off)[cch] = vv[x];
       }
     }
     pending = true;

@@ -27,8 +27,8 @@ namespace loki {
 
 template <typename T>
 struct DecodeArgs {
-  const T *k_hat;      // [B, Hkv, S_cap, D]
-  const T *v;          // [B, Hkv, S_cap, D]
+  const T *k_hat;      // [B, Hkv, S_cap, D]; paged: [num_pages, Hkv, page_size, D]
+  const T *v;          // same layout as k_hat
   const T *q;          // [B, Hq, D]
   const float *P;      // [Hkv, D, D]
   float *out;          // [B, Hq, D]
@@ -42,7 +42,72 @@ struct DecodeArgs {
   int32_t lpt;         // 16-byte chunks per token in the score stream (power of two)
   int32_t nck;         // chunks that hold the first d dims: ceil(d / elements per chunk)
   float scale_log2;    // softmax scale * log2(e)
+  // per-sequence lengths (null: every row has seq_len tokens and k picks);
+  // seq_len and k are then the largest values, and idx rows are k_stride long
+  const int32_t *seq_lens;  // [B] or null
+  const int32_t *ks;        // [B] or null
+  int32_t k_stride;         // entries per idx row (= k without per-sequence k)
+  // paged cache (used by the PAGED instantiations only)
+  const int32_t *table;     // [B, pages_per_seq] page ids
+  int32_t pages_per_seq;
+  int32_t page_shift;       // page size = 1 << page_shift tokens
+  int32_t num_pages;
 };
+
+// Tokens of one (batch, KV head) row, by position.  Contiguous caches: rows
+// of [B, Hkv, S_cap, D].  Paged caches: token t lives in page
+// table[t >> shift] (clamped into the pool) at slot t & (page - 1), the pool
+// laid out [num_pages, Hkv, page, D].
+template <typename T, int D, bool PAGED>
+struct Rows {
+  const T *k, *v;        // contiguous: the row's token 0; paged: the pools
+  const int32_t *table;  // paged: this sequence's page ids
+  int32_t shift, hkv, g, last_page;
+  __device__ __forceinline__ size_t off(int t) const {
+    if constexpr (!PAGED) {
+      return (size_t)t * D;
+    } else {
+      const int p = min(max(__ldg(table + (t >> shift)), 0), last_page);
+      return ((((size_t)p * hkv + g) << shift) + (size_t)(t & ((1 << shift) - 1))) * D;
+    }
+  }
+  __device__ __forceinline__ const T *key(int t) const { return k + off(t); }
+  __device__ __forceinline__ const T *val(int t) const { return v + off(t); }
+};
+
+template <typename T, int D, bool PAGED>
+__device__ __forceinline__ Rows<T, D, PAGED> make_rows(const DecodeArgs<T> &a, int b, int g) {
+  Rows<T, D, PAGED> r;
+  if constexpr (PAGED) {
+    r.k = a.k_hat;
+    r.v = a.v;
+    r.table = a.table + (size_t)b * a.pages_per_seq;
+    r.shift = a.page_shift;
+    r.hkv = a.n_kv_heads;
+    r.g = g;
+    r.last_page = a.num_pages - 1;
+  } else {
+    const size_t off = ((size_t)b * a.n_kv_heads + g) * a.capacity * D;
+    r.k = a.k_hat + off;
+    r.v = a.v + off;
+    r.table = nullptr;
+    r.shift = r.hkv = r.g = r.last_page = 0;
+  }
+  return r;
+}
+
+// Tokens attended by batch entry b: its own length when lengths are given
+// (clamped into [1, seq_len]), else seq_len.
+template <typename T>
+__device__ __forceinline__ int row_seq_len(const DecodeArgs<T> &a, int b) {
+  return a.seq_lens ? min(max(__ldg(a.seq_lens + b), 1), a.seq_len) : a.seq_len;
+}
+// Tokens selected for batch entry b: its own k when given, else k; clamped
+// into [1, min(S_b, k)].
+template <typename T>
+__device__ __forceinline__ int row_k(const DecodeArgs<T> &a, int b, int S_b) {
+  return a.ks ? min(max(__ldg(a.ks + b), 1), min(S_b, a.k)) : min(S_b, a.k);
+}
 
 // ---------------------------------------------------------------------------
 // shared memory
@@ -166,7 +231,8 @@ struct ScoreStream {
   static constexpr int TPW = 32 / LPT;        // tokens per warp instruction
   static_assert(TS >= TPW && TS % TPW == 0, "a stage must hold whole warp steps");
 
-  __device__ __forceinline__ static void issue(const T *Krow, int t0, int len, int nck, int s,
+  template <class R>
+  __device__ __forceinline__ static void issue(const R &rows, int t0, int len, int nck, int s,
                                                unsigned char *wring) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char *st = wring + (s % NS) * SB;
@@ -175,7 +241,7 @@ struct ScoreStream {
     for (int it = 0; it < TS * LPT / 32; ++it) {
       const int q = it * 32 + lane;
       const int t = q / LPT, c = q % LPT;
-      if (base + t < len && c < nck) cp_async16(st + q * 16, Krow + (size_t)(t0 + base + t) * D + c * VEC);
+      if (base + t < len && c < nck) cp_async16(st + q * 16, rows.key(t0 + base + t) + c * VEC);
     }
   }
 
@@ -225,13 +291,13 @@ struct ScoreStream {
 };
 
 // Prologue: put the first NS-1 stages of this warp in flight.
-template <typename T, int D, int LPT, int SB = kWarpStageBytes, int NS = kStages>
-__device__ __forceinline__ void score_prologue(const T *Krow, int t0, int len, int nck, unsigned char *ring) {
+template <typename T, int D, int LPT, int SB = kWarpStageBytes, int NS = kStages, class R>
+__device__ __forceinline__ void score_prologue(const R &rows, int t0, int len, int nck, unsigned char *ring) {
   using SS = ScoreStream<T, D, LPT, SB, NS>;
   unsigned char *wring = ring + (threadIdx.x >> 5) * (SB * NS);
 #pragma unroll
   for (int s = 0; s < NS - 1; ++s) {
-    SS::issue(Krow, t0, len, nck, s, wring);
+    SS::issue(rows, t0, len, nck, s, wring);
     cp_async_commit();
   }
 }
@@ -239,8 +305,8 @@ __device__ __forceinline__ void score_prologue(const T *Krow, int t0, int len, i
 // The key stream: leaves score_key(score) of every token of [t0, t0+len) in
 // keys[] and counts each key's top bits in the skewed histogram hist.  Ends
 // with __syncthreads().
-template <typename T, int D, int LPT, int SB, int NS, int HSHIFT>
-__device__ __forceinline__ void score_keys_loop(const T *Krow, int t0, int len, int nck, unsigned char *ring,
+template <typename T, int D, int LPT, int SB, int NS, int HSHIFT, class R>
+__device__ __forceinline__ void score_keys_loop(const R &rows, int t0, int len, int nck, unsigned char *ring,
                                                 const float *u, uint32_t *keys, uint32_t *hist) {
   using SS = ScoreStream<T, D, LPT, SB, NS>;
   constexpr int VEC = VecN<T>::value;
@@ -253,7 +319,7 @@ __device__ __forceinline__ void score_keys_loop(const T *Krow, int t0, int len, 
   for (int s = 0; s < ns; ++s) {
     cp_async_wait<NS - 2>();
     __syncwarp();
-    SS::issue(Krow, t0, len, nck, s + NS - 1, wring);
+    SS::issue(rows, t0, len, nck, s + NS - 1, wring);
     cp_async_commit();
     SS::template consume_keys<HSHIFT>(len, nck, s, wring, uv, keys, hist);
   }
@@ -345,8 +411,9 @@ struct RowStream {
   static constexpr int CPR = RB / 16;            // chunks per row
   static constexpr int TA = kWarpStageBytes / (2 * RB);
 
-  __device__ __forceinline__ static void issue(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
-                                               int s, unsigned char *wring) {
+  template <class R>
+  __device__ __forceinline__ static void issue(const R &rows, const int32_t *ids, int tok0, int cnt, int s,
+                                               unsigned char *wring) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
     const int base = (s * kWarps + warp) * TA;
@@ -357,7 +424,7 @@ struct RowStream {
       const int i = base + t;
       if (i < cnt) {
         const int tok = GATHER ? ids[i] : tok0 + i;
-        const T *src = (c < CPR ? Kb : Vb) + (size_t)tok * D + (c % CPR) * VEC;
+        const T *src = (c < CPR ? rows.key(tok) : rows.val(tok)) + (c % CPR) * VEC;
         cp_async16(st + q * 16, src);
       }
     }
@@ -370,21 +437,21 @@ struct RowStream {
   }
 };
 
-template <typename T, int D, bool GATHER>
-__device__ __forceinline__ void attend_prologue(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+template <typename T, int D, bool GATHER, class R>
+__device__ __forceinline__ void attend_prologue(const R &rows, const int32_t *ids, int tok0, int cnt,
                                                 unsigned char *ring) {
   unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
-    RowStream<T, D, GATHER>::issue(Kb, Vb, ids, tok0, cnt, s, wring);
+    RowStream<T, D, GATHER>::issue(rows, ids, tok0, cnt, s, wring);
     cp_async_commit();
   }
 }
 
-template <typename T, int D, int G, bool GATHER>
-__device__ __forceinline__ void attend_loop(const T *__restrict__ Kb, const T *__restrict__ Vb,
-                                            const int32_t *ids, int tok0, int cnt, const float *qhat,
-                                            unsigned char *ring, float *pm, float *pl, float *pacc) {
+template <typename T, int D, int G, bool GATHER, class R>
+__device__ __forceinline__ void attend_loop(const R &rows, const int32_t *ids, int tok0, int cnt,
+                                            const float *qhat, unsigned char *ring, float *pm, float *pl,
+                                            float *pacc) {
   using RS = RowStream<T, D, GATHER>;
   constexpr int VEC = RS::VEC;
   constexpr int LPR = D / VEC;
@@ -413,7 +480,7 @@ __device__ __forceinline__ void attend_loop(const T *__restrict__ Kb, const T *_
   for (int s = 0; s < ns; ++s) {
     cp_async_wait<kStages - 2>();
     __syncwarp();
-    RS::issue(Kb, Vb, ids, tok0, cnt, s + kStages - 1, wring);
+    RS::issue(rows, ids, tok0, cnt, s + kStages - 1, wring);
     cp_async_commit();
     const unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
     const int base = (s * kWarps + warp) * RS::TA;
@@ -558,8 +625,8 @@ struct MmaRowStream {
 
   __device__ __forceinline__ static int swz(int c, int r) { return (c & ~7) | ((c ^ r) & 7); }
 
-  __device__ __forceinline__ static void issue(const __nv_bfloat16 *Kb, const __nv_bfloat16 *Vb,
-                                               const int32_t *ids, int tok0, int cnt, int s,
+  template <class R>
+  __device__ __forceinline__ static void issue(const R &rows, const int32_t *ids, int tok0, int cnt, int s,
                                                unsigned char *wring) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char *st = wring + (s % NST) * TB;
@@ -571,7 +638,7 @@ struct MmaRowStream {
       const int i = base + r;
       const bool valid = i < cnt;
       const int tok = valid ? (GATHER ? ids[i] : tok0 + i) : 0;
-      const __nv_bfloat16 *src = (c < CPT / 2 ? Kb : Vb) + (size_t)tok * D + (c % (CPT / 2)) * 8;
+      const __nv_bfloat16 *src = (c < CPT / 2 ? rows.key(tok) : rows.val(tok)) + (c % (CPT / 2)) * 8;
       cp_async16_zfill(st + r * REC + swz(c, r) * 16, src, valid);
     }
   }
@@ -583,14 +650,14 @@ struct MmaRowStream {
   }
 };
 
-template <int D, int G, bool GATHER>
-__device__ __forceinline__ void attend_mma_prologue(const __nv_bfloat16 *Kb, const __nv_bfloat16 *Vb,
-                                                    const int32_t *ids, int tok0, int cnt, unsigned char *ring) {
+template <int D, int G, bool GATHER, class R>
+__device__ __forceinline__ void attend_mma_prologue(const R &rows, const int32_t *ids, int tok0, int cnt,
+                                                    unsigned char *ring) {
   using RS = MmaRowStream<D, G, GATHER>;
   unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
 #pragma unroll
   for (int s = 0; s < RS::NST - 1; ++s) {
-    RS::issue(Kb, Vb, ids, tok0, cnt, s, wring);
+    RS::issue(rows, ids, tok0, cnt, s, wring);
     cp_async_commit();
   }
 }
@@ -618,11 +685,10 @@ __device__ __forceinline__ void build_query_tiles(const float *qhat, unsigned ch
   __syncthreads();
 }
 
-template <int D, int G, bool GATHER>
-__device__ __forceinline__ void attend_mma_loop(const __nv_bfloat16 *__restrict__ Kb,
-                                                const __nv_bfloat16 *__restrict__ Vb, const int32_t *ids,
-                                                int tok0, int cnt, const unsigned char *qt, unsigned char *ring,
-                                                float *pm, float *pl, float *pacc) {
+template <int D, int G, bool GATHER, class R>
+__device__ __forceinline__ void attend_mma_loop(const R &rows, const int32_t *ids, int tok0, int cnt,
+                                                const unsigned char *qt, unsigned char *ring, float *pm, float *pl,
+                                                float *pacc) {
   using RS = MmaRowStream<D, G, GATHER>;
   constexpr int KS = D / 16;  // k-steps of the logit product
   constexpr int MT = D / 16;  // 16-dim tiles of the output product
@@ -640,7 +706,7 @@ __device__ __forceinline__ void attend_mma_loop(const __nv_bfloat16 *__restrict_
   for (int s = 0; s < nt; ++s) {
     cp_async_wait<RS::NST - 2>();
     __syncwarp();
-    RS::issue(Kb, Vb, ids, tok0, cnt, s + RS::NST - 1, wring);
+    RS::issue(rows, ids, tok0, cnt, s + RS::NST - 1, wring);
     cp_async_commit();
     const unsigned char *st = wring + (s % RS::NST) * RS::TB;
     const int base = (s * kWarps + warp) * RS::TILE;
@@ -742,25 +808,25 @@ __device__ __forceinline__ void attend_mma_loop(const __nv_bfloat16 *__restrict_
 // (there the CUDA-core loop, at 2G+1 instructions per cache element, can no
 // longer keep up with HBM); CUDA cores for smaller groups and for fp32 caches
 // (whose 1e-4 tolerance rules out bf16 operands).
-template <typename T, int D, int G, bool GATHER>
-__device__ __forceinline__ void attend_prologue_any(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+template <typename T, int D, int G, bool GATHER, class R>
+__device__ __forceinline__ void attend_prologue_any(const R &rows, const int32_t *ids, int tok0, int cnt,
                                                     unsigned char *ring) {
   if constexpr (std::is_same<T, __nv_bfloat16>::value && G >= 4)
-    attend_mma_prologue<D, G, GATHER>(Kb, Vb, ids, tok0, cnt, ring);
+    attend_mma_prologue<D, G, GATHER>(rows, ids, tok0, cnt, ring);
   else
-    attend_prologue<T, D, GATHER>(Kb, Vb, ids, tok0, cnt, ring);
+    attend_prologue<T, D, GATHER>(rows, ids, tok0, cnt, ring);
 }
 
 // qtiles: 8*D words of shared memory that nothing else uses during the call.
-template <typename T, int D, int G, bool GATHER>
-__device__ __forceinline__ void attend_loop_any(const T *Kb, const T *Vb, const int32_t *ids, int tok0, int cnt,
+template <typename T, int D, int G, bool GATHER, class R>
+__device__ __forceinline__ void attend_loop_any(const R &rows, const int32_t *ids, int tok0, int cnt,
                                                 const float *qhat, unsigned char *qtiles, unsigned char *ring,
                                                 float *pm, float *pl, float *pacc) {
   if constexpr (std::is_same<T, __nv_bfloat16>::value && G >= 4) {
     build_query_tiles<D, G>(qhat, qtiles);
-    attend_mma_loop<D, G, GATHER>(Kb, Vb, ids, tok0, cnt, qtiles, ring, pm, pl, pacc);
+    attend_mma_loop<D, G, GATHER>(rows, ids, tok0, cnt, qtiles, ring, pm, pl, pacc);
   } else {
-    attend_loop<T, D, G, GATHER>(Kb, Vb, ids, tok0, cnt, qhat, ring, pm, pl, pacc);
+    attend_loop<T, D, G, GATHER>(rows, ids, tok0, cnt, qhat, ring, pm, pl, pacc);
   }
 }
 
@@ -801,7 +867,7 @@ __device__ __forceinline__ void cluster_combine(int ncta, int rank, const float 
   }
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -818,14 +884,15 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kerne
   float *scratch = reinterpret_cast<float *>(smem + L.slots);
   unsigned char *ring = reinterpret_cast<unsigned char *>(smem + L.ring);
 
-  const int t0 = min(a.seq_len, rank * a.chunk);
-  const int len = min(a.seq_len, t0 + a.chunk) - t0;
-  const size_t row_off = (size_t)row * a.capacity * D;
+  const int S = row_seq_len(a, b);
+  const int t0 = min(S, rank * a.chunk);
+  const int len = min(S, t0 + a.chunk) - t0;
+  const Rows<T, D, PAGED> rows = make_rows<T, D, PAGED>(a, b, g);
   rotate_queries<T, D, G>(a, b, g, qhat, u, scratch, false, [&] {
-    attend_prologue_any<T, D, G, false>(a.k_hat + row_off, a.v + row_off, nullptr, t0, len, ring);
+    attend_prologue_any<T, D, G, false>(rows, nullptr, t0, len, ring);
   });
-  attend_loop_any<T, D, G, false>(a.k_hat + row_off, a.v + row_off, nullptr, t0, len, qhat,
-                                  reinterpret_cast<unsigned char *>(scratch), ring, pm, pl, pacc);
+  attend_loop_any<T, D, G, false>(rows, nullptr, t0, len, qhat, reinterpret_cast<unsigned char *>(scratch), ring,
+                                  pm, pl, pacc);
   cluster.sync();
   const int Hq = a.n_kv_heads * G;
   cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);

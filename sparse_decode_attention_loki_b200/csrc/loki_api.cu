@@ -277,17 +277,17 @@ loki_status allow_smem(Kern kern, const DevInfo &di, SmemGate &gate, bool cluste
   return LOKI_OK;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 struct DenseGate {
   static SmemGate gate;
 };
-template <typename T, int D, int G>
-SmemGate DenseGate<T, D, G>::gate;
+template <typename T, int D, int G, bool PAGED>
+SmemGate DenseGate<T, D, G, PAGED>::gate;
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a, void *stream, Plan *used) {
-  auto kern = dense_decode_kernel<T, D, G>;
-  loki_status s = allow_smem(kern, di, DenseGate<T, D, G>::gate, true);
+  auto kern = dense_decode_kernel<T, D, G, PAGED>;
+  loki_status s = allow_smem(kern, di, DenseGate<T, D, G, PAGED>::gate, true);
   if (s != LOKI_OK) return s;
   Plan pl;
   s = plan_dense(kern, di, sh, &pl);
@@ -352,18 +352,18 @@ loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepP
   return LOKI_OK;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 struct StepGate {
   static SmemGate gate;
 };
-template <typename T, int D, int G>
-SmemGate StepGate<T, D, G>::gate;
+template <typename T, int D, int G, bool PAGED>
+SmemGate StepGate<T, D, G, PAGED>::gate;
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da, void *ws, void *stream,
                      StepPlan *used) {
-  auto kern = loki_decode_kernel<T, D, G>;
-  loki_status s = allow_smem(kern, di, StepGate<T, D, G>::gate, true);
+  auto kern = loki_decode_kernel<T, D, G, PAGED>;
+  loki_status s = allow_smem(kern, di, StepGate<T, D, G, PAGED>::gate, true);
   if (s != LOKI_OK) return s;
   StepPlan pl;
   s = plan_step(kern, di, sh, &pl);
@@ -387,14 +387,21 @@ loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da,
 }
 
 // ---------------------------------------------------------------------------
+template <typename T, int D, int G, bool PAGED>
+loki_status dispatch_p(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
+                       void *stream, Plan *used) {
+  if (dense) return run_dense<T, D, G, PAGED>(di, sh, a, stream, used);
+  StepPlan sp;
+  loki_status s = run_step<T, D, G, PAGED>(di, sh, a, ws, stream, used ? &sp : nullptr);
+  if (s == LOKI_OK && used) *used = Plan{sp.ncta, sp.chunk, sp.smem};
+  return s;
+}
+
 template <typename T, int D, int G>
 loki_status dispatch(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
                      void *stream, Plan *used) {
-  if (dense) return run_dense<T, D, G>(di, sh, a, stream, used);
-  StepPlan sp;
-  loki_status s = run_step<T, D, G>(di, sh, a, ws, stream, used ? &sp : nullptr);
-  if (s == LOKI_OK && used) *used = Plan{sp.ncta, sp.chunk, sp.smem};
-  return s;
+  if (a.table != nullptr) return dispatch_p<T, D, G, true>(dense, di, sh, a, ws, stream, used);
+  return dispatch_p<T, D, G, false>(dense, di, sh, a, ws, stream, used);
 }
 
 template <typename T, int D>
@@ -409,10 +416,17 @@ loki_status dispatch_g(bool dense, const DevInfo &di, const DecodeShape &sh, con
   return fail(LOKI_ERR_UNSUPPORTED, "group size %d", sh.G);
 }
 
+// Per-sequence lengths and paging of a decode call (all null: a contiguous
+// cache where every row has seq_len tokens and takes k).
+struct VarPage {
+  const int32_t *seq_lens = nullptr, *ks = nullptr, *table = nullptr;
+  int32_t pages_per_seq = 0, page_shift = 0, num_pages = 0;
+};
+
 template <typename T>
 loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense, const void *q, const float *P,
                           int32_t d, int32_t k, float scale, float *out, int32_t *idx, void *ws, void *stream,
-                          Plan *used = nullptr) {
+                          Plan *used = nullptr, const VarPage &vp = VarPage()) {
   DevInfo di;
   loki_status s = device_info(&di);
   if (s != LOKI_OK) return s;
@@ -435,49 +449,46 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   while (lpt < a.nck) lpt *= 2;
   a.lpt = lpt;
   a.scale_log2 = resolve_scale(scale, sh.D);
+  a.seq_lens = vp.seq_lens;
+  a.ks = vp.ks;
+  a.k_stride = k;
+  a.table = vp.table;
+  a.pages_per_seq = vp.pages_per_seq;
+  a.page_shift = vp.page_shift;
+  a.num_pages = vp.num_pages;
   if (sh.D == 64) return dispatch_g<T, 64>(dense, di, sh, a, ws, stream, used);
   return dispatch_g<T, 128>(dense, di, sh, a, ws, stream, used);
 }
 
-template <int D>
+template <int D, bool PAGED>
 struct AppendTcGate {
   static SmemGate gate;
 };
-template <int D>
-SmemGate AppendTcGate<D>::gate;
+template <int D, bool PAGED>
+SmemGate AppendTcGate<D, PAGED>::gate;
 
-template <typename T, int D>
+template <typename T, int D, bool PAGED>
 struct AppendGate {
   static SmemGate gate;
 };
-template <typename T, int D>
-SmemGate AppendGate<T, D>::gate;
+template <typename T, int D, bool PAGED>
+SmemGate AppendGate<T, D, PAGED>::gate;
 
-template <typename T, int D>
-loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const void *k_new, const void *v_new,
-                       const float *P, void *stream) {
+// Launch the append of a.n_vec = B * n_new vectors per KV head (a filled in
+// except per_cta).
+template <typename T, int D, bool PAGED>
+loki_status launch_append(AppendArgs<T> a, void *stream) {
   DevInfo di;
   loki_status s = device_info(&di);
   if (s != LOKI_OK) return s;
-  AppendArgs<T> a;
-  a.k_hat = static_cast<T *>(c->k_hat);
-  a.v = static_cast<T *>(c->v);
-  a.k_new = static_cast<const T *>(k_new);
-  a.v_new = static_cast<const T *>(v_new);
-  a.P = P;
-  a.n_kv_heads = c->n_kv_heads;
-  a.capacity = c->capacity;
-  a.pos = pos;
-  a.n_new = n_new;
-  a.n_vec = c->batch * n_new;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     if (a.n_vec >= kTcMinVectors) {
       // a bulk append: the rotation is a GEMM per head, on the tensor cores
-      auto kern = append_tc_kernel<D>;
-      s = allow_smem(kern, di, AppendTcGate<D>::gate, false);
+      auto kern = append_tc_kernel<D, PAGED>;
+      s = allow_smem(kern, di, AppendTcGate<D, PAGED>::gate, false);
       if (s != LOKI_OK) return s;
       // persistent: one CTA per SM over the (head, tile) units
-      const long long units = (long long)c->n_kv_heads * ((a.n_vec + kTcM - 1) / kTcM);
+      const long long units = (long long)a.n_kv_heads * ((a.n_vec + kTcM - 1) / kTcM);
       if (units > INT32_MAX) return fail(LOKI_ERR_UNSUPPORTED, "bulk append of %d vectors per head is too large", a.n_vec);
       a.per_cta = 0;
       dim3 grid((unsigned)(units < di.sms ? units : di.sms), 1, 1);
@@ -490,23 +501,40 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   // enough CTAs to cover the SMs twice (heads x column blocks x chunks), at
   // least one 8-vector batch each
   const int col_blocks = D / kAppendCols;
-  const long long base = (long long)c->n_kv_heads * col_blocks;
+  const long long base = (long long)a.n_kv_heads * col_blocks;
   const long long want = (2LL * di.sms + base - 1) / base;
   long long per = (a.n_vec + want - 1) / want;
   per = ((per + kAppendBatch - 1) / kAppendBatch) * kAppendBatch;
   if (per < kAppendBatch) per = kAppendBatch;
   a.per_cta = (int)per;
   const long long chunks = (a.n_vec + per - 1) / per;
-  if (chunks > 65535 || c->n_kv_heads > 65535)
+  if (chunks > 65535 || a.n_kv_heads > 65535)
     return fail(LOKI_ERR_UNSUPPORTED, "append of %d vectors per head is too large", a.n_vec);
   const int smem = append_smem_words(D) * 4;
-  s = allow_smem(append_kernel<T, D>, di, AppendGate<T, D>::gate, false);
+  s = allow_smem(append_kernel<T, D, PAGED>, di, AppendGate<T, D, PAGED>::gate, false);
   if (s != LOKI_OK) return s;
-  dim3 grid((unsigned)c->n_kv_heads, (unsigned)col_blocks, (unsigned)chunks);
-  append_kernel<T, D><<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+  dim3 grid((unsigned)a.n_kv_heads, (unsigned)col_blocks, (unsigned)chunks);
+  append_kernel<T, D, PAGED><<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "append_kernel launch");
   return LOKI_OK;
+}
+
+template <typename T, int D>
+loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const void *k_new, const void *v_new,
+                       const float *P, void *stream) {
+  AppendArgs<T> a{};
+  a.k_hat = static_cast<T *>(c->k_hat);
+  a.v = static_cast<T *>(c->v);
+  a.k_new = static_cast<const T *>(k_new);
+  a.v_new = static_cast<const T *>(v_new);
+  a.P = P;
+  a.n_kv_heads = c->n_kv_heads;
+  a.capacity = c->capacity;
+  a.pos = pos;
+  a.n_new = n_new;
+  a.n_vec = c->batch * n_new;
+  return launch_append<T, D, false>(a, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -538,6 +566,53 @@ loki_status noalloc_scratch(void **addr) {
   }
   *addr = g_noalloc_addr[dev];
   return LOKI_OK;
+}
+
+// A paged cache and its sequence table, checked and described as the
+// contiguous cache the decode planner knows: B = batch, capacity =
+// pages_per_seq * page_size (kernels use the pages, not the capacity).
+loki_status check_paged(const loki_paged_cache *c, const loki_seq_table *q, loki_cache *flat, DecodeShape *sh,
+                        int *shift) {
+  if (!c || !q) return fail(LOKI_ERR_INVALID_ARG, "paged cache or sequence table is NULL");
+  if (c->page_size < 1 || c->page_size > 65536 || (c->page_size & (c->page_size - 1)) != 0)
+    return fail(LOKI_ERR_INVALID_ARG, "page_size %d is not a power of two in [1, 65536]", c->page_size);
+  if (c->num_pages < 1) return fail(LOKI_ERR_INVALID_ARG, "num_pages %d must be >= 1", c->num_pages);
+  if (q->batch < 1 || q->pages_per_seq < 1)
+    return fail(LOKI_ERR_INVALID_ARG, "batch %d and pages_per_seq %d must be >= 1", q->batch, q->pages_per_seq);
+  if (!q->block_table || !aligned(q->block_table, 4))
+    return fail(LOKI_ERR_INVALID_ARG, "block_table must be a non-NULL 4-byte aligned device array");
+  if (q->seq_lens && !aligned(q->seq_lens, 4)) return fail(LOKI_ERR_INVALID_ARG, "seq_lens must be 4-byte aligned");
+  const long long cap = (long long)q->pages_per_seq * c->page_size;
+  if (cap > (1LL << 30)) return fail(LOKI_ERR_UNSUPPORTED, "pages_per_seq * page_size = %lld tokens", cap);
+  if (q->max_seq_len < 1 || q->max_seq_len > cap)
+    return fail(LOKI_ERR_INVALID_ARG, "max_seq_len %d outside [1, pages_per_seq * page_size = %lld]", q->max_seq_len,
+                cap);
+  if ((long long)c->num_pages * c->n_kv_heads * c->page_size > (1LL << 40))
+    return fail(LOKI_ERR_UNSUPPORTED, "page pool too large");
+  flat->dtype = c->dtype;
+  flat->batch = q->batch;
+  flat->n_kv_heads = c->n_kv_heads;
+  flat->head_dim = c->head_dim;
+  flat->capacity = (int32_t)cap;
+  flat->k_hat = c->k_hat;
+  flat->v = c->v;
+  loki_status s = check_cache(flat, sh);
+  if (s != LOKI_OK) return s;
+  int sft = 0;
+  while ((1 << sft) < c->page_size) ++sft;
+  *shift = sft;
+  return LOKI_OK;
+}
+
+VarPage paging_of(const loki_paged_cache *c, const loki_seq_table *q, int shift, const int32_t *ks) {
+  VarPage vp;
+  vp.seq_lens = q->seq_lens;
+  vp.ks = ks;
+  vp.table = q->block_table;
+  vp.pages_per_seq = q->pages_per_seq;
+  vp.page_shift = shift;
+  vp.num_pages = c->num_pages;
+  return vp;
 }
 
 // PCA workspace: per-head means [H, D] then covariances [H, D, D], fp64,
@@ -731,6 +806,103 @@ loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, i
   shape[2] = (int32_t)(rows * pl.ncta);
   shape[3] = 0;
   return LOKI_OK;
+}
+
+loki_status loki_paged_append(const loki_paged_cache *cache, const loki_seq_table *seqs, const int32_t *pos,
+                              int32_t n_new, const void *k_new, const void *v_new, const float *P, void *stream) {
+  loki_cache flat;
+  DecodeShape sh;
+  int shift = 0;
+  loki_status s = check_paged(cache, seqs, &flat, &sh, &shift);
+  if (s != LOKI_OK) return s;
+  if (!pos || !aligned(pos, 4)) return fail(LOKI_ERR_INVALID_ARG, "pos must be a non-NULL 4-byte aligned device array");
+  if (n_new < 1) return fail(LOKI_ERR_INVALID_ARG, "n_new %d must be >= 1", n_new);
+  if ((long long)sh.B * n_new > (1LL << 30)) return fail(LOKI_ERR_UNSUPPORTED, "append too large");
+  if (!k_new || !v_new || !P) return fail(LOKI_ERR_INVALID_ARG, "k_new, v_new or P is NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(P, 16))
+    return fail(LOKI_ERR_INVALID_ARG, "k_new, v_new and P must be 16-byte aligned");
+  auto fill = [&](auto *tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    AppendArgs<T> a{};
+    a.k_hat = static_cast<T *>(cache->k_hat);
+    a.v = static_cast<T *>(cache->v);
+    a.k_new = static_cast<const T *>(k_new);
+    a.v_new = static_cast<const T *>(v_new);
+    a.P = P;
+    a.n_kv_heads = sh.Hkv;
+    a.capacity = flat.capacity;
+    a.pos = 0;
+    a.n_new = n_new;
+    a.n_vec = sh.B * n_new;
+    a.pos_arr = pos;
+    a.table = seqs->block_table;
+    a.pages_per_seq = seqs->pages_per_seq;
+    a.page_shift = shift;
+    a.num_pages = cache->num_pages;
+    return a;
+  };
+  if (cache->dtype == LOKI_F32) {
+    const AppendArgs<float> a = fill(static_cast<float *>(nullptr));
+    return sh.D == 64 ? launch_append<float, 64, true>(a, stream) : launch_append<float, 128, true>(a, stream);
+  }
+  const AppendArgs<__nv_bfloat16> a = fill(static_cast<__nv_bfloat16 *>(nullptr));
+  return sh.D == 64 ? launch_append<__nv_bfloat16, 64, true>(a, stream)
+                    : launch_append<__nv_bfloat16, 128, true>(a, stream);
+}
+
+loki_status loki_paged_decode_workspace_size(const loki_paged_cache *cache, const loki_seq_table *seqs,
+                                             int32_t n_q_heads, size_t *bytes) {
+  loki_cache flat;
+  DecodeShape sh;
+  int shift = 0;
+  loki_status s = check_paged(cache, seqs, &flat, &sh, &shift);
+  if (s != LOKI_OK) return s;
+  return loki_decode_workspace_size(&flat, seqs->max_seq_len, n_q_heads, bytes);
+}
+
+loki_status loki_paged_decode_attention(const loki_paged_cache *cache, const loki_seq_table *seqs, int32_t n_q_heads,
+                                        const void *q, const float *P, int32_t d, const int32_t *ks, int32_t k_max,
+                                        float scale, float *out, int32_t *idx, void *workspace,
+                                        size_t workspace_bytes, void *stream) {
+  loki_cache flat;
+  DecodeShape sh;
+  int shift = 0;
+  loki_status s = check_paged(cache, seqs, &flat, &sh, &shift);
+  if (s != LOKI_OK) return s;
+  s = check_decode(&flat, seqs->max_seq_len, n_q_heads, q, P, out, &sh);
+  if (s != LOKI_OK) return s;
+  if (d < 1 || d > sh.D) return fail(LOKI_ERR_INVALID_ARG, "d=%d outside [1, D=%d]", d, sh.D);
+  if (k_max < 1 || k_max > sh.S) return fail(LOKI_ERR_INVALID_ARG, "k_max=%d outside [1, max_seq_len=%d]", k_max, sh.S);
+  if (ks && !aligned(ks, 4)) return fail(LOKI_ERR_INVALID_ARG, "ks must be 4-byte aligned");
+  if (!idx) return fail(LOKI_ERR_INVALID_ARG, "idx is NULL");
+  if (!aligned(idx, 4)) return fail(LOKI_ERR_INVALID_ARG, "idx must be 4-byte aligned");
+  if (!workspace) return fail(LOKI_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(LOKI_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = ws_layout((long long)sh.B * sh.Hkv, sh.G, sh.D).total;
+  if (workspace_bytes < need)
+    return fail(LOKI_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes this call needs",
+                workspace_bytes, need);
+  const VarPage vp = paging_of(cache, seqs, shift, ks);
+  if (cache->dtype == LOKI_F32)
+    return decode_common<float>(&flat, sh, false, q, P, d, k_max, scale, out, idx, workspace, stream, nullptr, vp);
+  return decode_common<__nv_bfloat16>(&flat, sh, false, q, P, d, k_max, scale, out, idx, workspace, stream, nullptr,
+                                      vp);
+}
+
+loki_status dense_paged_decode_attention(const loki_paged_cache *cache, const loki_seq_table *seqs,
+                                         int32_t n_q_heads, const void *q, const float *P, float scale, float *out,
+                                         void *stream) {
+  loki_cache flat;
+  DecodeShape sh;
+  int shift = 0;
+  loki_status s = check_paged(cache, seqs, &flat, &sh, &shift);
+  if (s != LOKI_OK) return s;
+  s = check_decode(&flat, seqs->max_seq_len, n_q_heads, q, P, out, &sh);
+  if (s != LOKI_OK) return s;
+  const VarPage vp = paging_of(cache, seqs, shift, nullptr);
+  if (cache->dtype == LOKI_F32)
+    return decode_common<float>(&flat, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream, nullptr, vp);
+  return decode_common<__nv_bfloat16>(&flat, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream, nullptr, vp);
 }
 
 loki_status loki_pca_workspace_size(int32_t n_heads, int32_t head_dim, size_t *bytes) {

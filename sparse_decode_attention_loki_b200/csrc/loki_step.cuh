@@ -411,7 +411,7 @@ __device__ __forceinline__ void lowrank_query(const DecodeArgs<T> &a, int b, int
 }
 
 // ---------------------------------------------------------------------------
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel(const __grid_constant__ StepArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -432,25 +432,23 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   uint32_t *rw = smem + L.ring;  // the ring as words, for the select buffers
   uint32_t *keys = smem + L.keys;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int S = a.da.seq_len;
-  const uint32_t k = (uint32_t)a.da.k;
+  const int S = row_seq_len(a.da, b);
+  const uint32_t k = (uint32_t)row_k(a.da, b, S);
   const int t0 = min(S, rank * a.da.chunk);
   const int len = min(S, t0 + a.da.chunk) - t0;
-  const size_t row_off = (size_t)row * a.da.capacity * D;
-  const T *Krow = a.da.k_hat + row_off;
-  const T *Vrow = a.da.v + row_off;
+  const Rows<T, D, PAGED> rows = make_rows<T, D, PAGED>(a.da, b, g);
   constexpr int MAXL = D / VecN<T>::value;
 
   // 1. key stream; the low-rank group query is formed while its first stages
   // are in flight (neither depends on the rotate grid)
   lowrank_query<T, D, G>(a.da, b, g, qhat, reinterpret_cast<float *>(hist), u, [&] {
-    LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(Krow, t0, len, a.da.nck, ring)));
+    LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
   });
   for (int e = tid; e < skewed_words(kDig1Bins); e += kThreads) hist[e] = 0u;
   __syncthreads();
   cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
-                    (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(Krow, t0, len, a.da.nck,
+                    (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(rows, t0, len, a.da.nck,
                                                                                        ring, u, keys, hist)));
 
   // 2. cluster radix select; the ring is idle until the gather
@@ -645,8 +643,10 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     }
     take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
   }
-  int32_t *idx_row = a.da.idx + (size_t)row * k;
+  int32_t *idx_row = a.da.idx + (size_t)row * a.da.k_stride;
   write_selection_vec(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
+  // a row shorter than the longest one: the rest of its idx row is -1
+  for (int i = (int)k + rank * kThreads + tid; i < a.da.k_stride; i += ncta * kThreads) idx_row[i] = -1;
   cluster.sync();  // the whole row of idx is written and visible to the cluster
 
   griddep_wait();  // q_hat is written
@@ -659,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   int32_t *ids = reinterpret_cast<int32_t *>(keys);
   for (int i = tid; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), S - 1);
   __syncthreads();
-  attend_prologue_any<T, D, G, true>(Krow, Vrow, ids, 0, s1 - s0, ring);
-  attend_loop_any<T, D, G, true>(Krow, Vrow, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
+  attend_prologue_any<T, D, G, true>(rows, ids, 0, s1 - s0, ring);
+  attend_loop_any<T, D, G, true>(rows, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
                                  pm, pl, pacc);
 
   // 4. log-sum-exp merge of the cluster's states

@@ -29,6 +29,8 @@ def test_header_declares_the_abi():
     assert set(names) == {"loki_append", "loki_decode_workspace_size", "loki_decode_attention",
                           "loki_decode_attention_noalloc", "dense_decode_attention", "loki_decode_launch_shape",
                           "loki_topk_jaccard", "loki_device_error_count", "loki_pca_workspace_size",
+                          "loki_paged_append", "loki_paged_decode_workspace_size", "loki_paged_decode_attention",
+                          "dense_paged_decode_attention",
                           "loki_pca_calibrate", "loki_status_string", "loki_last_error", "loki_version"}
 
 
@@ -50,7 +52,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 7
+    assert lib.loki_version() == 8
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -185,3 +187,72 @@ def test_append_pointer_validation(lib):
     assert lib.loki_append(ctypes.byref(c), 0, 1, FAKE, FAKE + 4, FAKE, None) == 1
     assert lib.loki_append(ctypes.byref(c), 0, 1, FAKE, FAKE, None, None) == 1
     assert lib.loki_append(None, 0, 1, FAKE, FAKE, FAKE, None) == 1
+
+
+def _paged(dtype=1, H=2, D=128, page=16, pages=10, k=4096, v=8192):
+    from sparse_decode_attention_loki_b200 import _lib
+    return _lib.loki_paged_cache(dtype, H, D, page, pages, k, v)
+
+
+def _seqs(B=2, pps=4, max_len=50, table=FAKE, lens=FAKE):
+    from sparse_decode_attention_loki_b200 import _lib
+    return _lib.loki_seq_table(B, pps, max_len, table, lens)
+
+
+def test_paged_workspace_size_and_cache_validation(lib):
+    n = ctypes.c_size_t(0)
+    c, q = _paged(), _seqs()
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 4, ctypes.byref(n)) == 0
+    assert n.value == _ws_bytes(4, 2, 128)
+    bad_caches = [_paged(page=24), _paged(page=0), _paged(page=1 << 17), _paged(pages=0), _paged(dtype=5),
+                  _paged(H=0), _paged(k=0), _paged(v=FAKE + 8)]
+    for bc in bad_caches:
+        assert lib.loki_paged_decode_workspace_size(ctypes.byref(bc), ctypes.byref(q), 4, ctypes.byref(n)) == 1
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(_paged(D=96)), ctypes.byref(q), 4,
+                                                ctypes.byref(n)) == 2
+    bad_seqs = [_seqs(B=0), _seqs(pps=0), _seqs(max_len=0), _seqs(max_len=65), _seqs(table=None),
+                _seqs(table=FAKE + 2), _seqs(lens=FAKE + 2)]
+    for bq in bad_seqs:
+        assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), ctypes.byref(bq), 4, ctypes.byref(n)) == 1
+    assert lib.loki_paged_decode_workspace_size(None, ctypes.byref(q), 4, ctypes.byref(n)) == 1
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), None, 4, ctypes.byref(n)) == 1
+    # NULL seq_lens is allowed (every sequence at max_seq_len)
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), ctypes.byref(_seqs(lens=None)), 4,
+                                                ctypes.byref(n)) == 0
+
+
+def test_paged_decode_validation(lib):
+    c, q = _paged(), _seqs()
+    need = _ws_bytes(4, 2, 128)
+    base = dict(hq=4, qp=FAKE, P=FAKE, d=32, ks=FAKE, kmax=10, out=FAKE, idx=FAKE, ws=WS, wsb=need)
+    def call(**kw):
+        a = dict(base)
+        a.update(kw)
+        return lib.loki_paged_decode_attention(ctypes.byref(c), ctypes.byref(q), a["hq"], a["qp"], a["P"], a["d"],
+                                               a["ks"], a["kmax"], 0.0, a["out"], a["idx"], a["ws"], a["wsb"], None)
+    assert call(d=0) == 1
+    assert call(d=129) == 1
+    assert call(kmax=0) == 1
+    assert call(kmax=51) == 1            # beyond max_seq_len
+    assert call(ks=FAKE + 2) == 1
+    assert call(idx=None) == 1
+    assert call(ws=None) == 1
+    assert call(ws=WS + 16) == 1
+    assert call(wsb=need - 1) == 1
+    assert call(hq=3) == 1
+    assert call(hq=6) == 2               # group of 3
+    assert call(qp=None) == 1
+    assert lib.dense_paged_decode_attention(ctypes.byref(c), ctypes.byref(q), 3, FAKE, FAKE, 0.0, FAKE, None) == 1
+    assert lib.dense_paged_decode_attention(ctypes.byref(c), ctypes.byref(q), 4, None, FAKE, 0.0, FAKE, None) == 1
+
+
+def test_paged_append_validation(lib):
+    c, q = _paged(), _seqs()
+    assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), None, 1, FAKE, FAKE, FAKE, None) == 1
+    assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), FAKE + 2, 1, FAKE, FAKE, FAKE, None) == 1
+    assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), FAKE, 0, FAKE, FAKE, FAKE, None) == 1
+    assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), FAKE, 1, None, FAKE, FAKE, None) == 1
+    assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), FAKE, 1, FAKE, FAKE + 4, FAKE, None) == 1
+    assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), FAKE, 1, FAKE, FAKE, None, None) == 1
+    assert lib.loki_paged_append(ctypes.byref(_paged(page=3)), ctypes.byref(q), FAKE, 1, FAKE, FAKE, FAKE,
+                                 None) == 1

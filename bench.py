@@ -229,6 +229,47 @@ def time_pca(L, calib, dev, stream, reps: int = 3):
             "kernels": "pca_mean_kernel, pca_cov_kernel, pca_jacobi_kernel"}
 
 
+def time_paged(L, w, cache, qs, P, flush, stream, dev, steps: int, warmup: int, page: int = 16):
+    """Device time of loki_paged_decode_attention on a paged copy of the cache
+    (pages of `page` tokens in a shuffled order, every sequence at seq_len),
+    L2 flushed before each call like the main loop."""
+    import torch
+    B, Hkv, S, D = w.batch, w.n_kv_heads, w.seq_len, w.head_dim
+    pps = (S + page - 1) // page
+    gen_t = torch.Generator(device="cpu")
+    gen_t.manual_seed(7)
+    perm = torch.randperm(B * pps, generator=gen_t).to(dev)
+    table = perm.view(B, pps).to(torch.int32).contiguous()
+    pcache = L.PagedLokiCache(B * pps, Hkv, D, page, dtype=cache.dtype, device=dev)
+    pad = pps * page - S
+    for src, dst in ((cache.k_hat, pcache.k_hat), (cache.v, pcache.v)):
+        x = src[:, :, :S]
+        if pad:
+            x = torch.cat([x, torch.zeros((B, Hkv, pad, D), dtype=x.dtype, device=dev)], dim=2)
+        x = x.view(B, Hkv, pps, page, D).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv, page, D)
+        dst[perm.long()] = x
+    seqs = L.SeqTable(table, None, S)
+    out = torch.empty((B, w.n_q_heads, D), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
+    ws = cache.workspace(S, w.n_q_heads)
+    for i in range(max(3, warmup)):
+        L.loki_paged_decode_attention(pcache, seqs, qs[i % len(qs)], P, w.d, w.k, out=out, idx=idx, workspace=ws)
+    torch.cuda.synchronize()
+    tot = 0.0
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i & 7))
+        evs[i][0].record(stream)
+        L.loki_paged_decode_attention(pcache, seqs, qs[i % len(qs)], P, w.d, w.k, out=out, idx=idx, workspace=ws)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    tot = sum(a.elapsed_time(b) for a, b in evs) * 1000.0
+    us = tot / steps
+    del pcache
+    return {"us": us, "page_size": page, "pages": int(B * pps), "steps": steps,
+            "hbm_gbs": w.loki_bytes() / (us * 1e-6) / 1e9, "layout": "shuffled pages, every sequence at seq_len"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -378,6 +419,8 @@ def run_ours(args):
         for i in range(n):
             t_exact += ex_ev[i][0].elapsed_time(ex_ev[i][1])
         done += n
+    # ---------------- the same step on a paged copy of the cache (16-token pages, shuffled)
+    paged = time_paged(L, w, cache, qs, P, flush, stream, dev, steps=min(args.steps, 500), warmup=args.warmup)
     jac = []
     for j in range(NSET):
         L.loki_decode_attention(cache, S, qs[j], P, w.d, w.k, out=out, idx=idx)
@@ -423,6 +466,7 @@ def run_ours(args):
             "append_us": app_us,
             "prefill_append": None if prefill is None else dict(prefill, frac=prefill["hbm_gbs"] / peak),
             "pca_calibrate": pca,
+            "paged": dict(paged, frac=paged["hbm_gbs"] / peak),
             "exact_topk": {"us": t_exact * 1000.0 / ex_steps, "d": D, "k": w.k, "steps": ex_steps,
                            "jaccard_vs_loki": {"mean": float(jaccard.mean()), "min": float(jaccard.min()),
                                                "rows": int(jaccard.numel())}},

@@ -6,11 +6,12 @@
 // compute exact softmax attention over them.  The dense kernel is the "Full
 // Attention" baseline (same page, "Experimental setup").
 //
-// This file holds the pieces: the query rotation, the low-rank score stream,
-// the ordered write of a selection, the gather/stream attention loops (CUDA
-// cores, or warp-level tensor cores for query groups of 4+), the cluster
-// log-sum-exp combine and the dense decode kernel.  loki_step.cuh chains them
-// into the four kernels of one Loki step.
+// This file holds the pieces: token addressing (contiguous or paged caches),
+// the query rotation, the low-rank score stream, the gather/stream attention
+// loops (CUDA cores, or warp-level tensor cores for query groups of 4+), the
+// cluster log-sum-exp combine and the dense decode kernel.  loki_step.cuh
+// chains them, with the cluster top-k select, into the two kernels of one
+// Loki step.
 //
 // Dense decode: one thread-block cluster of `ncta` CTAs owns one (batch, KV
 // head) row; CTA r streams the contiguous token range [r*chunk, (r+1)*chunk)
@@ -350,54 +351,7 @@ struct SelectState {
 };
 
 // ---------------------------------------------------------------------------
-// 4. write this CTA's selected indices, ascending, from position st.offset of
-//    the row of idx.  Each warp owns a contiguous segment of the CTA's tokens.
-__device__ __forceinline__ void write_selection(const uint32_t *keys, int len, int t0, const SelectState &st,
-                                                uint32_t k, uint32_t *ctl, int32_t *idx_row) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int seg = (((len + kWarps - 1) / kWarps) + 31) & ~31;
-  const int sbeg = min(len, warp * seg), send = min(len, sbeg + seg);
-  uint32_t wg = 0u, we = 0u;
-  for (int j0 = sbeg; j0 < send; j0 += 32) {
-    const int j = j0 + lane;
-    const bool in = j < send;
-    const uint32_t km = in ? (keys[j] & st.mask) : 0u;
-    wg += __popc(__ballot_sync(kFull, in && km > st.prefix));
-    we += __popc(__ballot_sync(kFull, in && km == st.prefix));
-  }
-  if (lane == 0) {
-    ctl[kCtlWarpGt + warp] = wg;
-    ctl[kCtlWarpEq + warp] = we;
-  }
-  __syncthreads();
-  uint32_t eq_base = 0u, sel_base = 0u;
-  for (int w = 0; w < warp; ++w) {
-    const uint32_t want = st.take > eq_base ? st.take - eq_base : 0u;
-    sel_base += ctl[kCtlWarpGt + w] + min(ctl[kCtlWarpEq + w], want);
-    eq_base += ctl[kCtlWarpEq + w];
-  }
-  int32_t *dst = idx_row + st.offset;
-  uint32_t run_eq = eq_base, run_sel = sel_base;
-  const uint32_t lt = lanemask_lt();
-  for (int j0 = sbeg; j0 < send; j0 += 32) {
-    const int j = j0 + lane;
-    const bool in = j < send;
-    const uint32_t km = in ? (keys[j] & st.mask) : 0u;
-    const bool gt = in && km > st.prefix;
-    const bool eq = in && km == st.prefix;
-    const uint32_t eb = __ballot_sync(kFull, eq);
-    const uint32_t eq_rank = run_eq + __popc(eb & lt);
-    const bool sel = gt || (eq && eq_rank < st.take);
-    const uint32_t sb = __ballot_sync(kFull, sel);
-    const uint32_t p = run_sel + __popc(sb & lt);
-    if (sel && st.offset + p < k) dst[p] = t0 + j;  // bound: the row holds k entries
-    run_eq += __popc(eb);
-    run_sel += __popc(sb);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// 5. exact attention over `cnt` rows -- gathered through ids[] (shared memory,
+// 4. exact attention over `cnt` rows -- gathered through ids[] (shared memory,
 //    already clamped into the row) or the contiguous rows tok0 .. tok0+cnt-1.
 //    Rows are cut into blocks of TA = kWarpStageBytes/(2*row bytes); warp w
 //    streams blocks w, w+8, ... through its ring slice, each row as its K row
@@ -424,7 +378,7 @@ struct RowStream {
       const int i = base + t;
       if (i < cnt) {
         const int tok = GATHER ? ids[i] : tok0 + i;
-        const T *src = (c < CPR ? rows.key(tok) : rows.val(tok)) + (c % CPR) * VEC;
+        const T *src = (c < CPR ? rows.k : rows.v) + rows.off(tok) + (c % CPR) * VEC;
         cp_async16(st + q * 16, src);
       }
     }
@@ -638,7 +592,7 @@ struct MmaRowStream {
       const int i = base + r;
       const bool valid = i < cnt;
       const int tok = valid ? (GATHER ? ids[i] : tok0 + i) : 0;
-      const __nv_bfloat16 *src = (c < CPT / 2 ? rows.key(tok) : rows.val(tok)) + (c % (CPT / 2)) * 8;
+      const __nv_bfloat16 *src = (c < CPT / 2 ? rows.k : rows.v) + rows.off(tok) + (c % (CPT / 2)) * 8;
       cp_async16_zfill(st + r * REC + swz(c, r) * 16, src, valid);
     }
   }
@@ -831,7 +785,7 @@ __device__ __forceinline__ void attend_loop_any(const R &rows, const int32_t *id
 }
 
 // ---------------------------------------------------------------------------
-// 6. log-sum-exp combine of the cluster's partial states: CTA r writes the
+// 5. log-sum-exp combine of the cluster's partial states: CTA r writes the
 //    output elements r*256 + t (stride ncta*256); each reads the (max, sum,
 //    acc) of its head from every CTA through distributed shared memory, all
 //    loads issued before the first use.  Must follow a cluster barrier that

@@ -9,10 +9,10 @@
 //   decode  one thread-block cluster of ncta CTAs per row, about one wave of
 //           CTAs in all; CTA r owns tokens [r*chunk, (r+1)*chunk):
 //     1. the first stages of its low-rank key stream go in flight (cp.async
-//        ring) while it forms u from q and P_g[:, :d] itself, then it
-//        streams K_hat[i, :d], keeps one order-preserving uint32 key per
-//        token in shared memory and histograms the keys' top 11 bits on the
-//        way;
+//        ring) before it waits for the rotate grid (a programmatic
+//        dependency) and reads u; then it streams K_hat[i, :d], keeps one
+//        order-preserving uint32 key per token in shared memory and
+//        histograms the keys' top 11 bits on the way;
 //     2. cluster radix select over 11/11/10-bit digits: every CTA adds the
 //        non-zero bins of its histogram into the leader CTA's (distributed
 //        shared memory reductions), the leader finds the bucket of the k-th
@@ -24,8 +24,7 @@
 //        CTA writes its indices in ascending order (should a CTA's candidates
 //        overflow its slot at the leader, the cluster refines with distributed
 //        histogram passes instead);
-//     3. (only now waiting for the rotate grid, a programmatic dependency)
-//        the k selected rows are split evenly over the cluster: gather K_hat
+//     3. the k selected rows are split evenly over the cluster: gather K_hat
 //        and V rows through the ring, online softmax per query head;
 //     4. the CTAs' (max, sum, acc) states are merged through distributed
 //        shared memory with the log-sum-exp rule into out.
@@ -175,7 +174,7 @@ constexpr int kHloc = kRecv3 + skewed_words(1 << kDig3Bits);
 static_assert(kHloc + (1 << kDig2Bits) <= kRingWords, "select buffers must fit in the ring");
 static_assert(kSlots + kMaxCluster * 256 <= kRingWords, "candidate slots must fit in the ring");
 
-// ctl words (write_selection uses 48..63)
+// ctl words (write_selection_bal uses 48..63)
 constexpr int kSelWtot = 0;     // [0..7] block-scan scratch
 constexpr int kSelBucket = 8;   // [8..10] bucket, count above it, count in it (this CTA's search)
 constexpr int kSelFirst = 16;   // [16..18] the leader's first-digit result
@@ -263,10 +262,12 @@ __device__ __forceinline__ void refine_pass(cg::cluster_group &cluster, int ncta
 // Write the CTA's selection, ascending: keys whose masked value is above
 // `prefix`, and the first `take` keys (in token order) whose masked value
 // equals it, from position `offset` of the row.  Warp w owns a contiguous
-// segment of the CTA's tokens (a multiple of 128); a counting sweep gives
-// each warp its offset, a second sweep compacts with warp scans, four keys
-// per lane and step.
-__device__ __forceinline__ void write_selection_vec(const uint32_t *keys, int len, int t0, const SelectState &st,
+// segment of the CTA's tokens (a multiple of 128).  A counting sweep (four
+// keys per lane and load) gives each warp its offset; the writing sweep takes
+// 32 tokens per ballot, four ballots in flight: lane l's position is the
+// selected count before it, popc of the above-mask below l plus the ties
+// below l that are still taken, min(popc(tie-mask below l), ties left).
+__device__ __forceinline__ void write_selection_bal(const uint32_t *keys, int len, int t0, const SelectState &st,
                                                     uint32_t k, uint32_t *ctl, int32_t *idx_row) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = (((len + kWarps - 1) / kWarps) + 127) & ~127;
@@ -305,109 +306,29 @@ __device__ __forceinline__ void write_selection_vec(const uint32_t *keys, int le
     run_eq += ctl[kCtlWarpEq + w];
   }
   int32_t *dst = idx_row + st.offset;
+  const uint32_t lt = lanemask_lt();
   for (int j0 = sbeg; j0 < send; j0 += 128) {
-    const int j = j0 + 4 * lane;
-    uint32_t kk[4] = {0u, 0u, 0u, 0u};
-    if (j < send) {
-      const uint4 v = *reinterpret_cast<const uint4 *>(keys + j);
-      kk[0] = v.x; kk[1] = v.y; kk[2] = v.z; kk[3] = v.w;
+    uint32_t gb[4], eb[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int j = j0 + 32 * x + lane;
+      const bool in = j < send;
+      const uint32_t km = in ? (keys[j] & st.mask) : 0u;
+      gb[x] = __ballot_sync(kFull, in && km > st.prefix);
+      eb[x] = __ballot_sync(kFull, in && km == st.prefix);
     }
-    uint32_t ng = 0u, ne = 0u;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (j + e < send) {
-        const uint32_t km = kk[e] & st.mask;
-        ng += km > st.prefix;
-        ne += km == st.prefix;
-      }
-    }
-    // warp scan of (ties << 16 | above): at most 128 of each per step
-    const uint32_t packed = (ne << 16) | ng;
-    const uint32_t incl = warp_incl_scan(packed);
-    const uint32_t excl = incl - packed;
-    const uint32_t tot = __shfl_sync(kFull, incl, 31);
-    uint32_t eq_rank = run_eq + (excl >> 16);  // tie rank of this lane's first tie in the CTA
-    uint32_t pos = run_sel + (excl & 0xffffu) + (min(take, eq_rank) - min(take, run_eq));
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (j + e < send) {
-        const uint32_t km = kk[e] & st.mask;
-        bool sel = km > st.prefix;
-        if (km == st.prefix) {
-          sel = eq_rank < take;
-          ++eq_rank;
-        }
-        if (sel) {
-          if (st.offset + pos < k) dst[pos] = t0 + j + e;  // bound: the row holds k entries
-          ++pos;
-        }
-      }
-    }
-    const uint32_t new_eq = run_eq + (tot >> 16);
-    run_sel += (tot & 0xffffu) + (min(take, new_eq) - min(take, run_eq));
-    run_eq = new_eq;
-  }
-}
-
-// u[j] = sum_i qs[i] * P_g[i][j] for j < d (zero beyond), qs = the sum of the
-// G queries of the row (fp32): by linearity equal to sum_h q_hat_h[:d].
-// Its loads of P and q are issued first; `after_loads()` runs while they are
-// in flight.  Thread (c4 = tid % C4P, part = tid / C4P) holds the float4 of columns
-// [4c4, 4c4+4) of the rows of its part (C4P = ceil(d/4) rounded up to a
-// power of two); all its loads of P are issued before the first use, then the
-// parts are added in a fixed order in shared memory.  qs: D floats, red:
-// 4*kThreads floats of scratch.  Ends with __syncthreads().
-template <typename T, int D, int G, typename F>
-__device__ __forceinline__ void lowrank_query(const DecodeArgs<T> &a, int b, int g, float *qs, float *red, float *u,
-                                              F &&after_loads) {
-  constexpr int RMAX = D / 8;  // rows per part when C4P = 32 (the most)
-  const int tid = threadIdx.x;
-  const int c4n = (a.d + 3) >> 2;
-  int C4P = 1;
-  while (C4P < c4n) C4P <<= 1;
-  const int parts = kThreads / C4P;                 // >= 8
-  const int rpp = parts >= D ? 1 : D / parts;       // rows per part, <= RMAX
-  const int c4 = tid % C4P, part = tid / C4P;
-  const bool active = c4 < c4n && part * rpp < D;  // parts beyond D rows stay idle
-  const float *Pg = a.P + (size_t)g * D * D + 4 * c4;
-  float4 pv[RMAX];
-#pragma unroll
-  for (int x = 0; x < RMAX; ++x)
-    pv[x] = (active && x < rpp) ? __ldg(reinterpret_cast<const float4 *>(Pg + (size_t)(part * rpp + x) * D))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-  const T *qg = a.q + ((size_t)b * a.n_kv_heads * G + (size_t)g * G) * D;
-  float qv[G];
-  const int iq = tid < D ? tid : 0;
-#pragma unroll
-  for (int h = 0; h < G; ++h) qv[h] = to_f32(qg[(size_t)h * D + iq]);
-  after_loads();  // the caller's own loads go in flight behind these
-  if (tid < D) {
-    float s = 0.f;
-#pragma unroll
-    for (int h = 0; h < G; ++h) s += qv[h];
-    qs[tid] = s;
-  }
-  __syncthreads();
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int x = 0; x < RMAX; ++x) {
-    if (active && x < rpp) {
-      const float qv = qs[part * rpp + x];
-      acc.x = fmaf(qv, pv[x].x, acc.x);
-      acc.y = fmaf(qv, pv[x].y, acc.y);
-      acc.z = fmaf(qv, pv[x].z, acc.z);
-      acc.w = fmaf(qv, pv[x].w, acc.w);
+    for (int x = 0; x < 4; ++x) {
+      const uint32_t left = take > run_eq ? take - run_eq : 0u;  // ties still taken
+      const uint32_t me = 1u << lane;
+      const uint32_t ties_below = __popc(eb[x] & lt);
+      const bool sel = (gb[x] & me) != 0u || ((eb[x] & me) != 0u && ties_below < left);
+      const uint32_t p = run_sel + __popc(gb[x] & lt) + min(ties_below, left);
+      if (sel && st.offset + p < k) dst[p] = t0 + j0 + 32 * x + lane;  // bound: the row holds k entries
+      run_sel += __popc(gb[x]) + min((uint32_t)__popc(eb[x]), left);
+      run_eq += __popc(eb[x]);
     }
   }
-  reinterpret_cast<float4 *>(red)[tid] = acc;  // red[(part * C4P + c4) * 4 + y]
-  __syncthreads();
-  for (int jj = tid; jj < D; jj += kThreads) {
-    float s = 0.f;
-    if (jj < a.d)
-      for (int p = 0; p < parts && p * rpp < D; ++p) s += red[(p * C4P + (jj >> 2)) * 4 + (jj & 3)];
-    u[jj] = s;
-  }
-  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -439,12 +360,12 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   const Rows<T, D, PAGED> rows = make_rows<T, D, PAGED>(a.da, b, g);
   constexpr int MAXL = D / VecN<T>::value;
 
-  // 1. key stream; the low-rank group query is formed while its first stages
-  // are in flight (neither depends on the rotate grid)
-  lowrank_query<T, D, G>(a.da, b, g, qhat, reinterpret_cast<float *>(hist), u, [&] {
-    LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
-  });
+  // 1. key stream: its first stages go in flight before the wait for the
+  // rotate grid, whose low-rank group query u the stream needs
+  LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
   for (int e = tid; e < skewed_words(kDig1Bins); e += kThreads) hist[e] = 0u;
+  griddep_wait();  // u and q_hat are written
+  if (tid < D) u[tid] = __ldcg(a.u + (size_t)row * D + tid);
   __syncthreads();
   cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
@@ -644,12 +565,11 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
   }
   int32_t *idx_row = a.da.idx + (size_t)row * a.da.k_stride;
-  write_selection_vec(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
+  write_selection_bal(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
   // a row shorter than the longest one: the rest of its idx row is -1
   for (int i = (int)k + rank * kThreads + tid; i < a.da.k_stride; i += ncta * kThreads) idx_row[i] = -1;
   cluster.sync();  // the whole row of idx is written and visible to the cluster
 
-  griddep_wait();  // q_hat is written
   for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
   // 3. attention over this CTA's even share of the k selected rows; the
   // indices are staged where the keys were (the share is at most chunk), and

@@ -173,6 +173,12 @@ constexpr int kRecv3 = kRecv2 + skewed_words(1 << kDig2Bits);
 constexpr int kHloc = kRecv3 + skewed_words(1 << kDig3Bits);
 static_assert(kHloc + (1 << kDig2Bits) <= kRingWords, "select buffers must fit in the ring");
 static_assert(kSlots + kMaxCluster * 256 <= kRingWords, "candidate slots must fit in the ring");
+// Rows with S + k <= kGatherWords take the gather path: the leader reads
+// every CTA's keys into its ring at kAllKeys, selects alone and writes the k
+// indices after them (kAllKeys + round4(S) + 4).
+constexpr int kAllKeys = skewed_words(1 << kDig2Bits);
+constexpr int kGatherWords = kRingWords - kAllKeys - 8;
+static_assert(kAllKeys % 4 == 0, "the gathered keys are stored 16 bytes at a time");
 
 // ctl words (write_selection_bal uses 48..63)
 constexpr int kSelWtot = 0;     // [0..7] block-scan scratch
@@ -374,7 +380,76 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
 
   // 2. cluster radix select; the ring is idle until the gather
   const bool leader = rank == 0;
+  int32_t *idx_row = a.da.idx + (size_t)row * a.da.k_stride;
+  const int s0 = (int)(((long long)rank * k) / ncta);  // this CTA's even share of the selection
+  const int s1 = (int)(((long long)(rank + 1) * k) / ncta);
+  int32_t *ids = reinterpret_cast<int32_t *>(keys);  // the share's indices, where the keys were
+  const bool gather = S + (int)k <= kGatherWords;    // uniform over the cluster
   cluster_wait();  // every CTA, the leader in particular, zeroed its histogram before its stream
+  if (gather) {
+    // a short row: the leader collects the histogram, then reads every CTA's
+    // keys (distributed shared memory; CTA r holds tokens [r*chunk, ..),
+    // chunk a multiple of 4) into its ring and selects alone
+    if (!leader) push_skewed(hist, kDig1Bins, dsmem_addr(hist, 0u));
+    cluster.sync();  // every stream is done; the leader's histogram holds the row's
+    uint32_t *all = rw + kAllKeys;
+    if (leader) {
+      const int n4 = (S + 3) >> 2;
+      for (int j0 = tid; j0 < n4; j0 += 4 * kThreads) {
+        uint4 v[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int j4 = j0 + x * kThreads;
+          if (j4 < n4) {
+            const int r = (4 * j4) / a.da.chunk;
+            v[x] = dsmem_ld_v4(dsmem_addr(keys + (4 * j4 - r * a.da.chunk), (uint32_t)r));
+          }
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+          if (j0 + x * kThreads < n4) reinterpret_cast<uint4 *>(all)[j0 + x * kThreads] = v[x];
+      }
+      __syncthreads();
+    }
+    int32_t *list = reinterpret_cast<int32_t *>(all + round4(S) + 4);
+    if (leader) {
+      constexpr int SH2 = 32 - kDig1Bits - kDig2Bits;
+      uint32_t *href = rw + kHref;
+      find_bucket(hist, kDig1Bins, k, ctl);
+      uint32_t rem = k - ctl[kSelBucket + 1], inb = ctl[kSelBucket + 2];
+      uint32_t pre = ctl[kSelBucket + 0] << (32 - kDig1Bits), msk = ~0u << (32 - kDig1Bits);
+      __syncthreads();  // ctl read before it is reused
+      for (int pass = 0; pass < 2 && inb != rem; ++pass) {
+        const int shift = pass == 0 ? SH2 : 0;
+        const int nb = pass == 0 ? (1 << kDig2Bits) : (1 << kDig3Bits);
+        for (int e = tid; e < skewed_words(1 << kDig2Bits); e += kThreads) href[e] = 0u;
+        __syncthreads();
+        for (int i = tid; i < S; i += kThreads) {
+          const uint32_t key = all[i];
+          if ((key & msk) == pre) atomicAdd(&href[hskew((int)((key >> shift) & (uint32_t)(nb - 1)))], 1u);
+        }
+        __syncthreads();
+        find_bucket(href, nb, rem, ctl);
+        rem -= ctl[kSelBucket + 1];
+        inb = ctl[kSelBucket + 2];
+        pre |= ctl[kSelBucket + 0] << shift;
+        msk |= (uint32_t)(nb - 1) << shift;
+        __syncthreads();  // ctl read before it is reused
+      }
+      write_selection_bal(all, S, 0, SelectState{pre, msk, rem, 0u}, k, ctl, list);
+    }
+    cluster.sync();  // the leader's list of the k indices is complete (and it read every CTA's keys)
+    const uint32_t src = dsmem_addr(list + s0, 0u);
+    for (int i = tid; i < s1 - s0; i += kThreads) {
+      const int v = (int)dsmem_ld_u32(src + 4u * (uint32_t)i);
+      idx_row[s0 + i] = v;
+      ids[i] = min(max(v, 0), S - 1);
+    }
+    // a row shorter than the longest one: the rest of its idx row is -1
+    for (int i = (int)k + rank * kThreads + tid; i < a.da.k_stride; i += ncta * kThreads) idx_row[i] = -1;
+    cluster_arrive();  // done reading the leader's ring
+    if (leader) cluster_wait();  // its ring is about to carry the gather
+  } else {
   if (!leader) push_skewed(hist, kDig1Bins, dsmem_addr(hist, 0u));
   cluster.sync();  // the leader's histogram holds the cluster's sum
   if (leader) {
@@ -564,26 +639,25 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     }
     take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
   }
-  int32_t *idx_row = a.da.idx + (size_t)row * a.da.k_stride;
   write_selection_bal(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
   // a row shorter than the longest one: the rest of its idx row is -1
   for (int i = (int)k + rank * kThreads + tid; i < a.da.k_stride; i += ncta * kThreads) idx_row[i] = -1;
   cluster.sync();  // the whole row of idx is written and visible to the cluster
+  // the share's indices, clamped into the row so that no load can leave the
+  // cache even if wrong
+  for (int i = tid; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), S - 1);
+  }  // gather / candidate paths
 
   for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
-  // 3. attention over this CTA's even share of the k selected rows; the
-  // indices are staged where the keys were (the share is at most chunk), and
-  // clamped into the row so that no load can leave the cache even if wrong
-  const int s0 = (int)(((long long)rank * k) / ncta);
-  const int s1 = (int)(((long long)(rank + 1) * k) / ncta);
-  int32_t *ids = reinterpret_cast<int32_t *>(keys);
-  for (int i = tid; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), S - 1);
+  // 3. attention over this CTA's even share of the k selected rows (the
+  // share is at most chunk)
   __syncthreads();
   attend_prologue_any<T, D, G, true>(rows, ids, 0, s1 - s0, ring);
   attend_loop_any<T, D, G, true>(rows, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
                                  pm, pl, pacc);
 
   // 4. log-sum-exp merge of the cluster's states
+  if (gather && !leader) cluster_wait();
   cluster.sync();
   const int Hq = a.da.n_kv_heads * G;
   cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);

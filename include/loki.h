@@ -98,9 +98,11 @@ LOKI_API loki_status loki_append(const loki_cache *cache, int32_t pos, int32_t n
 
 /* loki_decode_workspace_size -- bytes of device workspace that
  * loki_decode_attention needs for a cache of this shape with n_q_heads query
- * heads: the rotated queries and the low-rank group queries of every (batch,
- * KV head) row, B * Hkv * (G + 1) * D * 4 bytes plus alignment.  *bytes is a
- * host pointer. */
+ * heads: room for the rotated queries and the low-rank group queries of every
+ * (batch, KV head) row, B * Hkv * (G + 1) * D * 4 bytes plus alignment (the
+ * call writes them there when its query groups have 8 heads; smaller groups
+ * rotate their queries on chip and leave it untouched).  *bytes is a host
+ * pointer. */
 LOKI_API loki_status loki_decode_workspace_size(const loki_cache *cache, int32_t seq_len,
                                        int32_t n_q_heads, size_t *bytes);
 
@@ -126,9 +128,10 @@ LOKI_API loki_status loki_decode_workspace_size(const loki_cache *cache, int32_t
  * index; out_h = softmax(scale * q_hat_h . k_hat_i over the selected i, full D)
  * weighted sum of v_i.  Requires seq_len <= S_cap and G in {1, 2, 4, 8};
  * otherwise LOKI_ERR_INVALID_ARG or LOKI_ERR_UNSUPPORTED (also for seq_len
- * above 393216 tokens, whose scores would not fit on chip).  Enqueues two
- * kernels on the stream: the query rotation, then the decode kernel (scores,
- * selection, attention) as its programmatic dependent. */
+ * above 393216 tokens, whose scores would not fit on chip).  Enqueues one
+ * kernel on the stream (query rotation, scores, selection, attention); for
+ * query groups of 8 heads, two: the query rotation, then the decode kernel as
+ * its programmatic dependent. */
 LOKI_API loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len,
                                   int32_t n_q_heads, const void *q, const float *P,
                                   int32_t d, int32_t k, float scale, float *out,
@@ -305,9 +308,11 @@ LOKI_API loki_status loki_pca_calibrate(const void *keys, int32_t dtype, int32_t
 
 /* Launch shape a decode call with these sizes would use, for logging and
  * tests.  shape: host array of 4 int32.
- *   dense == 0 (loki_decode_attention): shape[0] CTAs of the query-rotation
- *     kernel, shape[1] CTAs per (batch, KV head) row in one cluster of the
- *     decode kernel, shape[2] CTAs of the decode kernel, shape[3] = 0.
+ *   dense == 0 (loki_decode_attention): shape[0] CTAs of the separate
+ *     query-rotation kernel (0 when the decode kernel rotates its own
+ *     queries, query groups of up to 4 heads), shape[1] CTAs per (batch, KV
+ *     head) row in one cluster of the decode kernel, shape[2] CTAs of the
+ *     decode kernel, shape[3] = 0.
  *   dense != 0 (dense_decode_attention): shape[1] CTAs per row in one
  *     cluster, shape[2] CTAs in all, shape[0] = shape[3] = 0.
  * k is checked (1 <= k <= seq_len) for dense == 0 but does not change the

@@ -380,10 +380,13 @@ loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da,
   a.da = da;
   a.qhat = reinterpret_cast<float *>(w + W.qhat);
   a.u = reinterpret_cast<float *>(w + W.u);
-  s = launch_ex(loki_rotate_kernel<T, D, G>, rows * (D / kRotCols), 0, 0, false, a, stream,
-                "loki_rotate_kernel launch");
-  if (s != LOKI_OK) return s;
-  return launch_ex(kern, rows * pl.ncta, pl.smem, pl.ncta, true, a, stream, "loki_decode_kernel launch");
+  if (!kRotateInKernel<G>) {
+    s = launch_ex(loki_rotate_kernel<T, D, G>, rows * (D / kRotCols), 0, 0, false, a, stream,
+                  "loki_rotate_kernel launch");
+    if (s != LOKI_OK) return s;
+  }
+  return launch_ex(kern, rows * pl.ncta, pl.smem, pl.ncta, !kRotateInKernel<G>, a, stream,
+                   "loki_decode_kernel launch");
 }
 
 // ---------------------------------------------------------------------------
@@ -801,7 +804,8 @@ loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, i
     s = decode_common<__nv_bfloat16>(cache, sh, dense != 0, nullptr, nullptr, 1, 1, 0.f, nullptr, nullptr, nullptr,
                                      nullptr, &pl);
   if (s != LOKI_OK) return s;
-  shape[0] = dense ? 0 : (int32_t)(rows * (sh.D / kRotCols));
+  const bool rot = !dense && sh.G > 4;  // kRotateInKernel<G> is G <= 4
+  shape[0] = rot ? (int32_t)(rows * (sh.D / kRotCols)) : 0;
   shape[1] = pl.ncta;
   shape[2] = (int32_t)(rows * pl.ncta);
   shape[3] = 0;

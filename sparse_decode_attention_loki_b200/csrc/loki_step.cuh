@@ -1,34 +1,40 @@
-// One Loki decode step in two kernels ("Loki: Low-rank Keys for Efficient
-// Sparse Attention", atlas.scime.ai summary, section "Approach": PCA-project
+// One Loki decode step ("Loki: Low-rank Keys for Efficient Sparse
+// Attention", atlas.scime.ai summary, section "Approach": PCA-project
 // queries and keys, rank tokens on the top-d principal dimensions, exact
-// attention over the top-k tokens).
+// attention over the top-k tokens), one kernel for query groups of up to 4
+// heads, two for 8:
 //
-//   rotate  D/32 CTAs per (batch, KV head) row: q_hat_h = q_h . P_g for the G
-//           query heads of the row (fp32, pre-scaled for the softmax) and the
-//           group's low-rank query u = sum_h q_hat_h[:d], into the workspace.
+//   rotate  (groups of 8 only) D/32 CTAs per (batch, KV head) row: q_hat_h =
+//           q_h . P_g for the G query heads of the row (fp32, pre-scaled for
+//           the softmax) and the group's low-rank query u = sum_h
+//           q_hat_h[:d], into the workspace.
 //   decode  one thread-block cluster of ncta CTAs per row, about one wave of
 //           CTAs in all; CTA r owns tokens [r*chunk, (r+1)*chunk):
 //     1. the first stages of its low-rank key stream go in flight (cp.async
-//        ring) before it waits for the rotate grid (a programmatic
-//        dependency) and reads u; then it streams K_hat[i, :d], keeps one
-//        order-preserving uint32 key per token in shared memory and
-//        histograms the keys' top 11 bits on the way;
+//        ring) while it forms q_hat and u from q and P_g (or, for groups of
+//        8, waits for the rotate grid and reads them); then it streams
+//        K_hat[i, :d], keeps one order-preserving uint32 key per token in
+//        shared memory and histograms the keys' top 11 bits on the way;
 //     2. cluster radix select over 11/11/10-bit digits: every CTA adds the
 //        non-zero bins of its histogram into the leader CTA's (distributed
-//        shared memory reductions), the leader finds the bucket of the k-th
-//        largest key and tells every CTA; each CTA sends the leader its keys in
-//        that bucket (the candidates, a few percent) and its count above it;
-//        the leader finishes the threshold on the candidates, derives every
-//        CTA's share of the selection (ties at the threshold go to the lower
-//        index) and hands each CTA its (threshold, ties to take, offset); each
-//        CTA writes its indices in ascending order (should a CTA's candidates
-//        overflow its slot at the leader, the cluster refines with distributed
-//        histogram passes instead);
+//        shared memory reductions).  A short row (S + k within the leader's
+//        ring) is then selected by the leader alone on all its keys, read
+//        from the cluster's shared memory, into an ascending list of k
+//        indices.  On a longer row the leader finds the bucket of the k-th
+//        largest key and tells every CTA; each CTA sends the leader its keys
+//        in that bucket (the candidates, a few percent) and its count above
+//        it; the leader finishes the threshold on the candidates, derives
+//        every CTA's share of the selection (ties at the threshold go to the
+//        lower index) and hands each CTA its (threshold, ties to take,
+//        offset); each CTA writes its indices in ascending order (should a
+//        CTA's candidates overflow its slot at the leader, the cluster
+//        refines with distributed histogram passes instead);
 //     3. the k selected rows are split evenly over the cluster: gather K_hat
 //        and V rows through the ring, online softmax per query head;
 //     4. the CTAs' (max, sum, acc) states are merged through distributed
 //        shared memory with the log-sum-exp rule into out.
-// Scores never leave the chip; the workspace holds only q_hat and u.
+// Scores never leave the chip; the workspace holds only q_hat and u (groups
+// of 8).
 #pragma once
 
 #include "decode.cuh"
@@ -64,6 +70,15 @@ struct StepArgs {
   float *qhat;       // [rows, G, D], pre-scaled by scale * log2(e)
   float *u;          // [rows, D], zero beyond d
 };
+
+// The decode kernel rotates its own queries when the rotation's scratch
+// ((kThreads/D + 1) * G * D floats) fits in the histogram words; larger query
+// groups take q_hat and u from the rotate grid below.
+template <int G>
+constexpr bool kRotateInKernel = G <= 4;
+static_assert((kThreads / 64 + 1) * 4 * 64 <= skewed_words(kDig1Bins) &&
+                  (kThreads / 128 + 1) * 4 * 128 <= skewed_words(kDig1Bins),
+              "the in-kernel rotation's scratch fits in the histogram words");
 
 // ---------------------------------------------------------------------------
 // rotate: CTA (row, cb) computes columns [32cb, 32cb + 32) of q_hat for the G
@@ -368,10 +383,20 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
 
   // 1. key stream: its first stages go in flight before the wait for the
   // rotate grid, whose low-rank group query u the stream needs
-  LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
+  if constexpr (kRotateInKernel<G>) {
+    // q_hat and u from q and P_g here (the histogram words are scratch until
+    // zeroed), with the stream's first stages in flight behind the loads
+    rotate_queries<T, D, G>(a.da, b, g, qhat, u, reinterpret_cast<float *>(hist), true, [&] {
+      LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
+    });
+  } else {
+    // q_hat and u from the rotate grid (a programmatic dependency)
+    LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
+    griddep_wait();
+    if (tid < D) u[tid] = __ldcg(a.u + (size_t)row * D + tid);
+    for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
+  }
   for (int e = tid; e < skewed_words(kDig1Bins); e += kThreads) hist[e] = 0u;
-  griddep_wait();  // u and q_hat are written
-  if (tid < D) u[tid] = __ldcg(a.u + (size_t)row * D + tid);
   __syncthreads();
   cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
@@ -648,7 +673,6 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   for (int i = tid; i < s1 - s0; i += kThreads) ids[i] = min(max(__ldcg(idx_row + s0 + i), 0), S - 1);
   }  // gather / candidate paths
 
-  for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
   // 3. attention over this CTA's even share of the k selected rows (the
   // share is at most chunk)
   __syncthreads();

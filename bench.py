@@ -4,7 +4,8 @@
 
 One timed step = one Loki decode layer-step (rotate q, low-rank scores, top-k,
 gather attention, combine) through the C ABI on a cache already resident in
-HBM.  Each step also appends the step's new token first (timed separately) and
+HBM: one kernel for query groups of up to 4 heads, a rotate + decode pair for
+groups of 8.  Each step also appends the step's new token first (timed separately) and
 runs the in-library dense decode on the same cache (timed separately).  L2 is
 flushed before every step by writing a buffer twice the L2 size; the flush is
 outside the timed events.  Device time from CUDA events on the launching
@@ -457,7 +458,8 @@ def run_ours(args):
             "hbm_gbs": ach,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                          "traffic": measured_traffic("loki_decode_step", w.name),
-                         "kernel": "loki_rotate_kernel + loki_decode_kernel (programmatic dependent pair)",
+                         "kernel": ("loki_decode_kernel (rotates its own queries)" if rot == 0 else
+                                    "loki_rotate_kernel + loki_decode_kernel (programmatic dependent pair)"),
                          "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
                          "algorithmic_bytes_per_launch": lb},
             "dense": {"us": dense_us, "hbm_gbs": dach, "frac": dach / peak, "bytes_per_launch": db,
@@ -473,7 +475,7 @@ def run_ours(args):
             "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256},
             "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gpu_launches": 4 * K,  # timed loop: append, rotate, decode, dense
+            "gpu_launches": (3 if rot == 0 else 4) * K,  # timed loop: append, [rotate,] decode, dense
             "clocks": clocks,
             "wall_s_timed_region": wall,
             "per_step_loki_us": {"p50": float(np.percentile(per_step_loki, 50)) * 1000.0,

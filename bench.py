@@ -420,6 +420,38 @@ def run_ours(args):
         for i in range(n):
             t_exact += ex_ev[i][0].elapsed_time(ex_ev[i][1])
         done += n
+    # ---------------- generation steps that append their token inside the call
+    ga_steps = min(args.steps, 1000)
+    kn3 = [x.view(B, Hkv, D) for x in kn]
+    vn3 = [x.view(B, Hkv, D) for x in vn]
+    for i in range(args.warmup):
+        L.loki_decode_attention_append(cache, S, kn3[i % NSET], vn3[i % NSET], qs[i % NSET], P, w.d, w.k,
+                                       out=out, idx=idx)
+        L.dense_decode_attention_append(cache, S, kn3[i % NSET], vn3[i % NSET], qs[i % NSET], P, out=dout)
+    torch.cuda.synchronize()
+    ga_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(min(CH, ga_steps))]
+    t_ga = t_gd = 0.0
+    done = 0
+    while done < ga_steps:
+        n = min(CH, ga_steps - done)
+        for i in range(n):
+            j = (done + i) % NSET
+            flush.fill_(float(i & 7))
+            ga_ev[i][0].record(stream)
+            L.loki_decode_attention_append(cache, S, kn3[j], vn3[j], qs[j], P, w.d, w.k, out=out, idx=idx)
+            ga_ev[i][1].record(stream)
+            flush.fill_(float((i + 1) & 7))
+            ga_ev[i][2].record(stream)
+            L.dense_decode_attention_append(cache, S, kn3[j], vn3[j], qs[j], P, out=dout)
+            ga_end = torch.cuda.Event(enable_timing=True)
+            ga_end.record(stream)
+            ga_ev[i].append(ga_end)
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_ga += ga_ev[i][0].elapsed_time(ga_ev[i][1])
+            t_gd += ga_ev[i][2].elapsed_time(ga_ev[i][3])
+            del ga_ev[i][3:]
+        done += n
     # ---------------- the same step on a paged copy of the cache (16-token pages, shuffled)
     paged = time_paged(L, w, cache, qs, P, flush, stream, dev, steps=min(args.steps, 500), warmup=args.warmup)
     jac = []
@@ -466,6 +498,10 @@ def run_ours(args):
                       "launch": {"cluster_ctas": dcl, "ctas": dct}},
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
             "append_us": app_us,
+            "step_with_append": {"loki_us": t_ga * 1000.0 / ga_steps, "dense_us": t_gd * 1000.0 / ga_steps,
+                                 "loki_separate_us": app_us + loki_us, "steps": ga_steps,
+                                 "note": "token appended inside the decode call (loki_decode_attention_append, "
+                                         "dense_decode_attention_append) vs loki_append followed by the step"},
             "prefill_append": None if prefill is None else dict(prefill, frac=prefill["hbm_gbs"] / peak),
             "pca_calibrate": pca,
             "paged": dict(paged, frac=paged["hbm_gbs"] / peak),

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 8
+#define LOKI_VERSION 9
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -169,6 +169,36 @@ LOKI_API loki_status dense_decode_attention(const loki_cache *cache, int32_t seq
                                    const float *P, float scale, float *out,
                                    void *stream);
 
+/* loki_decode_attention_append -- one generation step: append the step's
+ * token to every row, then the Loki step of loki_decode_attention over
+ * tokens [0, seq_len), the new token being token seq_len - 1.  The pages
+ * time the cache append apart from attention (summary page, "Key results")
+ * and find it dominates inference time in a Hugging Face setup ("Surprising
+ * findings"); here it happens inside the decode kernel.
+ *   k_new : [B, Hkv, D] the new keys, NOT rotated, in the cache dtype;
+ *   v_new : [B, Hkv, D] the new values; both 16-byte aligned.
+ * Position seq_len - 1 of k_hat receives k_new . P_g rounded to the cache
+ * dtype (the arithmetic of loki_append up to the fp32 summation order) and
+ * of v receives v_new; the new token is scored, selected and attended like
+ * any other.  Other arguments as loki_decode_attention.  One kernel for query
+ * groups of up to 4 heads (the CTA that owns the last position rotates and
+ * stores the token); for 8, the append kernel and then the two decode
+ * kernels. */
+LOKI_API loki_status loki_decode_attention_append(const loki_cache *cache, int32_t seq_len,
+                                         int32_t n_q_heads, const void *k_new,
+                                         const void *v_new, const void *q, const float *P,
+                                         int32_t d, int32_t k, float scale, float *out,
+                                         int32_t *idx, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
+/* dense_decode_attention_append -- the same generation step for the full
+ * attention baseline: append the token at position seq_len - 1 of every row,
+ * then dense_decode_attention over [0, seq_len).  One kernel. */
+LOKI_API loki_status dense_decode_attention_append(const loki_cache *cache, int32_t seq_len,
+                                          int32_t n_q_heads, const void *k_new,
+                                          const void *v_new, const void *q, const float *P,
+                                          float scale, float *out, void *stream);
+
 /* loki_device_error_count -- the number of bounded device-side waits that
  * have timed out in this process on the current device since the library was
  * loaded (a kernel that times out records it here, releases what it holds and
@@ -268,6 +298,19 @@ LOKI_API loki_status loki_paged_decode_attention(const loki_paged_cache *cache,
                                         const int32_t *ks, int32_t k_max, float scale,
                                         float *out, int32_t *idx, void *workspace,
                                         size_t workspace_bytes, void *stream);
+
+/* loki_paged_decode_attention_append -- loki_decode_attention_append on a
+ * paged cache: sequence b's new token (k_new[b], v_new[b], [B, Hkv, D]) is
+ * written at its position seq_lens[b] - 1, then the step attends tokens
+ * [0, seq_lens[b]).  Query groups of up to 4 heads (else
+ * LOKI_ERR_UNSUPPORTED).  Other arguments as loki_paged_decode_attention. */
+LOKI_API loki_status loki_paged_decode_attention_append(const loki_paged_cache *cache,
+                                               const loki_seq_table *seqs, int32_t n_q_heads,
+                                               const void *k_new, const void *v_new,
+                                               const void *q, const float *P, int32_t d,
+                                               const int32_t *ks, int32_t k_max, float scale,
+                                               float *out, int32_t *idx, void *workspace,
+                                               size_t workspace_bytes, void *stream);
 
 /* dense_decode_attention on a paged cache with per-sequence lengths. */
 LOKI_API loki_status dense_paged_decode_attention(const loki_paged_cache *cache,

@@ -13,14 +13,17 @@ from .api import (
     PagedLokiCache,
     SeqTable,
     dense_decode_attention,
+    dense_decode_attention_append,
     dense_paged_decode_attention,
     loki_append,
     loki_decode_attention,
+    loki_decode_attention_append,
     loki_decode_attention_noalloc,
     loki_decode_launch_shape,
     loki_decode_workspace_size,
     loki_paged_append,
     loki_paged_decode_attention,
+    loki_paged_decode_attention_append,
     loki_pca_calibrate,
     loki_pca_workspace_size,
     loki_status_string,
@@ -38,6 +41,9 @@ __all__ = [
     "SeqTable",
     "loki_paged_append",
     "loki_paged_decode_attention",
+    "loki_paged_decode_attention_append",
+    "loki_decode_attention_append",
+    "dense_decode_attention_append",
     "dense_paged_decode_attention",
     "loki_append",
     "loki_decode_attention",

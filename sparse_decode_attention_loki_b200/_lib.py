@@ -68,6 +68,11 @@ SIGNATURES = {
     "loki_decode_attention_noalloc": (_i32, [_cache_p, _i32, _i32, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp,
                                              _vp]),
     "dense_decode_attention": (_i32, [_cache_p, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _vp]),
+    "loki_decode_attention_append": (_i32, [_cache_p, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, ctypes.c_float,
+                                            _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "dense_decode_attention_append": (_i32, [_cache_p, _i32, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp]),
+    "loki_paged_decode_attention_append": (_i32, [_pcache_p, _seqs_p, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32,
+                                                  ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "loki_topk_jaccard": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp]),
     "loki_device_error_count": (_i32, [ctypes.POINTER(ctypes.c_uint32)]),
     "loki_decode_launch_shape": (_i32, [_cache_p, _i32, _i32, _i32, _i32, ctypes.POINTER(_i32)]),

@@ -164,6 +164,59 @@ def dense_decode_attention(cache: LokiCache, seq_len: int, q: torch.Tensor, P: t
     return out
 
 
+def _need_token(cache, k_new: torch.Tensor, v_new: torch.Tensor, B: int) -> None:
+    shp = (B, cache.n_kv_heads, cache.head_dim)
+    _need(k_new, "k_new", cache.dtype, shp, cache.device)
+    _need(v_new, "v_new", cache.dtype, shp, cache.device)
+
+
+def loki_decode_attention_append(cache: LokiCache, seq_len: int, k_new: torch.Tensor, v_new: torch.Tensor,
+                                 q: torch.Tensor, P: torch.Tensor, d: int, k: int, scale: float = 0.0,
+                                 out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                                 workspace: Optional[torch.Tensor] = None,
+                                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One generation step: write the new token (k_new rotated by P, v_new;
+    both [B, Hkv, D]) at position seq_len - 1 of every row, then the Loki
+    step over tokens [0, seq_len).  Returns (out, idx) as
+    loki_decode_attention."""
+    B, Hq, D = q.shape if q.dim() == 3 else (-1, -1, -1)
+    _need(q, "q", cache.dtype, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    _need_token(cache, k_new, v_new, cache.batch)
+    if out is None:
+        out = torch.empty((cache.batch, Hq, cache.head_dim), dtype=torch.float32, device=cache.device)
+    if idx is None:
+        idx = torch.empty((cache.batch, cache.n_kv_heads, int(k)), dtype=torch.int32, device=cache.device)
+    _need(out, "out", torch.float32, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(idx, "idx", torch.int32, (cache.batch, cache.n_kv_heads, int(k)), cache.device)
+    if workspace is None:
+        workspace = cache.workspace(seq_len, Hq)
+    _lib.check(_lib.load().loki_decode_attention_append(
+        cache.desc(), int(seq_len), int(Hq), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(P), int(d), int(k),
+        float(scale), _ptr(out), _ptr(idx), _ptr(workspace), int(workspace.numel()),
+        _stream_ptr(cache.device, stream)))
+    return out, idx
+
+
+def dense_decode_attention_append(cache: LokiCache, seq_len: int, k_new: torch.Tensor, v_new: torch.Tensor,
+                                  q: torch.Tensor, P: torch.Tensor, scale: float = 0.0,
+                                  out: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The generation step of the full-attention baseline: append the new
+    token at position seq_len - 1, then attend tokens [0, seq_len)."""
+    B, Hq, D = q.shape if q.dim() == 3 else (-1, -1, -1)
+    _need(q, "q", cache.dtype, (cache.batch, Hq, cache.head_dim), cache.device)
+    _need(P, "P", torch.float32, (cache.n_kv_heads, cache.head_dim, cache.head_dim), cache.device)
+    _need_token(cache, k_new, v_new, cache.batch)
+    if out is None:
+        out = torch.empty((cache.batch, Hq, cache.head_dim), dtype=torch.float32, device=cache.device)
+    _need(out, "out", torch.float32, (cache.batch, Hq, cache.head_dim), cache.device)
+    _lib.check(_lib.load().dense_decode_attention_append(
+        cache.desc(), int(seq_len), int(Hq), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(P), float(scale), _ptr(out),
+        _stream_ptr(cache.device, stream)))
+    return out
+
+
 def topk_jaccard(idx_a: torch.Tensor, idx_b: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """Per-row Jaccard similarity of two selections [..., k] int32 (ascending
     rows, as loki_decode_attention returns them).  Returns float32 [...]: the
@@ -279,6 +332,43 @@ def loki_paged_decode_attention(cache: PagedLokiCache, seqs: SeqTable, q: torch.
                                                _ptr(out), _ptr(idx), _ptr(workspace),
                                                workspace.numel() * workspace.element_size(),
                                                _stream_ptr(cache.device, stream)))
+    return out, idx
+
+
+def loki_paged_decode_attention_append(cache: PagedLokiCache, seqs: SeqTable, k_new: torch.Tensor,
+                                       v_new: torch.Tensor, q: torch.Tensor, P: torch.Tensor, d: int, k_max: int,
+                                       ks: Optional[torch.Tensor] = None, scale: float = 0.0,
+                                       out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                                       workspace: Optional[torch.Tensor] = None,
+                                       stream: Optional[torch.cuda.Stream] = None
+                                       ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One generation step on a paged cache: sequence b's new token (k_new[b],
+    v_new[b], [B, Hkv, D]) goes to its position seq_lens[b] - 1, then the Loki
+    step over its seq_lens[b] tokens."""
+    B, Hkv, D = seqs.batch, cache.n_kv_heads, cache.head_dim
+    if q.dim() != 3 or q.shape[0] != B or q.shape[2] != D:
+        raise ValueError(f"q must be [B={B}, Hq, D={D}], got {tuple(q.shape)}")
+    Hq = int(q.shape[1])
+    _need(q, "q", cache.dtype, (B, Hq, D), cache.device)
+    _need(P, "P", torch.float32, (Hkv, D, D), cache.device)
+    _need_token(cache, k_new, v_new, B)
+    if ks is not None:
+        _need(ks, "ks", torch.int32, (B,), cache.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=cache.device)
+    if idx is None:
+        idx = torch.empty((B, Hkv, int(k_max)), dtype=torch.int32, device=cache.device)
+    _need(out, "out", torch.float32, (B, Hq, D), cache.device)
+    _need(idx, "idx", torch.int32, (B, Hkv, int(k_max)), cache.device)
+    n = ctypes.c_size_t(0)
+    lib = _lib.load()
+    _lib.check(lib.loki_paged_decode_workspace_size(cache.desc(), seqs.desc(), Hq, ctypes.byref(n)))
+    if workspace is None or workspace.numel() * workspace.element_size() < n.value:
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=cache.device)
+    _lib.check(lib.loki_paged_decode_attention_append(
+        cache.desc(), seqs.desc(), Hq, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(P), int(d),
+        _ptr(ks) if ks is not None else None, int(k_max), float(scale), _ptr(out), _ptr(idx), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream_ptr(cache.device, stream)))
     return out, idx
 
 

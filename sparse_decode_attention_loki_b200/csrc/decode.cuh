@@ -53,6 +53,10 @@ struct DecodeArgs {
   int32_t pages_per_seq;
   int32_t page_shift;       // page size = 1 << page_shift tokens
   int32_t num_pages;
+  // a new token of every row, appended by the decode call itself at the
+  // row's last attended position (null: no append)
+  const T *k_new;           // [B, Hkv, D], not rotated
+  const T *v_new;           // [B, Hkv, D]
 };
 
 // Tokens of one (batch, KV head) row, by position.  Contiguous caches: rows
@@ -123,7 +127,8 @@ constexpr int kRingWords = kWarps * kWarpRingBytes / 4;
 __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 
 // rotation scratch: q staging + partial dot products
-__host__ __device__ inline int rot_words(int G, int D) { return G * D + (kThreads / D) * G * D; }
+// rotation scratch: G query heads and one appended key, then per-part sums
+__host__ __device__ constexpr int rot_words(int G, int D) { return (G + 1) * D * (1 + kThreads / D); }
 
 struct SmemLayout {
   int qhat, u, pm, pl, pacc, ctl, slots, ring, keys, words;
@@ -169,38 +174,57 @@ static_assert(kWarps == 8, "ctl layout assumes 8 warps");
 template <typename T, int D, int G, typename F>
 __device__ __forceinline__ void rotate_queries(const DecodeArgs<T> &a, int b, int g,
                                                float *qhat, float *u, float *scratch,
-                                               bool want_u, F &&after_loads) {
+                                               bool want_u, F &&after_loads, const T *xk = nullptr,
+                                               float *xk_hat = nullptr) {
   const int tid = threadIdx.x;
   const int Hq = a.n_kv_heads * G;
   const T *qg = a.q + ((size_t)b * Hq + (size_t)g * G) * D;
   constexpr int PARTS = kThreads / D;
   constexpr int IPP = D / PARTS;
+  constexpr int NH = G + 1;  // query heads, then the appended key (when xk)
   const int j = tid % D, part = tid / D;
   const float *Pg = a.P + (size_t)g * D * D + (size_t)part * IPP * D + j;
   float pv[IPP];
 #pragma unroll
   for (int ii = 0; ii < IPP; ++ii) pv[ii] = __ldg(Pg + (size_t)ii * D);
-  float *qs = scratch;  // [G][D]
+  float *qs = scratch;  // [NH][D]
   for (int i = tid; i < G * D; i += kThreads) qs[i] = to_f32(qg[i]);
+  if (xk != nullptr)
+    for (int i = tid; i < D; i += kThreads) qs[G * D + i] = to_f32(xk[i]);
   after_loads();
   __syncthreads();
   float acc[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) acc[h] = 0.f;
+  float accx = 0.f;
 #pragma unroll
   for (int ii = 0; ii < IPP; ++ii) {
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = fmaf(qs[h * D + part * IPP + ii], pv[ii], acc[h]);
   }
-  float *red = scratch + G * D;  // [PARTS][G][D]
+  if (xk != nullptr) {
 #pragma unroll
-  for (int h = 0; h < G; ++h) red[(part * G + h) * D + j] = acc[h];
+    for (int ii = 0; ii < IPP; ++ii) accx = fmaf(qs[G * D + part * IPP + ii], pv[ii], accx);
+  }
+  float *red = scratch + NH * D;  // [PARTS][NH][D]
+#pragma unroll
+  for (int h = 0; h < G; ++h) red[(part * NH + h) * D + j] = acc[h];
+  if (xk != nullptr) red[(part * NH + G) * D + j] = accx;
   __syncthreads();
   for (int e = tid; e < G * D; e += kThreads) {
+    const int h = e / D, jj = e % D;
     float s = 0.f;
 #pragma unroll
-    for (int p = 0; p < PARTS; ++p) s += red[p * G * D + e];
+    for (int p = 0; p < PARTS; ++p) s += red[(p * NH + h) * D + jj];
     qhat[e] = s;
+  }
+  if (xk != nullptr) {
+    for (int jj = tid; jj < D; jj += kThreads) {
+      float s = 0.f;
+#pragma unroll
+      for (int p = 0; p < PARTS; ++p) s += red[(p * NH + G) * D + jj];
+      xk_hat[jj] = s;
+    }
   }
   __syncthreads();
   if (want_u) {
@@ -215,6 +239,26 @@ __device__ __forceinline__ void rotate_queries(const DecodeArgs<T> &a, int b, in
   }
   __syncthreads();
   for (int e = tid; e < G * D; e += kThreads) qhat[e] *= a.scale_log2;
+  __syncthreads();
+}
+
+// Write the appended token of row (b, g) into the cache at position t: its
+// rotated key xk_hat rounded to the cache dtype (xk_hat then holds the
+// rounded values, as fp32) and its value.  The cache is the caller's
+// writable memory; Rows hands out read pointers.  Ends with __syncthreads().
+template <typename T, int D, bool PAGED>
+__device__ __forceinline__ void store_appended(const DecodeArgs<T> &a, const Rows<T, D, PAGED> &rows, int b, int g,
+                                               int t, float *xk_hat) {
+  T *kd = const_cast<T *>(rows.key(t));
+  T *vd = const_cast<T *>(rows.val(t));
+  const T *vs = a.v_new + ((size_t)b * a.n_kv_heads + g) * D;
+  for (int i = threadIdx.x; i < D; i += kThreads) {
+    T r;
+    from_f32(xk_hat[i], &r);
+    kd[i] = r;
+    xk_hat[i] = to_f32(r);
+    vd[i] = vs[i];
+  }
   __syncthreads();
 }
 
@@ -784,6 +828,37 @@ __device__ __forceinline__ void attend_loop_any(const R &rows, const int32_t *id
   }
 }
 
+// Fold one more token into the CTA's merged attention state (pm, pl, pacc,
+// log2 domain with q_hat pre-scaled): kr holds its key as the fp32 values of
+// the stored cache entry, vs its value.  lg: G floats of scratch.  Starts and
+// ends with __syncthreads().
+template <typename T, int D, int G>
+__device__ __forceinline__ void fold_token(const float *qhat, const float *kr, const T *vs, float *pm, float *pl,
+                                           float *pacc, float *lg) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __syncthreads();
+  if (warp < G) {
+    float s = 0.f;
+    for (int i = lane; i < D; i += 32) s = fmaf(qhat[warp * D + i], kr[i], s);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
+    if (lane == 0) lg[warp] = s;
+  }
+  __syncthreads();
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int h = e / D;
+    const float m0 = pm[h], x = lg[h], M = fmaxf(m0, x);
+    pacc[e] = fmaf(pacc[e], exp2f(m0 - M), exp2f(x - M) * to_f32(vs[e - h * D]));
+  }
+  __syncthreads();  // every pm read before it changes
+  if (tid < G) {
+    const float m0 = pm[tid], x = lg[tid], M = fmaxf(m0, x);
+    pl[tid] = fmaf(pl[tid], exp2f(m0 - M), exp2f(x - M));
+    pm[tid] = M;
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
 // 5. log-sum-exp combine of the cluster's partial states: CTA r writes the
 //    output elements r*256 + t (stride ncta*256); each reads the (max, sum,
@@ -842,11 +917,19 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kerne
   const int t0 = min(S, rank * a.chunk);
   const int len = min(S, t0 + a.chunk) - t0;
   const Rows<T, D, PAGED> rows = make_rows<T, D, PAGED>(a, b, g);
-  rotate_queries<T, D, G>(a, b, g, qhat, u, scratch, false, [&] {
-    attend_prologue_any<T, D, G, false>(rows, nullptr, t0, len, ring);
-  });
-  attend_loop_any<T, D, G, false>(rows, nullptr, t0, len, qhat, reinterpret_cast<unsigned char *>(scratch), ring,
+  // an appended token sits at the row's last position: the CTA that owns it
+  // rotates and stores it, streams the rest and folds it in at the end
+  const bool own = a.k_new != nullptr && len > 0 && S - 1 < t0 + len;
+  const int slen = own ? len - 1 : len;
+  const size_t nv = ((size_t)b * a.n_kv_heads + g) * D;
+  float *xkh = u;  // the dense kernel has no low-rank query
+  rotate_queries<T, D, G>(
+      a, b, g, qhat, u, scratch, false, [&] { attend_prologue_any<T, D, G, false>(rows, nullptr, t0, slen, ring); },
+      own ? a.k_new + nv : nullptr, xkh);
+  if (own) store_appended<T, D, PAGED>(a, rows, b, g, S - 1, xkh);
+  attend_loop_any<T, D, G, false>(rows, nullptr, t0, slen, qhat, reinterpret_cast<unsigned char *>(scratch), ring,
                                   pm, pl, pacc);
+  if (own) fold_token<T, D, G>(qhat, xkh, a.v_new + nv, pm, pl, pacc, scratch);
   cluster.sync();
   const int Hq = a.n_kv_heads * G;
   cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);

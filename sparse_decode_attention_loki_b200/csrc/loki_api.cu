@@ -400,9 +400,36 @@ loki_status dispatch_p(bool dense, const DevInfo &di, const DecodeShape &sh, con
   return s;
 }
 
+template <typename T, int D, bool PAGED>
+loki_status launch_append(AppendArgs<T> a, void *stream);
+
 template <typename T, int D, int G>
 loki_status dispatch(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
                      void *stream, Plan *used) {
+  if (!dense && a.k_new != nullptr && !kRotateInKernel<G>) {
+    // the decode kernel appends only for query groups of up to 4 heads: for
+    // 8, the append kernel writes the new token first (contiguous caches)
+    if (a.table != nullptr)
+      return fail(LOKI_ERR_UNSUPPORTED, "appending in a paged Loki decode needs query groups of up to 4 heads");
+    if (used == nullptr) {
+      AppendArgs<T> ap{};
+      ap.k_hat = const_cast<T *>(a.k_hat);
+      ap.v = const_cast<T *>(a.v);
+      ap.k_new = a.k_new;
+      ap.v_new = a.v_new;
+      ap.P = a.P;
+      ap.n_kv_heads = a.n_kv_heads;
+      ap.capacity = a.capacity;
+      ap.pos = sh.S - 1;
+      ap.n_new = 1;
+      ap.n_vec = sh.B;
+      loki_status s = launch_append<T, D, false>(ap, stream);
+      if (s != LOKI_OK) return s;
+    }
+    DecodeArgs<T> rest = a;
+    rest.k_new = rest.v_new = nullptr;
+    return dispatch_p<T, D, G, false>(dense, di, sh, rest, ws, stream, used);
+  }
   if (a.table != nullptr) return dispatch_p<T, D, G, true>(dense, di, sh, a, ws, stream, used);
   return dispatch_p<T, D, G, false>(dense, di, sh, a, ws, stream, used);
 }
@@ -424,6 +451,7 @@ loki_status dispatch_g(bool dense, const DevInfo &di, const DecodeShape &sh, con
 struct VarPage {
   const int32_t *seq_lens = nullptr, *ks = nullptr, *table = nullptr;
   int32_t pages_per_seq = 0, page_shift = 0, num_pages = 0;
+  const void *k_new = nullptr, *v_new = nullptr;  // a token appended by the call, [B, Hkv, D]
 };
 
 template <typename T>
@@ -459,6 +487,8 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   a.pages_per_seq = vp.pages_per_seq;
   a.page_shift = vp.page_shift;
   a.num_pages = vp.num_pages;
+  a.k_new = static_cast<const T *>(vp.k_new);
+  a.v_new = static_cast<const T *>(vp.v_new);
   if (sh.D == 64) return dispatch_g<T, 64>(dense, di, sh, a, ws, stream, used);
   return dispatch_g<T, 128>(dense, di, sh, a, ws, stream, used);
 }
@@ -781,6 +811,56 @@ loki_status dense_decode_attention(const loki_cache *cache, int32_t seq_len, int
   return decode_common<__nv_bfloat16>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream);
 }
 
+static loki_status check_new_token(const void *k_new, const void *v_new) {
+  if (!k_new || !v_new) return fail(LOKI_ERR_INVALID_ARG, "k_new or v_new is NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(LOKI_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+  return LOKI_OK;
+}
+
+loki_status loki_decode_attention_append(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads,
+                                         const void *k_new, const void *v_new, const void *q, const float *P,
+                                         int32_t d, int32_t k, float scale, float *out, int32_t *idx, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+  DecodeShape sh;
+  loki_status s = check_decode(cache, seq_len, n_q_heads, q, P, out, &sh);
+  if (s != LOKI_OK) return s;
+  s = check_new_token(k_new, v_new);
+  if (s != LOKI_OK) return s;
+  if (d < 1 || d > sh.D) return fail(LOKI_ERR_INVALID_ARG, "d=%d outside [1, D=%d]", d, sh.D);
+  if (k < 1 || k > seq_len) return fail(LOKI_ERR_INVALID_ARG, "k=%d outside [1, seq_len=%d]", k, seq_len);
+  if (!idx) return fail(LOKI_ERR_INVALID_ARG, "idx is NULL");
+  if (!aligned(idx, 4)) return fail(LOKI_ERR_INVALID_ARG, "idx must be 4-byte aligned");
+  if (!workspace) return fail(LOKI_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(LOKI_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = ws_layout((long long)sh.B * sh.Hkv, sh.G, sh.D).total;
+  if (workspace_bytes < need)
+    return fail(LOKI_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes this call needs",
+                workspace_bytes, need);
+  VarPage vp;
+  vp.k_new = k_new;
+  vp.v_new = v_new;
+  if (cache->dtype == LOKI_F32)
+    return decode_common<float>(cache, sh, false, q, P, d, k, scale, out, idx, workspace, stream, nullptr, vp);
+  return decode_common<__nv_bfloat16>(cache, sh, false, q, P, d, k, scale, out, idx, workspace, stream, nullptr, vp);
+}
+
+loki_status dense_decode_attention_append(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads,
+                                          const void *k_new, const void *v_new, const void *q, const float *P,
+                                          float scale, float *out, void *stream) {
+  DecodeShape sh;
+  loki_status s = check_decode(cache, seq_len, n_q_heads, q, P, out, &sh);
+  if (s != LOKI_OK) return s;
+  s = check_new_token(k_new, v_new);
+  if (s != LOKI_OK) return s;
+  VarPage vp;
+  vp.k_new = k_new;
+  vp.v_new = v_new;
+  if (cache->dtype == LOKI_F32)
+    return decode_common<float>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream, nullptr, vp);
+  return decode_common<__nv_bfloat16>(cache, sh, true, q, P, 1, 1, scale, out, nullptr, nullptr, stream, nullptr, vp);
+}
+
 loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, int32_t n_q_heads, int32_t k,
                                      int32_t dense, int32_t *shape) {
   DecodeShape sh;
@@ -887,6 +967,42 @@ loki_status loki_paged_decode_attention(const loki_paged_cache *cache, const lok
     return fail(LOKI_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes this call needs",
                 workspace_bytes, need);
   const VarPage vp = paging_of(cache, seqs, shift, ks);
+  if (cache->dtype == LOKI_F32)
+    return decode_common<float>(&flat, sh, false, q, P, d, k_max, scale, out, idx, workspace, stream, nullptr, vp);
+  return decode_common<__nv_bfloat16>(&flat, sh, false, q, P, d, k_max, scale, out, idx, workspace, stream, nullptr,
+                                      vp);
+}
+
+loki_status loki_paged_decode_attention_append(const loki_paged_cache *cache, const loki_seq_table *seqs,
+                                               int32_t n_q_heads, const void *k_new, const void *v_new, const void *q,
+                                               const float *P, int32_t d, const int32_t *ks, int32_t k_max,
+                                               float scale, float *out, int32_t *idx, void *workspace,
+                                               size_t workspace_bytes, void *stream) {
+  loki_cache flat;
+  DecodeShape sh;
+  int shift = 0;
+  loki_status s = check_paged(cache, seqs, &flat, &sh, &shift);
+  if (s != LOKI_OK) return s;
+  s = check_decode(&flat, seqs->max_seq_len, n_q_heads, q, P, out, &sh);
+  if (s != LOKI_OK) return s;
+  s = check_new_token(k_new, v_new);
+  if (s != LOKI_OK) return s;
+  if (sh.G > 4)
+    return fail(LOKI_ERR_UNSUPPORTED, "appending in a paged Loki decode needs query groups of up to 4 heads");
+  if (d < 1 || d > sh.D) return fail(LOKI_ERR_INVALID_ARG, "d=%d outside [1, D=%d]", d, sh.D);
+  if (k_max < 1 || k_max > sh.S) return fail(LOKI_ERR_INVALID_ARG, "k_max=%d outside [1, max_seq_len=%d]", k_max, sh.S);
+  if (ks && !aligned(ks, 4)) return fail(LOKI_ERR_INVALID_ARG, "ks must be 4-byte aligned");
+  if (!idx) return fail(LOKI_ERR_INVALID_ARG, "idx is NULL");
+  if (!aligned(idx, 4)) return fail(LOKI_ERR_INVALID_ARG, "idx must be 4-byte aligned");
+  if (!workspace) return fail(LOKI_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(LOKI_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = ws_layout((long long)sh.B * sh.Hkv, sh.G, sh.D).total;
+  if (workspace_bytes < need)
+    return fail(LOKI_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes this call needs",
+                workspace_bytes, need);
+  VarPage vp = paging_of(cache, seqs, shift, ks);
+  vp.k_new = k_new;
+  vp.v_new = v_new;
   if (cache->dtype == LOKI_F32)
     return decode_common<float>(&flat, sh, false, q, P, d, k_max, scale, out, idx, workspace, stream, nullptr, vp);
   return decode_common<__nv_bfloat16>(&flat, sh, false, q, P, d, k_max, scale, out, idx, workspace, stream, nullptr,

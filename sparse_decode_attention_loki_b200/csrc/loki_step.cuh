@@ -71,14 +71,13 @@ struct StepArgs {
   float *u;          // [rows, D], zero beyond d
 };
 
-// The decode kernel rotates its own queries when the rotation's scratch
-// ((kThreads/D + 1) * G * D floats) fits in the histogram words; larger query
+// The decode kernel rotates its own queries (and an appended key) when the
+// rotation's scratch (rot_words) fits in the histogram words; larger query
 // groups take q_hat and u from the rotate grid below.
 template <int G>
 constexpr bool kRotateInKernel = G <= 4;
-static_assert((kThreads / 64 + 1) * 4 * 64 <= skewed_words(kDig1Bins) &&
-                  (kThreads / 128 + 1) * 4 * 128 <= skewed_words(kDig1Bins),
-              "the in-kernel rotation's scratch fits in the histogram words");
+static_assert(rot_words(4, 64) <= skewed_words(kDig1Bins) && rot_words(4, 128) <= skewed_words(kDig1Bins),
+              "the in-kernel rotation's scratch (queries and an appended key) fits in the histogram words");
 
 // ---------------------------------------------------------------------------
 // rotate: CTA (row, cb) computes columns [32cb, 32cb + 32) of q_hat for the G
@@ -383,12 +382,20 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
 
   // 1. key stream: its first stages go in flight before the wait for the
   // rotate grid, whose low-rank group query u the stream needs
+  // an appended token sits at the row's last position: the CTA that owns it
+  // rotates and stores it, streams the rest and scores it from the stored
+  // values (query groups of up to 4 heads; the host appends first for 8)
+  const bool own = kRotateInKernel<G> && a.da.k_new != nullptr && len > 0 && S - 1 < t0 + len;
+  const int slen = own ? len - 1 : len;
+  float *xkh = pacc;  // D floats, free until the attention
   if constexpr (kRotateInKernel<G>) {
     // q_hat and u from q and P_g here (the histogram words are scratch until
     // zeroed), with the stream's first stages in flight behind the loads
-    rotate_queries<T, D, G>(a.da, b, g, qhat, u, reinterpret_cast<float *>(hist), true, [&] {
-      LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
-    });
+    rotate_queries<T, D, G>(
+        a.da, b, g, qhat, u, reinterpret_cast<float *>(hist), true,
+        [&] { LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, slen, a.da.nck, ring))); },
+        own ? a.da.k_new + ((size_t)b * a.da.n_kv_heads + g) * D : nullptr, xkh);
+    if (own) store_appended<T, D, PAGED>(a.da, rows, b, g, S - 1, xkh);
   } else {
     // q_hat and u from the rotate grid (a programmatic dependency)
     LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
@@ -400,8 +407,23 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   __syncthreads();
   cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
-                    (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(rows, t0, len, a.da.nck,
+                    (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(rows, t0, slen, a.da.nck,
                                                                                        ring, u, keys, hist)));
+  if (own) {
+    // the appended token's key, from its stored (rounded) values
+    if (warp == 0) {
+      float sc = 0.f;
+      for (int i = lane; i < a.da.d; i += 32) sc = fmaf(u[i], xkh[i], sc);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
+      if (lane == 0) {
+        const uint32_t key = score_key(sc);
+        keys[len - 1] = key;
+        atomicAdd(&hist[hskew((int)(key >> (32 - kDig1Bits)))], 1u);
+      }
+    }
+    __syncthreads();
+  }
 
   // 2. cluster radix select; the ring is idle until the gather
   const bool leader = rank == 0;

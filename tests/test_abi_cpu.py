@@ -30,7 +30,8 @@ def test_header_declares_the_abi():
                           "loki_decode_attention_noalloc", "dense_decode_attention", "loki_decode_launch_shape",
                           "loki_topk_jaccard", "loki_device_error_count", "loki_pca_workspace_size",
                           "loki_paged_append", "loki_paged_decode_workspace_size", "loki_paged_decode_attention",
-                          "dense_paged_decode_attention",
+                          "dense_paged_decode_attention", "loki_decode_attention_append",
+                          "dense_decode_attention_append", "loki_paged_decode_attention_append",
                           "loki_pca_calibrate", "loki_status_string", "loki_last_error", "loki_version"}
 
 
@@ -52,7 +53,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 8
+    assert lib.loki_version() == 9
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -256,3 +257,24 @@ def test_paged_append_validation(lib):
     assert lib.loki_paged_append(ctypes.byref(c), ctypes.byref(q), FAKE, 1, FAKE, FAKE, None, None) == 1
     assert lib.loki_paged_append(ctypes.byref(_paged(page=3)), ctypes.byref(q), FAKE, 1, FAKE, FAKE, FAKE,
                                  None) == 1
+
+
+def test_append_decode_validation(lib):
+    c = _cache(B=1, H=2, cap=64)
+    need = _ws_bytes(2, 1, 128)
+    base = (ctypes.byref(c), 10, 2)
+    tail = (FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE, WS, need, None)
+    assert lib.loki_decode_attention_append(*base, None, FAKE, *tail) == 1
+    assert lib.loki_decode_attention_append(*base, FAKE, None, *tail) == 1
+    assert lib.loki_decode_attention_append(*base, FAKE + 8, FAKE, *tail) == 1
+    assert lib.loki_decode_attention_append(ctypes.byref(c), 65, 2, FAKE, FAKE, *tail) == 1   # seq_len > capacity
+    assert lib.loki_decode_attention_append(*base, FAKE, FAKE, FAKE, FAKE, 8, 11, 0.0, FAKE, FAKE, WS, need,
+                                            None) == 1   # k > seq_len
+    assert lib.dense_decode_attention_append(*base, None, FAKE, FAKE, FAKE, 0.0, FAKE, None) == 1
+    assert lib.dense_decode_attention_append(*base, FAKE, FAKE + 4, FAKE, FAKE, 0.0, FAKE, None) == 1
+    pc, pq = _paged(), _seqs()
+    pneed = _ws_bytes(4, 2, 128)
+    assert lib.loki_paged_decode_attention_append(ctypes.byref(pc), ctypes.byref(pq), 4, None, FAKE, FAKE, FAKE, 32,
+                                                  None, 10, 0.0, FAKE, FAKE, WS, pneed, None) == 1
+    assert lib.loki_paged_decode_attention_append(ctypes.byref(pc), ctypes.byref(pq), 16, FAKE, FAKE, FAKE, FAKE, 32,
+                                                  None, 10, 0.0, FAKE, FAKE, WS, _ws_bytes(4, 8, 128), None) == 2

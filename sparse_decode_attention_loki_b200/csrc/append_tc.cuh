@@ -20,8 +20,9 @@
 // j one thread issues the 3 * D/16 MMAs (K = 16 each) into one of two TMEM
 // accumulators and commits them to that accumulator's mbarrier; meanwhile
 // all sixteen warps read back tile j-1's accumulator (tcgen05.ld; warp w:
-// TMEM lanes 32*(w%4) .., columns of quarter w/4), round and store it, and
-// copy tile j's values.  Key tiles are staged three deep (cp.async), so two tiles
+// TMEM lanes 32*(w%4) .., columns of quarter w/4), round it into tile j-1's
+// key stage (free once its MMAs are done) and store it from there row by
+// row, coalesced, and copy tile j's values.  Key tiles are staged three deep (cp.async), so two tiles
 // of keys are in flight while one is being multiplied.
 //
 // Shared-memory operand layout (no swizzle, "K-major"): 8x16-byte core
@@ -225,29 +226,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_c
     if (__syncthreads_or(!ok)) return false;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const int u = lo + j, g = u / tiles, f0 = (u - g * tiles) * kTcM;
-    const int r = 32 * (warp & 3) + lane;
-    const int col0 = QC * (warp >> 2);
-    const uint32_t tacc = tbase + (uint32_t)((j & 1) * D) + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)col0;
-    __nv_bfloat16 *dst = nullptr;
-    if (f0 + r < a.n_vec) {
-      const int b0 = f0 / a.n_new;
-      int b, t;
-      tile_row(a.n_new, b0, f0 - b0 * a.n_new, r, b, t);
-      const long long off = dst_off(g, b, t);
-      if (off >= 0) dst = a.k_hat + off + col0;
-    }
+    // the accumulator, rounded, into tile j's key stage (its MMAs are done),
+    // rows of D*2 bytes with 16-byte chunk c of row r at chunk c ^ (r % CH):
+    // a warp's 32 rows then spread over all banks
+    unsigned char *stg = As + (j % kTcStages) * Lay::kA;
+    {
+      const int r = 32 * (warp & 3) + lane;
+      const int col0 = QC * (warp >> 2);
+      const uint32_t tacc = tbase + (uint32_t)((j & 1) * D) + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)col0;
 #pragma unroll
-    for (int cb = 0; cb < QC / 16; ++cb) {
-      uint32_t v[16];
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-          : "r"(tacc + (uint32_t)(16 * cb)));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      if (dst != nullptr) {
-        uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * cb);
+      for (int cb = 0; cb < QC / 16; ++cb) {
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(tacc + (uint32_t)(16 * cb)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           uint32_t w4[4];
@@ -257,11 +253,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_c
                 __floats2bfloat162_rn(__uint_as_float(v[8 * x + 2 * y]), __uint_as_float(v[8 * x + 2 * y + 1]));
             w4[y] = *reinterpret_cast<const uint32_t *>(&h);
           }
-          d4[x] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          const int c = (col0 + 16 * cb) / 8 + x;
+          *reinterpret_cast<uint4 *>(stg + r * (D * 2) + ((c ^ (r & (CH - 1))) * 16)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    // out to the cache, two whole rows per warp instruction
+    const int b0 = f0 / a.n_new, t0 = f0 - b0 * a.n_new;
+#pragma unroll
+    for (int x = 0; x < NV; ++x) {
+      const int r = crow + RS * x;
+      if (f0 + r < a.n_vec) {
+        int b, t;
+        tile_row(a.n_new, b0, t0, r, b, t);
+        const long long off = dst_off(g, b, t);
+        if (off >= 0)
+          reinterpret_cast<uint4 *>(a.k_hat + off)[cch] =
+              *reinterpret_cast<const uint4 *>(stg + r * (D * 2) + ((cch ^ (r & (CH - 1))) * 16));
+      }
+    }
+    __syncthreads();  // the stage is read before it is refilled
     return true;
   };
 

@@ -439,9 +439,15 @@ template <typename T, int D, bool GATHER, class R>
 __device__ __forceinline__ void attend_prologue(const R &rows, const int32_t *ids, int tok0, int cnt,
                                                 unsigned char *ring) {
   unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+  // a share that fits the ring goes in flight whole: one memory round trip
+  const bool whole = cnt <= kStages * kWarps * RowStream<T, D, GATHER>::TA;
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
     RowStream<T, D, GATHER>::issue(rows, ids, tok0, cnt, s, wring);
+    cp_async_commit();
+  }
+  if (whole) {
+    RowStream<T, D, GATHER>::issue(rows, ids, tok0, cnt, kStages - 1, wring);
     cp_async_commit();
   }
 }
@@ -475,11 +481,17 @@ __device__ __forceinline__ void attend_loop(const R &rows, const int32_t *ids, i
   }
 
   const int ns = RS::warp_stages(cnt);
+  const bool whole = cnt <= kStages * kWarps * RS::TA;  // the prologue issued every stage
   for (int s = 0; s < ns; ++s) {
-    cp_async_wait<kStages - 2>();
-    __syncwarp();
-    RS::issue(rows, ids, tok0, cnt, s + kStages - 1, wring);
-    cp_async_commit();
+    if (whole) {
+      if (s == 0) cp_async_wait<0>();
+      __syncwarp();
+    } else {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
+      RS::issue(rows, ids, tok0, cnt, s + kStages - 1, wring);
+      cp_async_commit();
+    }
     const unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
     const int base = (s * kWarps + warp) * RS::TA;
     float lg[U][G];
@@ -653,9 +665,15 @@ __device__ __forceinline__ void attend_mma_prologue(const R &rows, const int32_t
                                                     unsigned char *ring) {
   using RS = MmaRowStream<D, G, GATHER>;
   unsigned char *wring = ring + (threadIdx.x >> 5) * kWarpRingBytes;
+  // a share that fits the ring goes in flight whole: one memory round trip
+  const bool whole = cnt <= RS::NST * kWarps * RS::TILE;
 #pragma unroll
   for (int s = 0; s < RS::NST - 1; ++s) {
     RS::issue(rows, ids, tok0, cnt, s, wring);
+    cp_async_commit();
+  }
+  if (whole) {
+    RS::issue(rows, ids, tok0, cnt, RS::NST - 1, wring);
     cp_async_commit();
   }
 }
@@ -701,11 +719,17 @@ __device__ __forceinline__ void attend_mma_loop(const R &rows, const int32_t *id
 
   const int nt = RS::warp_tiles(cnt);
   const int r8 = lane & 7, mi = lane >> 3;
+  const bool whole = cnt <= RS::NST * kWarps * RS::TILE;  // the prologue issued every tile
   for (int s = 0; s < nt; ++s) {
-    cp_async_wait<RS::NST - 2>();
-    __syncwarp();
-    RS::issue(rows, ids, tok0, cnt, s + RS::NST - 1, wring);
-    cp_async_commit();
+    if (whole) {
+      if (s == 0) cp_async_wait<0>();
+      __syncwarp();
+    } else {
+      cp_async_wait<RS::NST - 2>();
+      __syncwarp();
+      RS::issue(rows, ids, tok0, cnt, s + RS::NST - 1, wring);
+      cp_async_commit();
+    }
     const unsigned char *st = wring + (s % RS::NST) * RS::TB;
     const int base = (s * kWarps + warp) * RS::TILE;
 

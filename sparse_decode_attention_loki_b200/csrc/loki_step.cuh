@@ -380,11 +380,11 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   const Rows<T, D, PAGED> rows = make_rows<T, D, PAGED>(a.da, b, g);
   constexpr int MAXL = D / VecN<T>::value;
 
-  // 1. key stream: its first stages go in flight before the wait for the
-  // rotate grid, whose low-rank group query u the stream needs
-  // an appended token sits at the row's last position: the CTA that owns it
-  // rotates and stores it, streams the rest and scores it from the stored
-  // values (query groups of up to 4 heads; the host appends first for 8)
+  // 1. the queries (q_hat, u) and the key stream; the stream's first stages
+  // go in flight before u is needed.  An appended token sits at the row's
+  // last position: the CTA that owns it rotates and stores it, streams the
+  // rest and scores it from the stored values (query groups of up to 4 heads;
+  // the host appends first for 8)
   const bool own = kRotateInKernel<G> && a.da.k_new != nullptr && len > 0 && S - 1 < t0 + len;
   const int slen = own ? len - 1 : len;
   float *xkh = pacc;  // D floats, free until the attention

@@ -48,12 +48,23 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(src: str) -> str:
+    """The source without comments and blank space, so that a comment edit
+    does not count as a kernel change (string literals hold no comment
+    markers in these files)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def source_hash() -> str:
+    """Hash of the kernel sources' code (comments and spacing ignored)."""
     h = hashlib.sha1()
     d = os.path.join(ROOT, "sparse_decode_attention_loki_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -541,6 +541,80 @@ def run_ours(args):
     return 0
 
 
+def run_sweep(args):
+    """Loki against the in-library dense kernel on every point of the
+    Mistral-7B-like sweep (S x B x d_f x k_f), one JSON line per point.  The
+    cache of one (S, B) serves its nine (d_f, k_f) points; device-timed with
+    CUDA events, L2 flushed before every call, median of args.sweep_reps."""
+    import torch
+
+    import sparse_decode_attention_loki_b200 as L
+    from sparse_decode_attention_loki_b200.calibration import pca_bases
+    from workloads import mistral_sweep_points
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    peak, _ = peaks()
+    pts = [w for w in mistral_sweep_points() if args.sweep_filter in w.name]
+    groups = {}
+    for w in pts:
+        groups.setdefault((w.seq_len, w.batch), []).append(w)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            flush.fill_(1.0)
+            fn()
+        ts = []
+        for i in range(reps):
+            flush.fill_(float(i & 7))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1000.0)
+        return float(np.median(ts))
+
+    for (S, B), ws in groups.items():
+        w0 = ws[0]
+        Hkv, Hq, D = w0.n_kv_heads, w0.n_q_heads, w0.head_dim
+        P = pca_bases([gen.calibration_keys(w0, g) for g in range(Hkv)]).to(dev)
+        cache = L.LokiCache(B, Hkv, D, S, dtype=torch.bfloat16, device=dev)
+        g_dev = torch.Generator(device=dev)
+        g_dev.manual_seed(w0.seed * 131)
+        for h in range(Hkv):  # one KV head at a time: the prompt never holds two full copies
+            k_h = gen.device_keys(gen.make_key_model(w0, h), B, S, g_dev, dev, torch.bfloat16)
+            v_h = torch.randn((B, S, D), generator=g_dev, device=dev).to(torch.bfloat16)
+            kk = torch.zeros((B, Hkv, S, D), dtype=torch.bfloat16, device=dev) if h == 0 else kk
+            vv = torch.zeros((B, Hkv, S, D), dtype=torch.bfloat16, device=dev) if h == 0 else vv
+            kk[:, h] = k_h
+            vv[:, h] = v_h
+            del k_h, v_h
+        L.loki_append(cache, 0, kk, vv, P)
+        del kk, vv
+        q = torch.randn((B, Hq, D), generator=g_dev, device=dev).to(torch.bfloat16)
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+        dense_us = timed(lambda: L.dense_decode_attention(cache, S, q, P, out=out), args.sweep_reps)
+        for w in ws:
+            idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
+            loki_us = timed(lambda: L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx),
+                            args.sweep_reps)
+            lb, db = w.loki_bytes(), w.dense_bytes()
+            print(json.dumps({"sweep": "mistral-7b-gqa", "workload": w.name, "seq_len": S, "batch": B,
+                              "d_f": w.d_f, "k_f": w.k_f, "d": w.d, "k": w.k, "loki_us": loki_us,
+                              "dense_us": dense_us, "speedup_vs_dense": dense_us / loki_us,
+                              "byte_ratio": db / lb, "loki_frac": lb / (loki_us * 1e-6) / 1e9 / peak,
+                              "dense_frac": db / (dense_us * 1e-6) / 1e9 / peak, "reps": args.sweep_reps,
+                              "l2": "flushed before every call"}), flush=True)
+        del cache
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -550,11 +624,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle CPU time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", choices=["mistral"], default=None,
+                    help="time Loki and dense on every Mistral sweep point instead of the bench step")
+    ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
+    ap.add_argument("--sweep-reps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps; the number is not a valid bench value", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 

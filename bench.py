@@ -82,6 +82,14 @@ def measured_traffic(kernel: str, workload: str):
     return None
 
 
+def lowrank_width(d, dtype, D):
+    """Width of the low-rank key plane a cache for reduced dimension d keeps:
+    d rounded up to whole 16-byte chunks (0 when that reaches D: no plane)."""
+    per = 8 if dtype == "bf16" else 4
+    d_lr = (d + per - 1) // per * per
+    return d_lr if d_lr < D else 0
+
+
 def workload_config(w, n_gpus):
     return {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * n_gpus,
             "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
@@ -214,8 +222,12 @@ def time_prefill(L, cache, k_pre, v_pre, P, stream, dev, reps: int = 5):
         if i >= 2:
             ts.append(e0.elapsed_time(e1) * 1000.0)
     us = float(np.median(ts))
-    nbytes = 4 * k_pre.numel() * k_pre.element_size()  # keys in, rotated keys out, values in, values out
+    # keys in, rotated keys out, values in, values out, and the low-rank plane's copy
+    nbytes = 4 * k_pre.numel() * k_pre.element_size()
+    if cache.k_lr is not None:
+        nbytes += k_pre.numel() // k_pre.shape[-1] * cache.d_lr * k_pre.element_size()
     return {"us": us, "vectors_per_kv_head": int(k_pre.shape[0] * k_pre.shape[2]), "bytes": nbytes,
+            "lowrank_plane": cache.d_lr,
             "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "reps": reps,
             "kernel": "append_tc_kernel" if (k_pre.dtype == torch.bfloat16
                                              and k_pre.shape[0] * k_pre.shape[2] >= 256) else "append_kernel"}
@@ -307,7 +319,9 @@ def run_ours(args):
     calib = [gen.calibration_keys(w, g) for g in range(Hkv)]
     P = pca_bases(calib).to(dev)
     pca = time_pca(L, calib, dev, stream)
-    cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev)
+    # the cache keeps a low-rank key plane as wide as d (contiguous score rows)
+    d_lr = lowrank_width(w.d, w.dtype, D)
+    cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, lowrank_dim=d_lr)
     g_dev = torch.Generator(device=dev)
     g_dev.manual_seed(w.seed * 131 + rank)
     if S > 1:
@@ -411,6 +425,27 @@ def run_ours(args):
         for i in range(n):
             t_e2e += e2e_ev[i][0].elapsed_time(e2e_ev[i][1])
         done += n
+    # ---------------- the same step on the same k_hat and v without the low-rank plane
+    cache_np = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, k_hat=cache.k_hat, v=cache.v)
+    np_steps = min(args.steps, 1000)
+    for i in range(args.warmup):
+        L.loki_decode_attention(cache_np, S, qs[i % NSET], P, w.d, w.k, out=out, idx=idx)
+    torch.cuda.synchronize()
+    np_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CH, np_steps))]
+    t_np = 0.0
+    done = 0
+    while done < np_steps:
+        n = min(CH, np_steps - done)
+        for i in range(n):
+            flush.fill_(float(i & 7))
+            np_ev[i][0].record(stream)
+            L.loki_decode_attention(cache_np, S, qs[(done + i) % NSET], P, w.d, w.k, out=out, idx=idx)
+            np_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_np += np_ev[i][0].elapsed_time(np_ev[i][1])
+        done += n
+    del cache_np
     # ---------------- Exact-TopK baseline (d = D) and the agreement of the two selections
     idx_exact = torch.empty_like(idx)
     for i in range(args.warmup):
@@ -508,6 +543,10 @@ def run_ours(args):
             "dense": {"us": dense_us, "hbm_gbs": dach, "frac": dach / peak, "bytes_per_launch": db,
                       "launch": {"cluster_ctas": dcl, "ctas": dct}},
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
+            "lowrank_plane": {"d_lr": d_lr, "bytes": B * Hkv * S * d_lr * (2 if w.dtype == "bf16" else 4),
+                              "no_plane_us": t_np * 1000.0 / np_steps, "no_plane_steps": np_steps,
+                              "note": "value streams the scores from the cache's low-rank key plane; "
+                                      "no_plane_us reads them from the k_hat rows (same results)"},
             "append_us": app_us,
             "step_with_append": {"loki_us": t_ga * 1000.0 / ga_steps, "dense_us": t_gd * 1000.0 / ga_steps,
                                  "loki_separate_us": app_us + loki_us, "steps": ga_steps,
@@ -597,20 +636,33 @@ def run_sweep(args):
         del kk, vv
         q = torch.randn((B, Hq, D), generator=g_dev, device=dev).to(torch.bfloat16)
         out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        # one low-rank plane per reduced dimension, each a view of the same k_hat and v
+        planes = {}
+        for w in ws:
+            d_lr = lowrank_width(w.d, "bf16", D)
+            if d_lr and d_lr not in planes:
+                c = L.LokiCache(B, Hkv, D, S, dtype=torch.bfloat16, device=dev, k_hat=cache.k_hat, v=cache.v,
+                                lowrank_dim=d_lr)
+                c.k_lr.copy_(cache.k_hat[..., :d_lr])
+                planes[d_lr] = c
         torch.cuda.synchronize()
         dense_us = timed(lambda: L.dense_decode_attention(cache, S, q, P, out=out), args.sweep_reps)
         for w in ws:
             idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
-            loki_us = timed(lambda: L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx),
+            lc = planes.get(lowrank_width(w.d, "bf16", D), cache)
+            loki_us = timed(lambda: L.loki_decode_attention(lc, S, q, P, w.d, w.k, out=out, idx=idx),
                             args.sweep_reps)
+            np_us = timed(lambda: L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx),
+                          args.sweep_reps)
             lb, db = w.loki_bytes(), w.dense_bytes()
             print(json.dumps({"sweep": "mistral-7b-gqa", "workload": w.name, "seq_len": S, "batch": B,
                               "d_f": w.d_f, "k_f": w.k_f, "d": w.d, "k": w.k, "loki_us": loki_us,
+                              "loki_no_plane_us": np_us, "d_lr": lc.d_lr,
                               "dense_us": dense_us, "speedup_vs_dense": dense_us / loki_us,
                               "byte_ratio": db / lb, "loki_frac": lb / (loki_us * 1e-6) / 1e9 / peak,
                               "dense_frac": db / (dense_us * 1e-6) / 1e9 / peak, "reps": args.sweep_reps,
                               "l2": "flushed before every call"}), flush=True)
-        del cache
+        del cache, planes
         torch.cuda.empty_cache()
     return 0
 

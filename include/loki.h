@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 9
+#define LOKI_VERSION 10
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -64,8 +64,21 @@ typedef enum { LOKI_F32 = 0, LOKI_BF16 = 1 } loki_dtype;
  *   k_hat : [B, Hkv, S_cap, D] keys already rotated into the PCA basis
  *           (k_hat = k . P_g), in `dtype`; 16-byte aligned.
  *   v     : [B, Hkv, S_cap, D] values, unrotated, in `dtype`; 16-byte aligned.
+ *   k_lr  : optional low-rank key plane, [B, Hkv, S_cap, d_lr] in `dtype`,
+ *           16-byte aligned, or NULL.  It holds a copy of the first d_lr
+ *           dimensions of every key row, k_lr[b][g][t][j] = k_hat[b][g][t][j]
+ *           for j < d_lr, kept by every call that writes keys (loki_append and
+ *           the *_append decode calls).  A Loki decode with d <= d_lr streams
+ *           the low-rank scores from it instead of from k_hat: HBM serves
+ *           reads in whole 128-byte lines, so reading d < 64 bf16 dimensions
+ *           of each 256-byte k_hat row costs a full line per token, while the
+ *           plane's rows are contiguous.  Results are bit-identical with and
+ *           without the plane.  Costs d_lr / D of the key cache in memory.
+ *   d_lr  : the plane's width, with d_lr * sizeof(dtype) a multiple of 16
+ *           bytes and d_lr <= D; ignored when k_lr is NULL.
  * The cache holds every token ever appended: entries are never evicted, so its
- * footprint equals a dense cache ("Limitations" section of the summary page). */
+ * footprint equals a dense cache ("Limitations" section of the summary page),
+ * plus the plane when there is one. */
 typedef struct {
   int32_t dtype;       /* loki_dtype                                          */
   int32_t batch;       /* B >= 1                                              */
@@ -74,6 +87,8 @@ typedef struct {
   int32_t capacity;    /* S_cap >= 1                                          */
   void *k_hat;
   void *v;
+  void *k_lr;          /* optional low-rank key plane, or NULL                */
+  int32_t d_lr;        /* its width (elements per token)                      */
 } loki_cache;
 
 /* loki_append -- rotate new keys into the PCA basis and append them, with
@@ -86,8 +101,9 @@ typedef struct {
  *                  principal direction of KV head g (column j = direction j,
  *                  sorted by descending eigenvalue).  16-byte aligned.
  * Computes k_hat[b][g][pos+t][j] = round_to_dtype( sum_i k_new[b][g][t][i] *
- * P[g][i][j] ) with fp32 accumulation and round-to-nearest-even, and copies
- * v_new unchanged.  Entries outside [pos, pos + n_new) are not touched.
+ * P[g][i][j] ) with fp32 accumulation and round-to-nearest-even, writes the
+ * same values for j < d_lr into the low-rank plane when the cache has one, and
+ * copies v_new unchanged.  Entries outside [pos, pos + n_new) are not touched.
  * bf16 caches with B * n_new >= 256 take the tensor-core path: P is split into
  * three bf16 terms (summing to P within 2^-27 relative) and the 3*D products
  * are accumulated in fp32 by tcgen05.mma before the single rounding.
@@ -126,7 +142,8 @@ LOKI_API loki_status loki_decode_workspace_size(const loki_cache *cache, int32_t
  * score_i = sum over the G query heads h of group g of q_hat_h[:d] . k_hat_i[:d];
  * the k tokens with the largest scores are selected, ties going to the lower
  * index; out_h = softmax(scale * q_hat_h . k_hat_i over the selected i, full D)
- * weighted sum of v_i.  Requires seq_len <= S_cap and G in {1, 2, 4, 8};
+ * weighted sum of v_i.  The scores read the cache's low-rank plane when it has
+ * one at least d wide, else k_hat; the gathered rows always come from k_hat.  Requires seq_len <= S_cap and G in {1, 2, 4, 8};
  * otherwise LOKI_ERR_INVALID_ARG or LOKI_ERR_UNSUPPORTED (also for seq_len
  * above 393216 tokens, whose scores would not fit on chip).  Enqueues one
  * kernel on the stream (query rotation, scores, selection, attention); for

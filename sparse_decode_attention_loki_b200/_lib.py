@@ -28,6 +28,8 @@ class loki_cache(ctypes.Structure):
         ("capacity", ctypes.c_int32),
         ("k_hat", ctypes.c_void_p),
         ("v", ctypes.c_void_p),
+        ("k_lr", ctypes.c_void_p),
+        ("d_lr", ctypes.c_int32),
     ]
 
 

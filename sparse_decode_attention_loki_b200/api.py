@@ -42,11 +42,18 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: Tuple[int, ...]
 class LokiCache:
     """A rotated-key KV cache in device memory: k_hat and v of shape
     [B, Hkv, capacity, D].  Keys are stored already rotated into the PCA basis;
-    nothing is ever evicted."""
+    nothing is ever evicted.
+
+    ``lowrank_dim`` (or an explicit ``k_lr`` of shape [B, Hkv, capacity, d_lr])
+    adds the low-rank key plane: a contiguous copy of the first d_lr dims of
+    every key, kept by every append, from which decodes with d <= d_lr stream
+    their scores (same results, fewer HBM lines read when d_lr * element size
+    is below 128 bytes)."""
 
     def __init__(self, batch: int, n_kv_heads: int, head_dim: int, capacity: int,
                  dtype: torch.dtype = torch.bfloat16, device=None,
-                 k_hat: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None):
+                 k_hat: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None,
+                 lowrank_dim: Optional[int] = None, k_lr: Optional[torch.Tensor] = None):
         if dtype not in _DTYPES:
             raise ValueError(f"cache dtype must be float32 or bfloat16, got {dtype}")
         device = torch.device(device if device is not None else "cuda")
@@ -62,8 +69,18 @@ class LokiCache:
         self.batch, self.n_kv_heads, self.head_dim, self.capacity = batch, n_kv_heads, head_dim, capacity
         self.dtype = dtype
         self.device = device
+        if k_lr is not None:
+            lowrank_dim = k_lr.shape[-1] if k_lr.dim() == 4 else -1
+        self.d_lr = int(lowrank_dim) if lowrank_dim else 0
+        if self.d_lr:
+            lshape = (batch, n_kv_heads, capacity, self.d_lr)
+            self.k_lr = k_lr if k_lr is not None else torch.empty(lshape, dtype=dtype, device=device)
+            _need(self.k_lr, "k_lr", dtype, lshape, device)
+        else:
+            self.k_lr = None
         self._desc = _lib.loki_cache(_DTYPES[dtype], batch, n_kv_heads, head_dim, capacity,
-                                     self.k_hat.data_ptr(), self.v.data_ptr())
+                                     self.k_hat.data_ptr(), self.v.data_ptr(),
+                                     self.k_lr.data_ptr() if self.k_lr is not None else None, self.d_lr)
 
     def desc(self) -> ctypes.POINTER(_lib.loki_cache):
         return ctypes.byref(self._desc)

@@ -24,6 +24,10 @@ struct AppendArgs {
   const T *k_new;    // [B, Hkv, n_new, D]
   const T *v_new;    // [B, Hkv, n_new, D]
   const float *P;    // [Hkv, D, D]
+  // the cache's low-rank key plane [B, Hkv, S_cap, d_lr] (contiguous caches;
+  // null: none): it receives the first d_lr dims of every appended key
+  T *k_lr;
+  int32_t d_lr;
   int32_t n_kv_heads;
   int32_t capacity;
   int32_t pos;
@@ -53,6 +57,13 @@ __device__ __forceinline__ long long append_dst(const AppendArgs<T> &a, int b, i
         min(max(__ldg(a.table + (size_t)b * a.pages_per_seq + (tok >> a.page_shift)), 0), a.num_pages - 1);
     return ((((long long)p * a.n_kv_heads + g) << a.page_shift) + (tok & ((1 << a.page_shift) - 1))) * D;
   }
+}
+
+// Element offset in the low-rank plane of new vector t of sequence b, head g
+// (contiguous caches).
+template <typename T>
+__device__ __forceinline__ long long append_lr_dst(const AppendArgs<T> &a, int b, int g, int t) {
+  return (((long long)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * a.d_lr;
 }
 
 constexpr int kAppendBatch = kWarps;   // vectors per batch: one per warp
@@ -107,6 +118,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
       const int b = f / a.n_new, t = f % a.n_new;
       const long long off = append_dst<T, D, PAGED>(a, b, g, t);
       if (off >= 0) from_f32(acc, a.k_hat + off + j);
+      if (!PAGED && a.k_lr != nullptr && j < a.d_lr) from_f32(acc, a.k_lr + append_lr_dst(a, b, g, t) + j);
     }
   }
 

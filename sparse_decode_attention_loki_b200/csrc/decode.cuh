@@ -57,6 +57,12 @@ struct DecodeArgs {
   // row's last attended position (null: no append)
   const T *k_new;           // [B, Hkv, D], not rotated
   const T *v_new;           // [B, Hkv, D]
+  // the cache's low-rank key plane [B, Hkv, S_cap, d_lr] (null: none;
+  // contiguous caches only), a copy of k_hat[..., :d_lr].  Written with every
+  // appended key; the score stream reads it when lr_read (d <= d_lr).
+  const T *k_lr;
+  int32_t d_lr;
+  bool lr_read;
 };
 
 // Tokens of one (batch, KV head) row, by position.  Contiguous caches: rows
@@ -66,6 +72,10 @@ struct DecodeArgs {
 template <typename T, int D, bool PAGED>
 struct Rows {
   const T *k, *v;        // contiguous: the row's token 0; paged: the pools
+  const T *s;            // contiguous: token 0 of the rows the score stream reads
+  T *lr;                 // contiguous: token 0 of the row's low-rank plane, or null
+  int32_t sstride;       // elements between the score rows of two tokens
+  int32_t d_lr;          // width of the low-rank plane
   const int32_t *table;  // paged: this sequence's page ids
   int32_t shift, hkv, g, last_page;
   __device__ __forceinline__ size_t off(int t) const {
@@ -78,6 +88,12 @@ struct Rows {
   }
   __device__ __forceinline__ const T *key(int t) const { return k + off(t); }
   __device__ __forceinline__ const T *val(int t) const { return v + off(t); }
+  // the first dims of token t's key as the score stream reads them: the
+  // low-rank plane's row when the call reads the plane, else the k_hat row
+  __device__ __forceinline__ const T *skey(int t) const {
+    if constexpr (!PAGED) return s + (size_t)t * sstride;
+    else return key(t);
+  }
 };
 
 template <typename T, int D, bool PAGED>
@@ -91,10 +107,19 @@ __device__ __forceinline__ Rows<T, D, PAGED> make_rows(const DecodeArgs<T> &a, i
     r.hkv = a.n_kv_heads;
     r.g = g;
     r.last_page = a.num_pages - 1;
+    r.s = nullptr;
+    r.lr = nullptr;
+    r.sstride = D;
+    r.d_lr = 0;
   } else {
-    const size_t off = ((size_t)b * a.n_kv_heads + g) * a.capacity * D;
+    const size_t row = (size_t)b * a.n_kv_heads + g;
+    const size_t off = row * a.capacity * D;
     r.k = a.k_hat + off;
     r.v = a.v + off;
+    r.lr = a.k_lr ? const_cast<T *>(a.k_lr) + row * a.capacity * a.d_lr : nullptr;
+    r.d_lr = a.k_lr ? a.d_lr : 0;
+    r.s = a.lr_read ? r.lr : r.k;
+    r.sstride = a.lr_read ? a.d_lr : D;
     r.table = nullptr;
     r.shift = r.hkv = r.g = r.last_page = 0;
   }
@@ -244,18 +269,21 @@ __device__ __forceinline__ void rotate_queries(const DecodeArgs<T> &a, int b, in
 
 // Write the appended token of row (b, g) into the cache at position t: its
 // rotated key xk_hat rounded to the cache dtype (xk_hat then holds the
-// rounded values, as fp32) and its value.  The cache is the caller's
+// rounded values, as fp32), the first d_lr of them into the low-rank plane
+// when the cache has one, and its value.  The cache is the caller's
 // writable memory; Rows hands out read pointers.  Ends with __syncthreads().
 template <typename T, int D, bool PAGED>
 __device__ __forceinline__ void store_appended(const DecodeArgs<T> &a, const Rows<T, D, PAGED> &rows, int b, int g,
                                                int t, float *xk_hat) {
   T *kd = const_cast<T *>(rows.key(t));
   T *vd = const_cast<T *>(rows.val(t));
+  T *ld = rows.lr ? rows.lr + (size_t)t * rows.d_lr : nullptr;
   const T *vs = a.v_new + ((size_t)b * a.n_kv_heads + g) * D;
   for (int i = threadIdx.x; i < D; i += kThreads) {
     T r;
     from_f32(xk_hat[i], &r);
     kd[i] = r;
+    if (ld != nullptr && i < rows.d_lr) ld[i] = r;
     xk_hat[i] = to_f32(r);
     vd[i] = vs[i];
   }
@@ -286,7 +314,7 @@ struct ScoreStream {
     for (int it = 0; it < TS * LPT / 32; ++it) {
       const int q = it * 32 + lane;
       const int t = q / LPT, c = q % LPT;
-      if (base + t < len && c < nck) cp_async16(st + q * 16, rows.key(t0 + base + t) + c * VEC);
+      if (base + t < len && c < nck) cp_async16(st + q * 16, rows.skey(t0 + base + t) + c * VEC);
     }
   }
 

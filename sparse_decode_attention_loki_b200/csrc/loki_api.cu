@@ -77,6 +77,7 @@ int env_int(const char *name, int dflt) {
 struct DecodeShape {
   int B, Hkv, D, Scap, S, Hq, G;
   size_t esize;
+  int d_lr;  // width of the cache's low-rank key plane, 0 without one
 };
 
 loki_status check_cache(const loki_cache *c, DecodeShape *sh) {
@@ -93,6 +94,15 @@ loki_status check_cache(const loki_cache *c, DecodeShape *sh) {
     return fail(LOKI_ERR_INVALID_ARG, "cache k_hat and v must be 16-byte aligned");
   if ((long long)c->batch * c->n_kv_heads > (1LL << 26))
     return fail(LOKI_ERR_UNSUPPORTED, "batch * n_kv_heads too large");
+  const int es = c->dtype == LOKI_F32 ? 4 : 2;
+  sh->d_lr = 0;
+  if (c->k_lr) {
+    if (c->d_lr < 1 || c->d_lr > c->head_dim || (c->d_lr * es) % 16 != 0)
+      return fail(LOKI_ERR_INVALID_ARG, "low-rank plane width d_lr=%d must be in [1, D=%d] with d_lr * %d bytes a "
+                  "multiple of 16", c->d_lr, c->head_dim, es);
+    if (!aligned(c->k_lr, 16)) return fail(LOKI_ERR_INVALID_ARG, "low-rank plane k_lr must be 16-byte aligned");
+    sh->d_lr = c->d_lr;
+  }
   sh->B = c->batch;
   sh->Hkv = c->n_kv_heads;
   sh->D = c->head_dim;
@@ -418,6 +428,8 @@ loki_status dispatch(bool dense, const DevInfo &di, const DecodeShape &sh, const
       ap.k_new = a.k_new;
       ap.v_new = a.v_new;
       ap.P = a.P;
+      ap.k_lr = const_cast<T *>(a.k_lr);
+      ap.d_lr = a.d_lr;
       ap.n_kv_heads = a.n_kv_heads;
       ap.capacity = a.capacity;
       ap.pos = sh.S - 1;
@@ -489,6 +501,9 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   a.num_pages = vp.num_pages;
   a.k_new = static_cast<const T *>(vp.k_new);
   a.v_new = static_cast<const T *>(vp.v_new);
+  a.k_lr = sh.d_lr > 0 ? static_cast<const T *>(c->k_lr) : nullptr;
+  a.d_lr = sh.d_lr;
+  a.lr_read = a.k_lr != nullptr && d <= sh.d_lr;
   if (sh.D == 64) return dispatch_g<T, 64>(dense, di, sh, a, ws, stream, used);
   return dispatch_g<T, 128>(dense, di, sh, a, ws, stream, used);
 }
@@ -562,6 +577,10 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   a.k_new = static_cast<const T *>(k_new);
   a.v_new = static_cast<const T *>(v_new);
   a.P = P;
+  if (c->k_lr) {
+    a.k_lr = static_cast<T *>(c->k_lr);
+    a.d_lr = c->d_lr;
+  }
   a.n_kv_heads = c->n_kv_heads;
   a.capacity = c->capacity;
   a.pos = pos;
@@ -629,6 +648,8 @@ loki_status check_paged(const loki_paged_cache *c, const loki_seq_table *q, loki
   flat->capacity = (int32_t)cap;
   flat->k_hat = c->k_hat;
   flat->v = c->v;
+  flat->k_lr = nullptr;  // paged pools have no low-rank plane
+  flat->d_lr = 0;
   loki_status s = check_cache(flat, sh);
   if (s != LOKI_OK) return s;
   int sft = 0;

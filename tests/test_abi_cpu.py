@@ -53,15 +53,15 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 9
+    assert lib.loki_version() == 10
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
 
 
-def _cache(dtype=1, B=1, H=2, D=128, cap=64, k=4096, v=8192):
+def _cache(dtype=1, B=1, H=2, D=128, cap=64, k=4096, v=8192, k_lr=None, d_lr=0):
     from sparse_decode_attention_loki_b200 import _lib
-    return _lib.loki_cache(dtype, B, H, D, cap, k, v)
+    return _lib.loki_cache(dtype, B, H, D, cap, k, v, k_lr, d_lr)
 
 
 FAKE = 1 << 20   # aligned non-null address; never dereferenced because validation fails first
@@ -278,3 +278,37 @@ def test_append_decode_validation(lib):
                                                   None, 10, 0.0, FAKE, FAKE, WS, pneed, None) == 1
     assert lib.loki_paged_decode_attention_append(ctypes.byref(pc), ctypes.byref(pq), 16, FAKE, FAKE, FAKE, FAKE, 32,
                                                   None, 10, 0.0, FAKE, FAKE, WS, _ws_bytes(4, 8, 128), None) == 2
+
+
+def test_cache_struct_layout():
+    # int32 x5, then three pointers from offset 24, then d_lr: the C layout
+    from sparse_decode_attention_loki_b200 import _lib
+    c = _lib.loki_cache
+    assert ctypes.sizeof(c) == 56
+    assert (c.k_hat.offset, c.v.offset, c.k_lr.offset, c.d_lr.offset) == (24, 32, 40, 48)
+
+
+@pytest.mark.parametrize("dtype,D,k_lr,d_lr,status", [
+    (1, 128, FAKE, 32, 0),        # bf16 plane of 32 dims (64-byte rows)
+    (1, 128, FAKE, 8, 0),         # 16-byte rows
+    (1, 128, FAKE, 128, 0),       # the whole key
+    (0, 64, FAKE, 4, 0),          # fp32: 16-byte rows
+    (1, 128, FAKE, 0, 1),         # empty plane
+    (1, 128, FAKE, 12, 1),        # 24-byte rows
+    (0, 64, FAKE, 6, 1),          # fp32 24-byte rows
+    (1, 128, FAKE, 136, 1),       # wider than the key
+    (1, 64, FAKE, 72, 1),
+    (1, 128, FAKE + 8, 32, 1),    # misaligned plane
+    (1, 128, None, 12, 0),        # no plane: d_lr is ignored
+])
+def test_lowrank_plane_validation(lib, dtype, D, k_lr, d_lr, status):
+    c = _cache(dtype=dtype, D=D, k_lr=k_lr, d_lr=d_lr)
+    n = ctypes.c_size_t(0)
+    assert lib.loki_decode_workspace_size(ctypes.byref(c), 10, 2, ctypes.byref(n)) == status
+    # the append and the decode validate the cache the same way (stopped
+    # before any launch by a bad range / a missing q)
+    assert lib.loki_append(ctypes.byref(c), 64, 1, FAKE, FAKE, FAKE, None) == 1
+    args = (ctypes.byref(c), 10, 2, None, FAKE, 8, 4, 0.0, FAKE, FAKE, WS, WSB, None)
+    assert lib.loki_decode_attention(*args) == 1
+    if status:
+        assert b"plane" in lib.loki_last_error()

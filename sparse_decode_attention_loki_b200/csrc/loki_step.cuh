@@ -351,6 +351,123 @@ __device__ __forceinline__ void write_selection_bal(const uint32_t *keys, int le
   }
 }
 
+// Per-warp token lists.  Once the first digit's bucket is known, every token
+// that can still be selected has key & mask >= prefix (above the bucket or in
+// it): a few times k/S of the tokens.  One ballot sweep compacts them, per
+// warp and in token order, into lists in the first-digit histogram's words
+// (free from then until the attention): warp w owns the same segment of the
+// tokens as in write_selection_bal and its list holds up to kListCap token
+// offsets (16 bits).  The refinement passes and the ordered write then visit
+// the lists instead of every token.
+constexpr int kCtlWarpN = 64;   // [64..71] entries of warp w's list
+constexpr int kCtlWarpAb = 72;  // [72..79] its tokens above the bucket
+constexpr int kCtlWarpCd = 80;  // [80..87] its tokens in the bucket
+constexpr int kListCap = 2 * skewed_words(kDig1Bins) / kWarps;  // 16-bit entries per warp
+static_assert(kListCap % 2 == 0 && kMaxChunk < 65536 && kGatherWords < 65536,
+              "list entries are 16-bit token offsets; each warp's list starts on a 4-byte boundary");
+
+// The lists of keys[0, len) for (prefix, mask).  Returns true (uniform over
+// the CTA) when every warp's list fit; the counts are in ctl either way.
+// Ends with __syncthreads().
+__device__ __forceinline__ bool list_sweep(const uint32_t *keys, int len, uint32_t prefix, uint32_t mask,
+                                           uint16_t *lists, uint32_t *ctl) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (((len + kWarps - 1) / kWarps) + 127) & ~127;
+  const int sbeg = min(len, warp * seg), send = min(len, sbeg + seg);
+  uint16_t *wl = lists + warp * kListCap;
+  const uint32_t lt = lanemask_lt();
+  uint32_t n = 0u, ab = 0u, cd = 0u;
+  for (int j0 = sbeg; j0 < send; j0 += 128) {
+    uint32_t gb[4], eb[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int j = j0 + 32 * x + lane;
+      const bool in = j < send;
+      const uint32_t km = in ? (keys[j] & mask) : 0u;
+      gb[x] = __ballot_sync(kFull, in && km > prefix);
+      eb[x] = __ballot_sync(kFull, in && km == prefix);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const uint32_t bx = gb[x] | eb[x];
+      const uint32_t p = n + __popc(bx & lt);
+      if (((bx >> lane) & 1u) != 0u && p < (uint32_t)kListCap) wl[p] = (uint16_t)(j0 + 32 * x + lane);
+      n += __popc(bx);
+      ab += __popc(gb[x]);
+      cd += __popc(eb[x]);
+    }
+  }
+  if (lane == 0) {
+    ctl[kCtlWarpN + warp] = n;
+    ctl[kCtlWarpAb + warp] = ab;
+    ctl[kCtlWarpCd + warp] = cd;
+  }
+  __syncthreads();
+  bool fit = true;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) fit &= ctl[kCtlWarpN + w] <= (uint32_t)kListCap;
+  return fit;
+}
+
+// write_selection_bal over the lists of list_sweep (which hold every token
+// the final (prefix, mask) can select, in token order).
+__device__ __forceinline__ void write_selection_list(const uint32_t *keys, const uint16_t *lists, int t0,
+                                                     const SelectState &st, uint32_t k, uint32_t *ctl,
+                                                     int32_t *idx_row) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t *wl = lists + warp * kListCap;
+  const int n = (int)ctl[kCtlWarpN + warp];
+  uint32_t gt = 0u, eq = 0u;
+  for (int i = lane; i < n; i += 32) {
+    const uint32_t km = keys[wl[i]] & st.mask;
+    gt += km > st.prefix;
+    eq += km == st.prefix;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    gt += __shfl_xor_sync(kFull, gt, off);
+    eq += __shfl_xor_sync(kFull, eq, off);
+  }
+  if (lane == 0) {
+    ctl[kCtlWarpGt + warp] = gt;
+    ctl[kCtlWarpEq + warp] = eq;
+  }
+  __syncthreads();
+  const uint32_t take = st.take;
+  uint32_t run_eq = 0u, run_sel = 0u;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t want = take > run_eq ? take - run_eq : 0u;
+    run_sel += ctl[kCtlWarpGt + w] + min(ctl[kCtlWarpEq + w], want);
+    run_eq += ctl[kCtlWarpEq + w];
+  }
+  int32_t *dst = idx_row + st.offset;
+  const uint32_t lt = lanemask_lt(), me = 1u << lane;
+  for (int i0 = 0; i0 < n; i0 += 64) {
+    // two ballots of 32 list entries in flight
+    uint32_t gb[2], eb[2];
+    int tok[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int i = i0 + 32 * x + lane;
+      const bool in = i < n;
+      tok[x] = in ? (int)wl[i] : 0;
+      const uint32_t km = in ? (keys[tok[x]] & st.mask) : 0u;
+      gb[x] = __ballot_sync(kFull, in && km > st.prefix);
+      eb[x] = __ballot_sync(kFull, in && km == st.prefix);
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const uint32_t left = take > run_eq ? take - run_eq : 0u;  // ties still taken
+      const uint32_t ties_below = __popc(eb[x] & lt);
+      const bool sel = (gb[x] & me) != 0u || ((eb[x] & me) != 0u && ties_below < left);
+      const uint32_t p = run_sel + __popc(gb[x] & lt) + min(ties_below, left);
+      if (sel && st.offset + p < k) dst[p] = t0 + tok[x];  // bound: the row holds k entries
+      run_sel += __popc(gb[x]) + min((uint32_t)__popc(eb[x]), left);
+      run_eq += __popc(eb[x]);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 template <typename T, int D, int G, bool PAGED>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel(const __grid_constant__ StepArgs<T> a) {
@@ -465,15 +582,28 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
       find_bucket(hist, kDig1Bins, k, ctl);
       uint32_t rem = k - ctl[kSelBucket + 1], inb = ctl[kSelBucket + 2];
       uint32_t pre = ctl[kSelBucket + 0] << (32 - kDig1Bits), msk = ~0u << (32 - kDig1Bits);
-      __syncthreads();  // ctl read before it is reused
+      // lists when they are likely to fit (tokens at or above the bucket: k - rem + inb)
+      const bool try_lists = k - rem + inb <= (uint32_t)(kWarps * kListCap * 3 / 4);
+      __syncthreads();  // ctl and the histogram read before they are reused
+      uint16_t *lists = reinterpret_cast<uint16_t *>(hist);
+      const bool listed = try_lists && list_sweep(all, S, pre, msk, lists, ctl);
       for (int pass = 0; pass < 2 && inb != rem; ++pass) {
         const int shift = pass == 0 ? SH2 : 0;
         const int nb = pass == 0 ? (1 << kDig2Bits) : (1 << kDig3Bits);
         for (int e = tid; e < skewed_words(1 << kDig2Bits); e += kThreads) href[e] = 0u;
         __syncthreads();
-        for (int i = tid; i < S; i += kThreads) {
-          const uint32_t key = all[i];
-          if ((key & msk) == pre) atomicAdd(&href[hskew((int)((key >> shift) & (uint32_t)(nb - 1)))], 1u);
+        if (listed) {
+          const uint16_t *wl = lists + warp * kListCap;
+          const int n = (int)ctl[kCtlWarpN + warp];
+          for (int i = lane; i < n; i += 32) {
+            const uint32_t key = all[wl[i]];
+            if ((key & msk) == pre) atomicAdd(&href[hskew((int)((key >> shift) & (uint32_t)(nb - 1)))], 1u);
+          }
+        } else {
+          for (int i = tid; i < S; i += kThreads) {
+            const uint32_t key = all[i];
+            if ((key & msk) == pre) atomicAdd(&href[hskew((int)((key >> shift) & (uint32_t)(nb - 1)))], 1u);
+          }
         }
         __syncthreads();
         find_bucket(href, nb, rem, ctl);
@@ -483,7 +613,10 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
         msk |= (uint32_t)(nb - 1) << shift;
         __syncthreads();  // ctl read before it is reused
       }
-      write_selection_bal(all, S, 0, SelectState{pre, msk, rem, 0u}, k, ctl, list);
+      if (listed)
+        write_selection_list(all, lists, 0, SelectState{pre, msk, rem, 0u}, k, ctl, list);
+      else
+        write_selection_bal(all, S, 0, SelectState{pre, msk, rem, 0u}, k, ctl, list);
     }
     cluster.sync();  // the leader's list of the k indices is complete (and it read every CTA's keys)
     const uint32_t src = dsmem_addr(list + s0, 0u);
@@ -517,8 +650,45 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   uint32_t *href = rw + kHref, *hdr = rw + kHdr;
 
   // this CTA's candidates (its keys in the bucket) into its slot at the
-  // leader, with its count of candidates and of keys above the bucket
-  {
+  // leader, with its count of candidates and of keys above the bucket: from
+  // the per-warp lists, or (when a list overflows) from sweeps of every key
+  uint16_t *lists = reinterpret_cast<uint16_t *>(hist);  // every histogram is dead from here to the attention
+  // lists when they are likely to fit: the cluster's tokens at or above the
+  // bucket number ctl[kSelFirst + 1] + ctl[kSelFirst + 2] (uniform decision)
+  const bool try_lists =
+      ctl[kSelFirst + 1] + ctl[kSelFirst + 2] <= (uint32_t)(ncta * kWarps * kListCap * 3 / 4);
+  const bool listed = try_lists && list_sweep(keys, len, prefix, mask, lists, ctl);
+  if (listed) {
+    uint32_t total = 0u, above = 0u, before = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const uint32_t c = ctl[kCtlWarpCd + w];
+      total += c;
+      above += ctl[kCtlWarpAb + w];
+      before += w < warp ? c : 0u;
+    }
+    if (refine && total <= (uint32_t)cap) {
+      // warp w's candidates at [before, before + its count) of the slot
+      const uint32_t slot = dsmem_addr(rw + kSlots + rank * cap, 0u);
+      const uint16_t *wl = lists + warp * kListCap;
+      const int n = (int)ctl[kCtlWarpN + warp];
+      const uint32_t lt = lanemask_lt();
+      uint32_t pos = before;
+      for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < n ? keys[wl[i]] : 0u;
+        const bool c = i < n && (key & mask) == prefix;
+        const uint32_t bc = __ballot_sync(kFull, c);
+        if (c) dsmem_st(slot + 4u * (pos + __popc(bc & lt)), key);
+        pos += __popc(bc);
+      }
+    }
+    if (tid == 0) {
+      const uint32_t h = dsmem_addr(hdr + 2 * rank, 0u);
+      dsmem_st(h, total);
+      dsmem_st(h + 4u, above);
+    }
+  } else {
     const int n4 = (len + 3) >> 2;
     uint32_t mine = 0u, above = 0u;
     for (int j4 = tid; j4 < n4; j4 += kThreads) {
@@ -686,7 +856,10 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     }
     take = min(eq, remaining > eq_before ? remaining - eq_before : 0u);
   }
-  write_selection_bal(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
+  if (listed)
+    write_selection_list(keys, lists, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
+  else
+    write_selection_bal(keys, len, t0, SelectState{prefix, mask, take, offset}, k, ctl, idx_row);
   // a row shorter than the longest one: the rest of its idx row is -1
   for (int i = (int)k + rank * kThreads + tid; i < a.da.k_stride; i += ncta * kThreads) idx_row[i] = -1;
   cluster.sync();  // the whole row of idx is written and visible to the cluster

@@ -226,6 +226,18 @@ def test_zero_query_selects_first_k(S, ncta):
         np.testing.assert_allclose(out[:, h], V[:, h // 4, :k].mean(axis=1), atol=5e-3)
 
 
+@pytest.mark.parametrize("S,k,ncta", [(6000, 600, None), (6000, 5000, None), (30000, 3000, 2), (30000, 15000, 2),
+                                     (30000, 3000, 16)])
+def test_select_lists_and_their_overflow(S, k, ncta):
+    # the select keeps per-warp lists of the tokens at or above the first
+    # digit's bucket; a large k overflows them (and the selection falls back
+    # to sweeps over every key), on short rows (one CTA selects all) and long
+    # ones (the cluster selects)
+    w = small_workload("bf16", 128, 2, S, Hkv=2, B=1, seed=S + k)
+    out, idx, ref, K_hat, V, *_ = run_decode(w, S, 32, k, ncta=ncta)
+    parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(128), "bf16")
+
+
 def test_full_budget_equals_dense():
     w = small_workload("bf16", 128, 4, 700)
     out, idx, ref, K_hat, V, inp, P32, cache, q, P = run_decode(w, 700, 128, 700)

@@ -442,27 +442,34 @@ def run_ours(args):
         for i in range(n):
             t_e2e += e2e_ev[i][0].elapsed_time(e2e_ev[i][1])
         done += n
-    # ---------------- the same step on the same k_hat and v without the low-rank plane
+    # ---------------- the decode alone, back to back (no other kernel of ours between two
+    # decodes), with and without the low-rank plane (same k_hat and v)
     cache_np = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, k_hat=cache.k_hat, v=cache.v)
     np_steps = min(args.steps, 1000)
-    for i in range(args.warmup):
-        L.loki_decode_attention(cache_np, S, qs[i % NSET], P, w.d, w.k, out=out, idx=idx)
-    torch.cuda.synchronize()
-    np_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CH, np_steps))]
-    t_np = 0.0
-    done = 0
-    while done < np_steps:
-        n = min(CH, np_steps - done)
-        queue_ahead(torch, n)
-        for i in range(n):
-            flush.fill_(float(i & 7))
-            np_ev[i][0].record(stream)
-            L.loki_decode_attention(cache_np, S, qs[(done + i) % NSET], P, w.d, w.k, out=out, idx=idx)
-            np_ev[i][1].record(stream)
+
+    def decode_only(c):
+        for i in range(args.warmup):
+            L.loki_decode_attention(c, S, qs[i % NSET], P, w.d, w.k, out=out, idx=idx)
         torch.cuda.synchronize()
-        for i in range(n):
-            t_np += np_ev[i][0].elapsed_time(np_ev[i][1])
-        done += n
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CH, np_steps))]
+        tot = 0.0
+        done = 0
+        while done < np_steps:
+            n = min(CH, np_steps - done)
+            queue_ahead(torch, n)
+            for i in range(n):
+                flush.fill_(float(i & 7))
+                ev[i][0].record(stream)
+                L.loki_decode_attention(c, S, qs[(done + i) % NSET], P, w.d, w.k, out=out, idx=idx)
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            for i in range(n):
+                tot += ev[i][0].elapsed_time(ev[i][1])
+            done += n
+        return tot * 1000.0 / np_steps
+
+    t_only = decode_only(cache)
+    t_np = decode_only(cache_np) * np_steps / 1000.0
     del cache_np
     # ---------------- Exact-TopK baseline (d = D) and the agreement of the two selections
     idx_exact = torch.empty_like(idx)
@@ -566,7 +573,14 @@ def run_ours(args):
             "lowrank_plane": {"d_lr": d_lr, "bytes": B * Hkv * S * d_lr * (2 if w.dtype == "bf16" else 4),
                               "no_plane_us": t_np * 1000.0 / np_steps, "no_plane_steps": np_steps,
                               "note": "value streams the scores from the cache's low-rank key plane; "
-                                      "no_plane_us reads them from the k_hat rows (same results)"},
+                                      "no_plane_us reads them from the k_hat rows (same results), "
+                                      "timed like decode_only_us"},
+            "decode_only_us": t_only,
+            "decode_only_note": "the same decode timed back to back with no other kernel of ours between "
+                                "two decodes; value is timed in the step loop (one-token append, decode, "
+                                "dense), where a dense kernel ran before each decode: that alone makes a "
+                                "short decode slower (state left on the SMs, most likely their "
+                                "instruction caches), even with the L2 flushed in between",
             "append_us": app_us,
             "step_with_append": {"loki_us": t_ga * 1000.0 / ga_steps, "dense_us": t_gd * 1000.0 / ga_steps,
                                  "loki_separate_us": app_us + loki_us, "steps": ga_steps,

@@ -5,10 +5,10 @@
 One timed step = one Loki decode layer-step (rotate q, low-rank scores, top-k,
 gather attention, combine) through the C ABI on a cache already resident in
 HBM: one kernel for query groups of up to 4 heads, a rotate + decode pair for
-groups of 8.  Each step also appends the step's new token first (timed separately) and
-runs the in-library dense decode on the same cache (timed separately).  L2 is
-flushed before every step by writing a buffer twice the L2 size; the flush is
-outside the timed events.  Device time from CUDA events on the launching
+groups of 8.  Each step also appends the step's new token first (timed separately).
+The in-library dense decode on the same cache is timed over K steps of its own.
+L2 is flushed before every step by writing a buffer twice the L2 size; the flush
+is outside the timed events.  Device time from CUDA events on the launching
 stream, summed over the K steps, max over ranks.
 
 With N GPUs (torchrun) each rank runs the whole workload on its own batch
@@ -361,7 +361,10 @@ def run_ours(args):
     flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
 
-    def step(i, ev=None):
+    # One Loki step: the one-token append, then the decode.  The dense baseline
+    # runs in a loop of its own (dense_step); `with_dense` runs it after the
+    # decode of the same step instead, for the interleaved figure.
+    def step(i, ev=None, with_dense=False):
         j = i % NSET
         flush.fill_(float(i & 7))
         if ev is not None:
@@ -372,17 +375,23 @@ def run_ours(args):
         L.loki_decode_attention(cache, S, qs[j], P, w.d, w.k, out=out, idx=idx)
         if ev is not None:
             ev[2].record(stream)
-        L.dense_decode_attention(cache, S, qs[j], P, out=dout)
-        if ev is not None:
-            ev[3].record(stream)
+        if with_dense:
+            L.dense_decode_attention(cache, S, qs[j], P, out=dout)
+
+    def dense_step(i, ev):
+        flush.fill_(float(i & 7))
+        ev[0].record(stream)
+        L.dense_decode_attention(cache, S, qs[i % NSET], P, out=dout)
+        ev[1].record(stream)
 
     for i in range(args.warmup):
         step(i)
+        L.dense_decode_attention(cache, S, qs[i % NSET], P, out=dout)
     torch.cuda.synchronize()
 
     # ---------------- device-timed region
     CH = CHUNK
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(min(CH, args.steps))]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(min(CH, args.steps))]
     t_app = t_loki = t_dense = 0.0
     per_step_loki = []
     pr = torch.cuda.get_device_properties(dev)
@@ -401,17 +410,40 @@ def run_ours(args):
         torch.cuda.synchronize()
         for i in range(n):
             e = evs[i]
-            a, b_, c = e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])
+            a, b_ = e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])
             t_app += a
             t_loki += b_
-            t_dense += c
             per_step_loki.append(b_)
         done += n
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     wall = time.perf_counter() - wall0
+    # the dense baseline, same steps, its own loop
+    done = 0
+    while done < args.steps:
+        n = min(CH, args.steps - done)
+        queue_ahead(torch, n)
+        for i in range(n):
+            dense_step(done + i, evs[i])
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_dense += evs[i][0].elapsed_time(evs[i][1])
+        done += n
     clocks = sampler.stop()
+    # the Loki step with the dense kernel run after each decode (interleaved)
+    il_steps = min(args.steps, 1000)
+    t_il = 0.0
+    done = 0
+    while done < il_steps:
+        n = min(CH, il_steps - done)
+        queue_ahead(torch, n)
+        for i in range(n):
+            step(done + i, evs[i], with_dense=True)
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_il += evs[i][1].elapsed_time(evs[i][2])
+        done += n
 
     # ---------------- end to end through host buffers (pinned), copies inside the events
     q_host = [q.cpu().pin_memory() for q in qs]
@@ -501,30 +533,30 @@ def run_ours(args):
                                        out=out, idx=idx)
         L.dense_decode_attention_append(cache, S, kn3[i % NSET], vn3[i % NSET], qs[i % NSET], P, out=dout)
     torch.cuda.synchronize()
-    ga_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(min(CH, ga_steps))]
-    t_ga = t_gd = 0.0
-    done = 0
-    while done < ga_steps:
-        n = min(CH, ga_steps - done)
-        queue_ahead(torch, n)
-        for i in range(n):
-            j = (done + i) % NSET
-            flush.fill_(float(i & 7))
-            ga_ev[i][0].record(stream)
-            L.loki_decode_attention_append(cache, S, kn3[j], vn3[j], qs[j], P, w.d, w.k, out=out, idx=idx)
-            ga_ev[i][1].record(stream)
-            flush.fill_(float((i + 1) & 7))
-            ga_ev[i][2].record(stream)
-            L.dense_decode_attention_append(cache, S, kn3[j], vn3[j], qs[j], P, out=dout)
-            ga_end = torch.cuda.Event(enable_timing=True)
-            ga_end.record(stream)
-            ga_ev[i].append(ga_end)
-        torch.cuda.synchronize()
-        for i in range(n):
-            t_ga += ga_ev[i][0].elapsed_time(ga_ev[i][1])
-            t_gd += ga_ev[i][2].elapsed_time(ga_ev[i][3])
-            del ga_ev[i][3:]
-        done += n
+    ga_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CH, ga_steps))]
+
+    def gen_loop(call):
+        tot = 0.0
+        done = 0
+        while done < ga_steps:
+            n = min(CH, ga_steps - done)
+            queue_ahead(torch, n)
+            for i in range(n):
+                j = (done + i) % NSET
+                flush.fill_(float(i & 7))
+                ga_ev[i][0].record(stream)
+                call(j)
+                ga_ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            for i in range(n):
+                tot += ga_ev[i][0].elapsed_time(ga_ev[i][1])
+            done += n
+        return tot
+
+    # each arm in a loop of its own, like the decode and the dense baseline
+    t_ga = gen_loop(lambda j: L.loki_decode_attention_append(cache, S, kn3[j], vn3[j], qs[j], P, w.d, w.k,
+                                                             out=out, idx=idx))
+    t_gd = gen_loop(lambda j: L.dense_decode_attention_append(cache, S, kn3[j], vn3[j], qs[j], P, out=dout))
     # ---------------- the same step on a paged copy of the cache (16-token pages, shuffled)
     paged = time_paged(L, w, cache, qs, P, flush, stream, dev, steps=min(args.steps, 500), warmup=args.warmup)
     jac = []
@@ -576,11 +608,11 @@ def run_ours(args):
                                       "no_plane_us reads them from the k_hat rows (same results), "
                                       "timed like decode_only_us"},
             "decode_only_us": t_only,
-            "decode_only_note": "the same decode timed back to back with no other kernel of ours between "
-                                "two decodes; value is timed in the step loop (one-token append, decode, "
-                                "dense), where a dense kernel ran before each decode: that alone makes a "
-                                "short decode slower (state left on the SMs, most likely their "
-                                "instruction caches), even with the L2 flushed in between",
+            "interleaved_with_dense_us": t_il * 1000.0 / il_steps,
+            "interleaved_note": "the step loop with the dense kernel run after each decode: a dense kernel "
+                                "before a decode slows a short decode (state left on the SMs, most likely "
+                                "their instruction caches), even with the L2 flushed in between; value and "
+                                "dense are timed in loops of their own",
             "append_us": app_us,
             "step_with_append": {"loki_us": t_ga * 1000.0 / ga_steps, "dense_us": t_gd * 1000.0 / ga_steps,
                                  "loki_separate_us": app_us + loki_us, "steps": ga_steps,
@@ -595,7 +627,7 @@ def run_ours(args):
             "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256},
             "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gpu_launches": (3 if rot == 0 else 4) * K,  # timed loop: append, [rotate,] decode, dense
+            "gpu_launches": (2 if rot == 0 else 3) * K,  # timed loop: append, [rotate,] decode
             "clocks": clocks,
             "wall_s_timed_region": wall,
             "per_step_loki_us": {"p50": float(np.percentile(per_step_loki, 50)) * 1000.0,

@@ -28,7 +28,10 @@
 //        lower index) and hands each CTA its (threshold, ties to take,
 //        offset); each CTA writes its indices in ascending order (should a
 //        CTA's candidates overflow its slot at the leader, the cluster
-//        refines with distributed histogram passes instead);
+//        refines with distributed histogram passes instead).  Once the
+//        first digit's bucket is known, both paths keep per-warp lists of
+//        the tokens at or above it and run their later passes and the
+//        ordered write over the lists;
 //     3. the k selected rows are split evenly over the cluster: gather K_hat
 //        and V rows through the ring, online softmax per query head;
 //     4. the CTAs' (max, sum, acc) states are merged through distributed

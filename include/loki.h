@@ -252,7 +252,9 @@ LOKI_API loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_
  * A paged rotated-key cache: fixed-size pages from one pool.
  *   k_hat : [num_pages, Hkv, page_size, D] rotated keys in `dtype`, 16-byte
  *           aligned; v : the same layout, values.
- * page_size is a power of two, 1 .. 65536 tokens. */
+ * page_size is a power of two, 1 .. 65536 tokens; a pool holds at most
+ * 2^31 - 1 rows (num_pages * Hkv * page_size; 512 GiB of bf16 keys at D = 128),
+ * else LOKI_ERR_UNSUPPORTED. */
 typedef struct {
   int32_t dtype;       /* loki_dtype                                          */
   int32_t n_kv_heads;  /* Hkv >= 1                                            */

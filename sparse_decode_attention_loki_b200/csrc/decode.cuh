@@ -88,6 +88,11 @@ struct Rows {
   }
   __device__ __forceinline__ const T *key(int t) const { return k + off(t); }
   __device__ __forceinline__ const T *val(int t) const { return v + off(t); }
+  // paged: the row of the pools that holds token t (off(t) / D)
+  __device__ __forceinline__ int phys(int t) const {
+    const int p = min(max(__ldg(table + (t >> shift)), 0), last_page);
+    return ((p * hkv + g) << shift) + (t & ((1 << shift) - 1));
+  }
   // the first dims of token t's key as the score stream reads them: the
   // low-rank plane's row when the call reads the plane, else the k_hat row
   __device__ __forceinline__ const T *skey(int t) const {
@@ -123,6 +128,22 @@ __device__ __forceinline__ Rows<T, D, PAGED> make_rows(const DecodeArgs<T> &a, i
     r.table = nullptr;
     r.shift = r.hkv = r.g = r.last_page = 0;
   }
+  return r;
+}
+
+// The page pools seen as one contiguous row array (row r at r * D): the
+// gather of a paged cache addresses physical rows (Rows::phys) through it.
+template <typename T, int D>
+__device__ __forceinline__ Rows<T, D, false> pool_rows(const DecodeArgs<T> &a) {
+  Rows<T, D, false> r;
+  r.k = a.k_hat;
+  r.v = a.v;
+  r.s = a.k_hat;
+  r.lr = nullptr;
+  r.sstride = D;
+  r.d_lr = 0;
+  r.table = nullptr;
+  r.shift = r.hkv = r.g = r.last_page = 0;
   return r;
 }
 

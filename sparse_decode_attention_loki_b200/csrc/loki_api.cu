@@ -639,8 +639,8 @@ loki_status check_paged(const loki_paged_cache *c, const loki_seq_table *q, loki
   if (q->max_seq_len < 1 || q->max_seq_len > cap)
     return fail(LOKI_ERR_INVALID_ARG, "max_seq_len %d outside [1, pages_per_seq * page_size = %lld]", q->max_seq_len,
                 cap);
-  if ((long long)c->num_pages * c->n_kv_heads * c->page_size > (1LL << 40))
-    return fail(LOKI_ERR_UNSUPPORTED, "page pool too large");
+  if ((long long)c->num_pages * c->n_kv_heads * c->page_size > (1LL << 31) - 1)
+    return fail(LOKI_ERR_UNSUPPORTED, "page pool of more than 2^31 - 1 rows (num_pages * n_kv_heads * page_size)");
   flat->dtype = c->dtype;
   flat->batch = q->batch;
   flat->n_kv_heads = c->n_kv_heads;

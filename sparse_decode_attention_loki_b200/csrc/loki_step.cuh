@@ -874,9 +874,21 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   // 3. attention over this CTA's even share of the k selected rows (the
   // share is at most chunk)
   __syncthreads();
-  attend_prologue_any<T, D, G, true>(rows, ids, 0, s1 - s0, ring);
-  attend_loop_any<T, D, G, true>(rows, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
-                                 pm, pl, pacc);
+  if constexpr (PAGED) {
+    // the share's token positions become rows of the page pools first (one
+    // page-table load each, all in flight at once), so that the gather loop
+    // computes no page addresses of its own
+    for (int i = tid; i < s1 - s0; i += kThreads) ids[i] = rows.phys(ids[i]);
+    __syncthreads();
+    const Rows<T, D, false> pool = pool_rows<T, D>(a.da);
+    attend_prologue_any<T, D, G, true>(pool, ids, 0, s1 - s0, ring);
+    attend_loop_any<T, D, G, true>(pool, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
+                                   pm, pl, pacc);
+  } else {
+    attend_prologue_any<T, D, G, true>(rows, ids, 0, s1 - s0, ring);
+    attend_loop_any<T, D, G, true>(rows, ids, 0, s1 - s0, qhat, reinterpret_cast<unsigned char *>(hist), ring,
+                                   pm, pl, pacc);
+  }
 
   // 4. log-sum-exp merge of the cluster's states
   if (gather && !leader) cluster_wait();

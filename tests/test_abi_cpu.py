@@ -211,6 +211,15 @@ def test_paged_workspace_size_and_cache_validation(lib):
         assert lib.loki_paged_decode_workspace_size(ctypes.byref(bc), ctypes.byref(q), 4, ctypes.byref(n)) == 1
     assert lib.loki_paged_decode_workspace_size(ctypes.byref(_paged(D=96)), ctypes.byref(q), 4,
                                                 ctypes.byref(n)) == 2
+    # a pool of 2^31 rows (num_pages * Hkv * page_size) is refused, one row less is not
+    big = _seqs(pps=1, max_len=50)
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(_paged(H=2, page=1 << 16, pages=1 << 14)),
+                                                ctypes.byref(big), 4, ctypes.byref(n)) == 2
+    assert b"2^31" in lib.loki_last_error()
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(_paged(H=1, page=1, pages=(1 << 31) - 1)),
+                                                ctypes.byref(big), 4, ctypes.byref(n)) == 1  # max_len > 1 token
+    assert lib.loki_paged_decode_workspace_size(ctypes.byref(_paged(H=1, page=64, pages=(1 << 25) - 1)),
+                                                ctypes.byref(big), 4, ctypes.byref(n)) == 0
     bad_seqs = [_seqs(B=0), _seqs(pps=0), _seqs(max_len=0), _seqs(max_len=65), _seqs(table=None),
                 _seqs(table=FAKE + 2), _seqs(lens=FAKE + 2)]
     for bq in bad_seqs:

@@ -474,6 +474,28 @@ def run_ours(args):
         for i in range(n):
             t_e2e += e2e_ev[i][0].elapsed_time(e2e_ev[i][1])
         done += n
+    # the same step through DecodeGraph (query in, decode, results out: one graph
+    # launch per step), one graph per query set
+    graphs = [L.DecodeGraph(cache, S, P, w.d, w.k, Hq) for _ in range(NSET)]
+    for j, gr in enumerate(graphs):
+        gr.q_host.copy_(q_host[j])
+    for i in range(args.warmup):
+        graphs[i % NSET].replay()
+    torch.cuda.synchronize()
+    t_e2g = 0.0
+    done = 0
+    while done < e2e_steps:
+        n = min(CH, e2e_steps - done)
+        for i in range(n):
+            flush.fill_(float(i & 7))
+            e2e_ev[i][0].record(stream)
+            graphs[(done + i) % NSET].replay()
+            e2e_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            t_e2g += e2e_ev[i][0].elapsed_time(e2e_ev[i][1])
+        done += n
+    del graphs
     # ---------------- the decode alone, back to back (no other kernel of ours between two
     # decodes), with and without the low-rank plane (same k_hat and v)
     cache_np = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, k_hat=cache.k_hat, v=cache.v)
@@ -569,10 +591,10 @@ def run_ours(args):
     d2h = out_host.numel() * 4 + idx_host.numel() * 4
 
     # ---------------- max over ranks
-    tt = torch.tensor([t_loki, t_dense, t_app, t_e2e], dtype=torch.float64, device=dev)
+    tt = torch.tensor([t_loki, t_dense, t_app, t_e2e, t_e2g], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    t_loki, t_dense, t_app, t_e2e = [float(x) for x in tt.tolist()]
+    t_loki, t_dense, t_app, t_e2e, t_e2g = [float(x) for x in tt.tolist()]
     rot, ncl, nct, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
     _, dcl, dct, _ = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
 
@@ -581,7 +603,8 @@ def run_ours(args):
         loki_us = t_loki * 1000.0 / K
         dense_us = t_dense * 1000.0 / K
         app_us = t_app * 1000.0 / K
-        e2e_us = t_e2e * 1000.0 / e2e_steps
+        e2e_us = t_e2g * 1000.0 / e2e_steps
+        e2e_eager_us = t_e2e * 1000.0 / e2e_steps
         peak, peak_kind = peaks()
         lb, db = w.loki_bytes(), w.dense_bytes()
         ach = lb / (loki_us * 1e-6) / 1e9
@@ -626,7 +649,11 @@ def run_ours(args):
                                                "rows": int(jaccard.numel())}},
             "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256},
             "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps,
+                    "path": "DecodeGraph.replay(): query copied in from pinned host memory, the decode, out "
+                            "and idx copied back, captured as one CUDA graph",
+                    "eager_value": e2e_eager_us / world,
+                    "eager_path": "the same copies and loki_decode_attention issued one by one from Python"},
             "gpu_launches": (2 if rot == 0 else 3) * K,  # timed loop: append, [rotate,] decode
             "clocks": clocks,
             "wall_s_timed_region": wall,

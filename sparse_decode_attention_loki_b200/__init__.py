@@ -9,6 +9,7 @@ C ABI of include/loki.h (libloki.so); this package is its Python binding.
 """
 from ._lib import LIB_PATH, LokiError, load as load_library
 from .api import (
+    DecodeGraph,
     LokiCache,
     PagedLokiCache,
     SeqTable,
@@ -33,6 +34,7 @@ from .api import (
 from .sharding import shard_batches
 
 __all__ = [
+    "DecodeGraph",
     "LIB_PATH",
     "LokiError",
     "load_library",

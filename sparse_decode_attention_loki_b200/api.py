@@ -455,3 +455,52 @@ def loki_status_string(status: int) -> str:
 
 def loki_version() -> int:
     return int(_lib.load().loki_version())
+
+
+class DecodeGraph:
+    """One Loki decode step from and to pinned host memory, captured once as a
+    CUDA graph and replayed: the copy of the query in (`q_host`), the decode
+    kernel(s) of loki_decode_attention, and the copies of the output and the
+    selected indices out (`out_host`, `idx_host`).  A replay launches the
+    whole step with one graph launch instead of four launches.
+
+    Fill `q_host` before `replay()`; read `out_host` / `idx_host` once the
+    stream has passed the replay (for example after torch.cuda.synchronize()).
+    The cache, seq_len, P, d and k are fixed at capture; the cache contents may
+    change between replays (an append before each step, say).  Capture happens
+    in the constructor, after one eager warm-up call (which sets the kernels'
+    attributes and allocates the workspace), so the constructor must not run
+    inside another capture."""
+
+    def __init__(self, cache: LokiCache, seq_len: int, P: torch.Tensor, d: int, k: int, n_q_heads: int,
+                 scale: float = 0.0):
+        dev = cache.device
+        self.cache, self.seq_len, self.P, self.d, self.k, self.scale = cache, int(seq_len), P, int(d), int(k), scale
+        shape = (cache.batch, int(n_q_heads), cache.head_dim)
+        self.q_host = torch.empty(shape, dtype=cache.dtype).pin_memory()
+        self.out_host = torch.empty(shape, dtype=torch.float32).pin_memory()
+        self.idx_host = torch.empty((cache.batch, cache.n_kv_heads, self.k), dtype=torch.int32).pin_memory()
+        self.q = torch.zeros(shape, dtype=cache.dtype, device=dev)
+        self.out = torch.empty(shape, dtype=torch.float32, device=dev)
+        self.idx = torch.empty((cache.batch, cache.n_kv_heads, self.k), dtype=torch.int32, device=dev)
+        self.workspace = cache.workspace(self.seq_len, int(n_q_heads))
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            self._step()  # warm-up: kernel attributes, first-call lookups
+        side.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=side):
+            self._step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+
+    def _step(self) -> None:
+        self.q.copy_(self.q_host, non_blocking=True)
+        loki_decode_attention(self.cache, self.seq_len, self.q, self.P, self.d, self.k, scale=self.scale,
+                              out=self.out, idx=self.idx, workspace=self.workspace)
+        self.out_host.copy_(self.out, non_blocking=True)
+        self.idx_host.copy_(self.idx, non_blocking=True)
+
+    def replay(self) -> None:
+        """Enqueue the step on the current stream."""
+        self.graph.replay()

@@ -278,13 +278,18 @@ def time_paged(L, w, cache, qs, P, flush, stream, dev, steps: int, warmup: int, 
     gen_t.manual_seed(7)
     perm = torch.randperm(B * pps, generator=gen_t).to(dev)
     table = perm.view(B, pps).to(torch.int32).contiguous()
-    pcache = L.PagedLokiCache(B * pps, Hkv, D, page, dtype=cache.dtype, device=dev)
+    pcache = L.PagedLokiCache(B * pps, Hkv, D, page, dtype=cache.dtype, device=dev,
+                              lowrank_dim=cache.d_lr or None)  # the same low-rank plane, paged
     pad = pps * page - S
-    for src, dst in ((cache.k_hat, pcache.k_hat), (cache.v, pcache.v)):
+    pairs = [(cache.k_hat, pcache.k_hat), (cache.v, pcache.v)]
+    if cache.k_lr is not None:
+        pairs.append((cache.k_lr, pcache.k_lr))
+    for src, dst in pairs:
+        W = src.shape[-1]
         x = src[:, :, :S]
         if pad:
-            x = torch.cat([x, torch.zeros((B, Hkv, pad, D), dtype=x.dtype, device=dev)], dim=2)
-        x = x.view(B, Hkv, pps, page, D).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv, page, D)
+            x = torch.cat([x, torch.zeros((B, Hkv, pad, W), dtype=x.dtype, device=dev)], dim=2)
+        x = x.view(B, Hkv, pps, page, W).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv, page, W)
         dst[perm.long()] = x
     seqs = L.SeqTable(table, None, S)
     out = torch.empty((B, w.n_q_heads, D), dtype=torch.float32, device=dev)
@@ -307,7 +312,8 @@ def time_paged(L, w, cache, qs, P, flush, stream, dev, steps: int, warmup: int, 
     us = tot / steps
     del pcache
     return {"us": us, "page_size": page, "pages": int(B * pps), "steps": steps,
-            "hbm_gbs": w.loki_bytes() / (us * 1e-6) / 1e9, "layout": "shuffled pages, every sequence at seq_len"}
+            "hbm_gbs": w.loki_bytes() / (us * 1e-6) / 1e9, "lowrank_plane": cache.d_lr,
+            "layout": "shuffled pages, every sequence at seq_len"}
 
 
 def run_ours(args):

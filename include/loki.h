@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 10
+#define LOKI_VERSION 11
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -252,6 +252,8 @@ LOKI_API loki_status loki_topk_jaccard(const int32_t *idx_a, const int32_t *idx_
  * A paged rotated-key cache: fixed-size pages from one pool.
  *   k_hat : [num_pages, Hkv, page_size, D] rotated keys in `dtype`, 16-byte
  *           aligned; v : the same layout, values.
+ *   k_lr, d_lr : optional low-rank key plane, as in loki_cache, in the pool
+ *           layout [num_pages, Hkv, page_size, d_lr] (same page ids), or NULL.
  * page_size is a power of two, 1 .. 65536 tokens; a pool holds at most
  * 2^31 - 1 rows (num_pages * Hkv * page_size; 512 GiB of bf16 keys at D = 128),
  * else LOKI_ERR_UNSUPPORTED. */
@@ -263,6 +265,8 @@ typedef struct {
   int32_t num_pages;   /* pages in each pool, >= 1                            */
   void *k_hat;
   void *v;
+  void *k_lr;          /* optional low-rank key plane pool, or NULL           */
+  int32_t d_lr;        /* its width (elements per token)                      */
 } loki_paged_cache;
 
 /* The sequences of a batch in a paged cache.

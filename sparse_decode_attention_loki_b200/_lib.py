@@ -42,6 +42,8 @@ class loki_paged_cache(ctypes.Structure):
         ("num_pages", ctypes.c_int32),
         ("k_hat", ctypes.c_void_p),
         ("v", ctypes.c_void_p),
+        ("k_lr", ctypes.c_void_p),
+        ("d_lr", ctypes.c_int32),
     ]
 
 

@@ -257,11 +257,13 @@ def topk_jaccard(idx_a: torch.Tensor, idx_b: torch.Tensor, stream: Optional[torc
 class PagedLokiCache:
     """A paged rotated-key cache: pools k_hat and v of shape
     [num_pages, Hkv, page_size, D] shared by the sequences of a batch through a
-    page table (see SeqTable)."""
+    page table (see SeqTable).  ``lowrank_dim`` (or ``k_lr``) adds a low-rank
+    key plane pool [num_pages, Hkv, page_size, d_lr], as in LokiCache."""
 
     def __init__(self, num_pages: int, n_kv_heads: int, head_dim: int, page_size: int,
                  dtype: torch.dtype = torch.bfloat16, device=None,
-                 k_hat: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None):
+                 k_hat: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None,
+                 lowrank_dim: Optional[int] = None, k_lr: Optional[torch.Tensor] = None):
         if dtype not in _DTYPES:
             raise ValueError(f"cache dtype must be float32 or bfloat16, got {dtype}")
         device = torch.device(device if device is not None else "cuda")
@@ -277,8 +279,18 @@ class PagedLokiCache:
         self.num_pages, self.n_kv_heads, self.head_dim, self.page_size = num_pages, n_kv_heads, head_dim, page_size
         self.dtype = dtype
         self.device = device
+        if k_lr is not None:
+            lowrank_dim = k_lr.shape[-1] if k_lr.dim() == 4 else -1
+        self.d_lr = int(lowrank_dim) if lowrank_dim else 0
+        if self.d_lr:
+            lshape = (num_pages, n_kv_heads, page_size, self.d_lr)
+            self.k_lr = k_lr if k_lr is not None else torch.empty(lshape, dtype=dtype, device=device)
+            _need(self.k_lr, "k_lr", dtype, lshape, device)
+        else:
+            self.k_lr = None
         self._desc = _lib.loki_paged_cache(_DTYPES[dtype], n_kv_heads, head_dim, page_size, num_pages,
-                                           self.k_hat.data_ptr(), self.v.data_ptr())
+                                           self.k_hat.data_ptr(), self.v.data_ptr(),
+                                           self.k_lr.data_ptr() if self.k_lr is not None else None, self.d_lr)
 
     def desc(self):
         return ctypes.byref(self._desc)

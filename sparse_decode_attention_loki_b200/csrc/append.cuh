@@ -24,8 +24,8 @@ struct AppendArgs {
   const T *k_new;    // [B, Hkv, n_new, D]
   const T *v_new;    // [B, Hkv, n_new, D]
   const float *P;    // [Hkv, D, D]
-  // the cache's low-rank key plane [B, Hkv, S_cap, d_lr] (contiguous caches;
-  // null: none): it receives the first d_lr dims of every appended key
+  // the cache's low-rank key plane (null: none), laid out like k_hat with
+  // rows of d_lr: it receives the first d_lr dims of every appended key
   T *k_lr;
   int32_t d_lr;
   int32_t n_kv_heads;
@@ -59,11 +59,11 @@ __device__ __forceinline__ long long append_dst(const AppendArgs<T> &a, int b, i
   }
 }
 
-// Element offset in the low-rank plane of new vector t of sequence b, head g
-// (contiguous caches).
-template <typename T>
-__device__ __forceinline__ long long append_lr_dst(const AppendArgs<T> &a, int b, int g, int t) {
-  return (((long long)b * a.n_kv_heads + g) * a.capacity + a.pos + t) * a.d_lr;
+// Element offset in the low-rank plane of the row whose k_hat offset is off
+// (>= 0): the same row index, rows of d_lr.
+template <typename T, int D>
+__device__ __forceinline__ long long append_lr_dst(const AppendArgs<T> &a, long long off) {
+  return off / D * a.d_lr;
 }
 
 constexpr int kAppendBatch = kWarps;   // vectors per batch: one per warp
@@ -117,8 +117,10 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
     if (f < f_end) {
       const int b = f / a.n_new, t = f % a.n_new;
       const long long off = append_dst<T, D, PAGED>(a, b, g, t);
-      if (off >= 0) from_f32(acc, a.k_hat + off + j);
-      if (!PAGED && a.k_lr != nullptr && j < a.d_lr) from_f32(acc, a.k_lr + append_lr_dst(a, b, g, t) + j);
+      if (off >= 0) {
+        from_f32(acc, a.k_hat + off + j);
+        if (a.k_lr != nullptr && j < a.d_lr) from_f32(acc, a.k_lr + append_lr_dst<T, D>(a, off) + j);
+      }
     }
   }
 

@@ -271,10 +271,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) append_tc_kernel(const __grid_c
         tile_row(a.n_new, b0, t0, r, b, t);
         const long long off = dst_off(g, b, t);
         const uint4 w = *reinterpret_cast<const uint4 *>(stg + r * (D * 2) + ((cch ^ (r & (CH - 1))) * 16));
-        if (off >= 0) reinterpret_cast<uint4 *>(a.k_hat + off)[cch] = w;
-        // the low-rank plane (d_lr a multiple of 8: whole 16-byte chunks)
-        if (!PAGED && a.k_lr != nullptr && cch * 8 < a.d_lr)
-          reinterpret_cast<uint4 *>(a.k_lr + append_lr_dst(a, b, g, t))[cch] = w;
+        if (off >= 0) {
+          reinterpret_cast<uint4 *>(a.k_hat + off)[cch] = w;
+          // the low-rank plane (d_lr a multiple of 8: whole 16-byte chunks)
+          if (a.k_lr != nullptr && cch * 8 < a.d_lr)
+            reinterpret_cast<uint4 *>(a.k_lr + append_lr_dst<__nv_bfloat16, D>(a, off))[cch] = w;
+        }
       }
     }
     __syncthreads();  // the stage is read before it is refilled

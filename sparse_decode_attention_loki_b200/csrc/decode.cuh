@@ -57,8 +57,9 @@ struct DecodeArgs {
   // row's last attended position (null: no append)
   const T *k_new;           // [B, Hkv, D], not rotated
   const T *v_new;           // [B, Hkv, D]
-  // the cache's low-rank key plane [B, Hkv, S_cap, d_lr] (null: none;
-  // contiguous caches only), a copy of k_hat[..., :d_lr].  Written with every
+  // the cache's low-rank key plane (null: none), a copy of k_hat[..., :d_lr]
+  // in the layout of k_hat with rows of d_lr: [B, Hkv, S_cap, d_lr], or
+  // [num_pages, Hkv, page_size, d_lr] for paged pools.  Written with every
   // appended key; the score stream reads it when lr_read (d <= d_lr).
   const T *k_lr;
   int32_t d_lr;
@@ -72,9 +73,9 @@ struct DecodeArgs {
 template <typename T, int D, bool PAGED>
 struct Rows {
   const T *k, *v;        // contiguous: the row's token 0; paged: the pools
-  const T *s;            // contiguous: token 0 of the rows the score stream reads
-  T *lr;                 // contiguous: token 0 of the row's low-rank plane, or null
-  int32_t sstride;       // elements between the score rows of two tokens
+  const T *s;            // the same for the rows the score stream reads (k or the plane)
+  T *lr;                 // the same for the low-rank plane, or null
+  int32_t sstride;       // elements per score row (D, or d_lr for the plane)
   int32_t d_lr;          // width of the low-rank plane
   const int32_t *table;  // paged: this sequence's page ids
   int32_t shift, hkv, g, last_page;
@@ -93,12 +94,15 @@ struct Rows {
     const int p = min(max(__ldg(table + (t >> shift)), 0), last_page);
     return ((p * hkv + g) << shift) + (t & ((1 << shift) - 1));
   }
+  // token t's row index from the bases k, v, s and lr: t (contiguous) or
+  // its pool row (paged)
+  __device__ __forceinline__ int row_of(int t) const {
+    if constexpr (!PAGED) return t;
+    else return phys(t);
+  }
   // the first dims of token t's key as the score stream reads them: the
   // low-rank plane's row when the call reads the plane, else the k_hat row
-  __device__ __forceinline__ const T *skey(int t) const {
-    if constexpr (!PAGED) return s + (size_t)t * sstride;
-    else return key(t);
-  }
+  __device__ __forceinline__ const T *skey(int t) const { return s + (size_t)row_of(t) * sstride; }
 };
 
 template <typename T, int D, bool PAGED>
@@ -112,10 +116,10 @@ __device__ __forceinline__ Rows<T, D, PAGED> make_rows(const DecodeArgs<T> &a, i
     r.hkv = a.n_kv_heads;
     r.g = g;
     r.last_page = a.num_pages - 1;
-    r.s = nullptr;
-    r.lr = nullptr;
-    r.sstride = D;
-    r.d_lr = 0;
+    r.lr = const_cast<T *>(a.k_lr);
+    r.d_lr = a.k_lr ? a.d_lr : 0;
+    r.s = a.lr_read ? r.lr : r.k;
+    r.sstride = a.lr_read ? a.d_lr : D;
   } else {
     const size_t row = (size_t)b * a.n_kv_heads + g;
     const size_t off = row * a.capacity * D;
@@ -298,7 +302,7 @@ __device__ __forceinline__ void store_appended(const DecodeArgs<T> &a, const Row
                                                int t, float *xk_hat) {
   T *kd = const_cast<T *>(rows.key(t));
   T *vd = const_cast<T *>(rows.val(t));
-  T *ld = rows.lr ? rows.lr + (size_t)t * rows.d_lr : nullptr;
+  T *ld = rows.lr ? rows.lr + (size_t)rows.row_of(t) * rows.d_lr : nullptr;
   const T *vs = a.v_new + ((size_t)b * a.n_kv_heads + g) * D;
   for (int i = threadIdx.x; i < D; i += kThreads) {
     T r;

@@ -648,8 +648,8 @@ loki_status check_paged(const loki_paged_cache *c, const loki_seq_table *q, loki
   flat->capacity = (int32_t)cap;
   flat->k_hat = c->k_hat;
   flat->v = c->v;
-  flat->k_lr = nullptr;  // paged pools have no low-rank plane
-  flat->d_lr = 0;
+  flat->k_lr = c->k_lr;
+  flat->d_lr = c->d_lr;
   loki_status s = check_cache(flat, sh);
   if (s != LOKI_OK) return s;
   int sft = 0;
@@ -940,6 +940,10 @@ loki_status loki_paged_append(const loki_paged_cache *cache, const loki_seq_tabl
     a.n_new = n_new;
     a.n_vec = sh.B * n_new;
     a.pos_arr = pos;
+    if (cache->k_lr) {
+      a.k_lr = static_cast<T *>(cache->k_lr);
+      a.d_lr = cache->d_lr;
+    }
     a.table = seqs->block_table;
     a.pages_per_seq = seqs->pages_per_seq;
     a.page_shift = shift;

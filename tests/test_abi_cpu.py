@@ -53,7 +53,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 10
+    assert lib.loki_version() == 11
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -190,9 +190,9 @@ def test_append_pointer_validation(lib):
     assert lib.loki_append(None, 0, 1, FAKE, FAKE, FAKE, None) == 1
 
 
-def _paged(dtype=1, H=2, D=128, page=16, pages=10, k=4096, v=8192):
+def _paged(dtype=1, H=2, D=128, page=16, pages=10, k=4096, v=8192, k_lr=None, d_lr=0):
     from sparse_decode_attention_loki_b200 import _lib
-    return _lib.loki_paged_cache(dtype, H, D, page, pages, k, v)
+    return _lib.loki_paged_cache(dtype, H, D, page, pages, k, v, k_lr, d_lr)
 
 
 def _seqs(B=2, pps=4, max_len=50, table=FAKE, lens=FAKE):
@@ -321,3 +321,15 @@ def test_lowrank_plane_validation(lib, dtype, D, k_lr, d_lr, status):
     assert lib.loki_decode_attention(*args) == 1
     if status:
         assert b"plane" in lib.loki_last_error()
+
+
+def test_paged_lowrank_plane_validation(lib):
+    from sparse_decode_attention_loki_b200 import _lib
+    assert ctypes.sizeof(_lib.loki_paged_cache) == 56
+    n = ctypes.c_size_t(0)
+    q = _seqs()
+    for k_lr, d_lr, status in [(FAKE, 32, 0), (FAKE, 12, 1), (FAKE, 136, 1), (FAKE + 8, 32, 1), (None, 12, 0)]:
+        c = _paged(k_lr=k_lr, d_lr=d_lr)
+        assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 4, ctypes.byref(n)) == status
+        if status:
+            assert b"plane" in lib.loki_last_error()

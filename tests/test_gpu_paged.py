@@ -229,3 +229,64 @@ def test_append_past_the_page_table_is_dropped():
             if changed[pg, sl]:
                 assert (pg, sl) in owned, (pg, sl)
     assert len(owned) == int(changed.sum())
+
+
+# ----------------------------------------------------------------------------- low-rank key plane pools
+def _plane_twin(su, d_lr):
+    """A paged cache on the same pools with a low-rank plane pool (filled with
+    GARBAGE, then kept by the appends)."""
+    c = su.L.PagedLokiCache(su.num_pages, su.Hkv, su.D, su.page, dtype=TD[su.dtype], device=su.dev,
+                            k_hat=su.cache.k_hat, v=su.cache.v, lowrank_dim=d_lr)
+    c.k_lr.fill_(GARBAGE)
+    return c
+
+
+@pytest.mark.parametrize("dtype,D,G,page,lens,d,d_lr", [
+    ("bf16", 128, 1, 16, [700, 333, 1024], 32, 32),     # CUDA-core append
+    ("bf16", 128, 4, 64, [300, 2000], 32, 64),          # tensor-core append (B * n_new >= 256), d < d_lr
+    ("f32", 64, 2, 32, [500, 129, 77], 16, 16),
+])
+def test_paged_plane_is_kept_and_read(dtype, D, G, page, lens, d, d_lr):
+    su = Setup(dtype, D, G, page, lens, seed=17 + G)
+    c = _plane_twin(su, d_lr)
+    pos = torch.zeros(su.B, dtype=torch.int32, device=su.dev)
+    su.L.loki_paged_append(c, su.seqs(), pos, su.k_new, su.v_new, su.P_dev)  # tokens [0, S_max) of every row
+    torch.cuda.synchronize()
+    # every written slot holds the first d_lr dims of its key; the rest is untouched
+    wr = torch.as_tensor(su.own_slot_mask([su.S_max] * su.B)).to(su.dev)
+    Kl = torch.as_tensor(su.logical(c.k_hat)).to(su.dev).permute(0, 2, 1, 3)[..., :d_lr]
+    Ll = torch.as_tensor(su.logical(torch.nn.functional.pad(c.k_lr, (0, D - d_lr)))).to(su.dev)
+    Ll = Ll.permute(0, 2, 1, 3)[..., :d_lr]
+    assert torch.equal(Ll[wr], Kl[wr])
+    assert bool((Ll[~wr] == GARBAGE).all())
+    k = max(1, min(lens) // 4)
+    o0, i0 = su.L.loki_paged_decode_attention(su.cache, su.seqs(), su.q, su.P_dev, d, k)
+    o1, i1 = su.L.loki_paged_decode_attention(c, su.seqs(), su.q, su.P_dev, d, k)
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1) and torch.equal(o0, o1)
+
+
+def test_paged_fused_append_keeps_the_plane():
+    # two identical setups (same seed): one read and kept through a plane, one without
+    runs = []
+    for plane in (False, True):
+        su = Setup("bf16", 128, 4, 16, [900, 401], seed=23)
+        c = _plane_twin(su, 32) if plane else su.cache
+        pos = torch.zeros(su.B, dtype=torch.int32, device=su.dev)
+        su.L.loki_paged_append(c, su.seqs(), pos, su.k_new, su.v_new, su.P_dev)
+        lens1 = torch.as_tensor(np.array(su.lens, dtype=np.int32) + 1).to(su.dev)
+        seqs1 = su.L.SeqTable(su.table, lens1, su.S_max + 1)
+        kn = torch.as_tensor(su.rng.standard_normal((su.B, su.Hkv, 128)), dtype=torch.float32).to(
+            torch.bfloat16).to(su.dev)
+        vn = torch.as_tensor(su.rng.standard_normal((su.B, su.Hkv, 128)), dtype=torch.float32).to(
+            torch.bfloat16).to(su.dev)
+        out, idx = su.L.loki_paged_decode_attention_append(c, seqs1, kn, vn, su.q, su.P_dev, 32, 100)
+        torch.cuda.synchronize()
+        if plane:
+            wr = torch.as_tensor(su.own_slot_mask([S + 1 for S in su.lens])).to(su.dev)
+            Kl = torch.as_tensor(su.logical(c.k_hat)).to(su.dev).permute(0, 2, 1, 3)[..., :32]
+            Ll = torch.as_tensor(su.logical(torch.nn.functional.pad(c.k_lr, (0, 96)))).to(su.dev)
+            assert torch.equal(Ll.permute(0, 2, 1, 3)[..., :32][wr], Kl[wr])
+        runs.append((out, idx, c.k_hat.clone()))
+    assert torch.equal(runs[0][2], runs[1][2])
+    assert torch.equal(runs[0][1], runs[1][1]) and torch.equal(runs[0][0], runs[1][0])

@@ -479,7 +479,9 @@ class DecodeGraph:
     Fill `q_host` before `replay()`; read `out_host` / `idx_host` once the
     stream has passed the replay (for example after torch.cuda.synchronize()).
     The cache, seq_len, P, d and k are fixed at capture; the cache contents may
-    change between replays (an append before each step, say).  Capture happens
+    change between replays (an append before each step, say).  `out` and `idx`
+    sit back to back in one device buffer, so that one copy brings both back
+    (`out_host` and `idx_host` are views of one pinned buffer).  Capture happens
     in the constructor, after one eager warm-up call (which sets the kernels'
     attributes and allocates the workspace), so the constructor must not run
     inside another capture."""
@@ -489,12 +491,16 @@ class DecodeGraph:
         dev = cache.device
         self.cache, self.seq_len, self.P, self.d, self.k, self.scale = cache, int(seq_len), P, int(d), int(k), scale
         shape = (cache.batch, int(n_q_heads), cache.head_dim)
+        ishape = (cache.batch, cache.n_kv_heads, self.k)
+        n_out, n_idx = shape[0] * shape[1] * shape[2], ishape[0] * ishape[1] * ishape[2]
         self.q_host = torch.empty(shape, dtype=cache.dtype).pin_memory()
-        self.out_host = torch.empty(shape, dtype=torch.float32).pin_memory()
-        self.idx_host = torch.empty((cache.batch, cache.n_kv_heads, self.k), dtype=torch.int32).pin_memory()
+        self.res_host = torch.empty(n_out + n_idx, dtype=torch.float32).pin_memory()
+        self.out_host = self.res_host[:n_out].view(shape)
+        self.idx_host = self.res_host[n_out:].view(torch.int32).view(ishape)
         self.q = torch.zeros(shape, dtype=cache.dtype, device=dev)
-        self.out = torch.empty(shape, dtype=torch.float32, device=dev)
-        self.idx = torch.empty((cache.batch, cache.n_kv_heads, self.k), dtype=torch.int32, device=dev)
+        self.res = torch.empty(n_out + n_idx, dtype=torch.float32, device=dev)
+        self.out = self.res[:n_out].view(shape)
+        self.idx = self.res[n_out:].view(torch.int32).view(ishape)
         self.workspace = cache.workspace(self.seq_len, int(n_q_heads))
         side = torch.cuda.Stream(dev)
         side.wait_stream(torch.cuda.current_stream(dev))
@@ -510,8 +516,7 @@ class DecodeGraph:
         self.q.copy_(self.q_host, non_blocking=True)
         loki_decode_attention(self.cache, self.seq_len, self.q, self.P, self.d, self.k, scale=self.scale,
                               out=self.out, idx=self.idx, workspace=self.workspace)
-        self.out_host.copy_(self.out, non_blocking=True)
-        self.idx_host.copy_(self.idx, non_blocking=True)
+        self.res_host.copy_(self.res, non_blocking=True)
 
     def replay(self) -> None:
         """Enqueue the step on the current stream."""

@@ -366,10 +366,12 @@ def test_invalid_arguments_raise_without_launch():
 
 
 # ----------------------------------------------------------------------------- full-size workloads
-def fill_cache_on_device(w, P_dev, S, capacity, seed=123):
-    """Whole cache through the GPU append kernel from device-drawn keys."""
+def fill_cache_on_device(w, P_dev, S, capacity, seed=123, d_lr=0):
+    """Whole cache through the GPU append kernel from device-drawn keys (with
+    a low-rank key plane d_lr wide when d_lr > 0)."""
     td = TORCH_DTYPE[w.dtype]
-    cache = L().LokiCache(w.batch, w.n_kv_heads, w.head_dim, capacity, dtype=td, device=DEV)
+    cache = L().LokiCache(w.batch, w.n_kv_heads, w.head_dim, capacity, dtype=td, device=DEV,
+                          lowrank_dim=d_lr or None)
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
     k_new = torch.empty((w.batch, w.n_kv_heads, S, w.head_dim), dtype=td, device=DEV)
@@ -382,12 +384,17 @@ def fill_cache_on_device(w, P_dev, S, capacity, seed=123):
 
 
 def full_size_check(w, S=None, n_rows=3, seed=0):
+    """The launch configuration bench.py times: a cache with a low-rank key
+    plane as wide as d (rounded up to 16 bytes) when that is narrower than D."""
     S = S or w.seq_len
     k = w.k if S == w.seq_len else max(1, min(S, int(np.floor(w.k_f * S + 1e-9))))
     d = w.d
+    per = 8 if w.dtype == "bf16" else 4
+    d_lr = (d + per - 1) // per * per
+    d_lr = d_lr if d_lr < w.head_dim else 0
     P32 = basis(w)
     P_dev = torch.from_numpy(P32).to(DEV)
-    cache = fill_cache_on_device(w, P_dev, S, S)
+    cache = fill_cache_on_device(w, P_dev, S, S, d_lr=d_lr)
     rng = np.random.default_rng(seed)
     rows = sorted({(int(rng.integers(0, w.batch)), int(rng.integers(0, w.n_kv_heads))) for _ in range(n_rows)})
     G = w.group
@@ -401,6 +408,8 @@ def full_size_check(w, S=None, n_rows=3, seed=0):
         cache.k_hat[b, g, :S] = torch.from_numpy(K_hat[0, 0]).to(td).to(DEV)
         cache.v[b, g, :S] = vt.to(DEV)
         host[(b, g)] = (K_hat, v64[None, None])
+    if d_lr:
+        cache.k_lr.copy_(cache.k_hat[..., :d_lr])  # the plane follows the rows written above
     Q = np.stack([gen.queries(w, b) for b in range(w.batch)])
     qt, q64 = gen.to_cache_dtype(Q, w.dtype)
     out, idx = L().loki_decode_attention(cache, S, qt.to(DEV), P_dev, d, k)

@@ -67,8 +67,8 @@ typedef enum { LOKI_F32 = 0, LOKI_BF16 = 1 } loki_dtype;
  *   k_lr  : optional low-rank key plane, [B, Hkv, S_cap, d_lr] in `dtype`,
  *           16-byte aligned, or NULL.  It holds a copy of the first d_lr
  *           dimensions of every key row, k_lr[b][g][t][j] = k_hat[b][g][t][j]
- *           for j < d_lr, kept by every call that writes keys (loki_append and
- *           the *_append decode calls).  A Loki decode with d <= d_lr streams
+ *           for j < d_lr, kept by every call that writes keys (loki_append,
+ *           loki_paged_append and the *_append decode calls).  A Loki decode with d <= d_lr streams
  *           the low-rank scores from it instead of from k_hat: HBM serves
  *           reads in whole 128-byte lines, so reading d < 64 bf16 dimensions
  *           of each 256-byte k_hat row costs a full line per token, while the

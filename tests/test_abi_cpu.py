@@ -333,3 +333,23 @@ def test_paged_lowrank_plane_validation(lib):
         assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 4, ctypes.byref(n)) == status
         if status:
             assert b"plane" in lib.loki_last_error()
+
+
+def test_the_abi_is_plain_c(lib):
+    # include/loki.h compiles as C99 (pedantic, warnings as errors) and a C
+    # program links libloki.so and gets its validation answers (no GPU needed)
+    import shutil
+    from sparse_decode_attention_loki_b200 import _lib
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "tests", "c_abi", "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "abi_check")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c_abi", "abi_check.c"), "-L", libdir, "-lloki",
+                        "-Wl,-rpath," + libdir, "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr

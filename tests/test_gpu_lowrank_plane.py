@@ -73,6 +73,9 @@ def _twin_caches(w, inp, P32, d_lr):
     ("bf16", 64, 2, 777, 8, 16, 0.5, 2),           # D = 64, ragged
     ("f32", 128, 1, 1000, 32, 32, 0.25, None),
     ("bf16", 128, 4, 2048, 96, 64, 0.25, None),    # d > d_lr: the plane is not read
+    ("f32", 128, 2, 20000, 32, 32, 0.25, 4),       # fp32 plane, candidate path
+    ("bf16", 128, 2, 9000, 40, 40, 0.125, None),   # an 80-byte plane row (not a power of two)
+    ("bf16", 128, 4, 30000, 64, 64, 0.5, 2),       # k_f 0.5: the select lists overflow
 ])
 def test_decode_with_plane_is_bit_identical(dtype, D, G, S, d, d_lr, kf, ncta):
     w = small_workload(dtype, D, G, S, Hkv=2, B=2, seed=91)

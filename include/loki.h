@@ -314,7 +314,9 @@ LOKI_API loki_status loki_paged_decode_workspace_size(const loki_paged_cache *ca
  *   idx   : [B, Hkv, k_max] int32 (written): row (b, g) holds the k_b
  *           selected positions in ascending order, then -1 up to k_max.
  * Everything else as loki_decode_attention (out [B, Hq, D] fp32, workspace of
- * loki_paged_decode_workspace_size bytes, two kernels on `stream`). */
+ * loki_paged_decode_workspace_size bytes, one kernel on `stream`, two for
+ * query groups of 8; the scores read the pool's low-rank plane when it has one
+ * at least d wide). */
 LOKI_API loki_status loki_paged_decode_attention(const loki_paged_cache *cache,
                                         const loki_seq_table *seqs, int32_t n_q_heads,
                                         const void *q, const float *P, int32_t d,

@@ -4,9 +4,15 @@
 
 One timed step = one Loki decode layer-step (rotate q, low-rank scores, top-k,
 gather attention, combine) through the C ABI on a cache already resident in
-HBM: one kernel for query groups of up to 4 heads, a rotate + decode pair for
-groups of 8.  Each step also appends the step's new token first (timed separately).
-The in-library dense decode on the same cache is timed over K steps of its own.
+HBM, by default on the largest single-GPU decode workload
+(llama3-8b-gqa-decode: B 8, 32 query / 8 KV heads, S 32768, d_f 0.5,
+k_f 0.125).  Each step also appends the step's new token first (timed
+separately).  The in-library dense decode on the same cache is timed over K
+steps of its own.  The same run also times a short-row decode
+(llama2-7b-decode) and the pages' generation run (llama2-13b-generation:
+prompt 3072, then 512 steps that append their token inside the call), Loki
+against dense, and the fp64 oracle on the host (one thread and the BLAS
+pool) with its dense attention beside it.
 L2 is flushed before every step by writing a buffer twice the L2 size; the flush
 is outside the timed events.  Device time from CUDA events on the launching
 stream, summed over the K steps, max over ranks.
@@ -35,7 +41,11 @@ from workloads import generators as gen  # noqa: E402
 
 METRIC = "Loki decode attention µs/layer-step and achieved HBM GB/s vs peak, vs dense"
 UNIT = "us/layer-step"
-DEFAULT_WORKLOAD = "llama2-7b-decode"
+DEFAULT_WORKLOAD = "llama3-8b-gqa-decode"
+# timed in the same run beside the main workload: a short-row decode, and the
+# generation run the pages quote their speed-up on
+EXTRA_DECODE = "llama2-7b-decode"
+GENERATION = "llama2-13b-generation"
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -114,36 +124,78 @@ def workload_config(w, n_gpus):
 
 
 # ------------------------------------------------------------------------------------ oracle arm
-def oracle_sample_us(w, budget_s: float, seed: int = 0):
-    """Time the fp64 oracle decode on whole (batch, KV head) rows of the
-    workload, one row at a time, until budget_s of CPU time is spent; scale the
-    mean row time to one layer-step (all B*Hkv rows).  Returns (us per
-    layer-step, rows timed, threads)."""
+_ROW_CACHE = {}
+
+
+def _oracle_rows(w, seed, distinct: int = 16):
+    """Seeded (batch, KV head) rows of the workload with their oracle inputs,
+    widened to fp64: (q64 [1, G, D], K_hat [1, 1, S, D], V [1, 1, S, D],
+    P [1, D, D]).  Up to `distinct` rows are drawn (and kept for later calls),
+    then they repeat."""
     import oracle
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
-    P32 = np.stack([oracle.pca_basis(gen.calibration_keys(w, g))[0]
-                    for g in range(w.n_kv_heads)]).astype(np.float32).astype(np.float64)
-    rng = np.random.default_rng(seed)
+    key = (w.name, seed)
+    if key not in _ROW_CACHE:
+        P32 = np.stack([oracle.pca_basis(gen.calibration_keys(w, g))[0]
+                        for g in range(w.n_kv_heads)]).astype(np.float32).astype(np.float64)
+        _ROW_CACHE[key] = (P32, np.random.default_rng(seed), [])
+    P32, rng, rows = _ROW_CACHE[key]
     G = w.group
-    times = []
-    t_start = time.perf_counter()
+    i = 0
     while True:
-        b, g = int(rng.integers(0, w.batch)), int(rng.integers(0, w.n_kv_heads))
-        _, k64 = gen.to_cache_dtype(gen.row_keys(w, b, g, w.seq_len), w.dtype)
-        _, v64 = gen.to_cache_dtype(gen.row_values(w, b, g, w.seq_len), w.dtype)
-        _, q64 = gen.to_cache_dtype(gen.queries(w, b)[g * G:(g + 1) * G][None], w.dtype)
-        K_hat = oracle.rotate_keys(k64[None, None], P32[g:g + 1], w.dtype)
-        t0 = time.perf_counter()
-        oracle.loki_decode(q64, K_hat, v64[None, None], P32[g:g + 1], w.seq_len, w.d, w.k)
-        times.append(time.perf_counter() - t0)
-        if sum(times) >= budget_s or time.perf_counter() - t_start > 3 * budget_s or len(times) >= 4096:
-            break
+        if i >= len(rows) and len(rows) < distinct:
+            b, g = int(rng.integers(0, w.batch)), int(rng.integers(0, w.n_kv_heads))
+            _, k64 = gen.to_cache_dtype(gen.row_keys(w, b, g, w.seq_len), w.dtype)
+            _, v64 = gen.to_cache_dtype(gen.row_values(w, b, g, w.seq_len), w.dtype)
+            _, q64 = gen.to_cache_dtype(gen.queries(w, b)[g * G:(g + 1) * G][None], w.dtype)
+            K_hat = oracle.rotate_keys(k64[None, None], P32[g:g + 1], w.dtype)
+            rows.append((q64, K_hat, v64[None, None], P32[g:g + 1]))
+        yield rows[i % len(rows)]
+        i += 1
+
+
+def oracle_sample_us(w, budget_s: float, seed: int = 0, threads=None, dense: bool = False):
+    """Time the fp64 oracle (the Loki decode, or with dense=True its dense
+    attention) on whole (batch, KV head) rows of the workload, one row at a
+    time, until budget_s of wall time is spent; scale the mean row time to one
+    layer-step (all B*Hkv rows).  threads: the BLAS thread limit (None: the
+    library's default pool).  Returns (us per layer-step, rows timed, thread
+    limit, effective cores = process CPU time / wall time over the timed calls)."""
+    import oracle
+    from threadpoolctl import threadpool_info, threadpool_limits
+    times, cpu = [], []
+    t_start = time.perf_counter()
+    with threadpool_limits(limits=threads):
+        limit = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        for q64, K_hat, v64, P in _oracle_rows(w, seed):
+            c0, t0 = time.process_time(), time.perf_counter()
+            if dense:
+                oracle.dense_decode(q64, K_hat, v64, P, w.seq_len)
+            else:
+                oracle.loki_decode(q64, K_hat, v64, P, w.seq_len, w.d, w.k)
+            times.append(time.perf_counter() - t0)
+            cpu.append(time.process_time() - c0)
+            if sum(times) >= budget_s or time.perf_counter() - t_start > 3 * budget_s or len(times) >= 4096:
+                break
     per_row = float(np.mean(times))
-    return per_row * w.rows * 1e6, len(times), threads
+    return per_row * w.rows * 1e6, len(times), limit, float(sum(cpu) / max(sum(times), 1e-12))
+
+
+def cpu_baseline(w, budget_s: float):
+    """The oracle's Loki decode with the default BLAS pool and with one
+    thread, and its dense attention beside it (default pool), each on a
+    bounded sample of rows."""
+    us, rows, limit, eff = oracle_sample_us(w, budget_s)
+    us1, rows1, _, eff1 = oracle_sample_us(w, budget_s / 2, threads=1)
+    dus, drows, dlimit, deff = oracle_sample_us(w, budget_s / 2, dense=True)
+    host = len(os.sched_getaffinity(0))
+    return {"value": us, "unit": UNIT, "cores": limit, "kind": "oracle",
+            "sample": f"{rows} calls on whole (batch, KV head) rows (up to 16 distinct rows, repeated), fp64 numpy "
+                      f"oracle, scaled to all {w.rows} rows of one layer-step; BLAS pool of {limit} threads, "
+                      f"{eff:.2f} cores busy on average",
+            "effective_cores": eff, "host_cores": host,
+            "single_thread": {"value": us1, "unit": UNIT, "cores": 1, "rows": rows1, "effective_cores": eff1},
+            "dense_fp64": {"value": dus, "unit": UNIT, "cores": dlimit, "rows": drows, "effective_cores": deff,
+                           "what": "the oracle's dense attention over all S tokens of each row"}}
 
 
 def run_reference(args):
@@ -157,9 +209,11 @@ def run_reference(args):
     per_step = []
     rows = 0
     threads = 1
+    effs = []
     for s in range(args.steps):
-        us, n, threads = oracle_sample_us(w, budget_s=budget / max(1, args.steps), seed=100 + s)
+        us, n, threads, eff = oracle_sample_us(w, budget_s=budget / max(1, args.steps), seed=100 + s)
         per_step.append(us)
+        effs.append(eff)
         rows += n
     value = float(np.mean(per_step))
     line = {
@@ -169,7 +223,9 @@ def run_reference(args):
         "data": "synthetic", "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{rows} whole (batch, KV head) rows of the workload, fp64 numpy oracle, "
-                                   f"scaled to all {w.rows} rows"},
+                                   f"scaled to all {w.rows} rows; BLAS pool of {threads} threads, "
+                                   f"{float(np.mean(effs)):.2f} cores busy on average",
+                         "effective_cores": float(np.mean(effs))},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -247,14 +303,17 @@ def time_prefill(L, cache, k_pre, v_pre, P, stream, dev, reps: int = 5):
                                              and k_pre.shape[0] * k_pre.shape[2] >= 256) else "append_kernel"}
 
 
-def time_pca(L, calib, dev, stream, reps: int = 3):
-    """Device time of the GPU calibration (loki_pca_calibrate) of every KV
-    head's basis from its calibration keys; median over reps."""
+def calibrate(L, calib, dev, stream, reps: int = 3):
+    """P of every KV head from its calibration keys on the GPU
+    (loki_pca_calibrate), and the device time of that calibration (median over
+    reps)."""
     import torch
     keys = torch.as_tensor(np.stack(calib).astype(np.float32)).to(dev)
     H, N, D = keys.shape
     ws = torch.empty(L.loki_pca_workspace_size(H, D), dtype=torch.uint8, device=dev)
-    L.loki_pca_calibrate(keys, workspace=ws)
+    P, _ = L.loki_pca_calibrate(keys, workspace=ws)
+    if reps < 1:
+        return P, None
     ts = []
     for _ in range(reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -263,8 +322,167 @@ def time_pca(L, calib, dev, stream, reps: int = 3):
         e1.record(stream)
         e1.synchronize()
         ts.append(e0.elapsed_time(e1) * 1000.0)
-    return {"us": float(np.median(ts)), "heads": int(H), "keys_per_head": int(N), "reps": reps,
-            "kernels": "pca_mean_kernel, pca_cov_kernel, pca_jacobi_kernel"}
+    return P, {"us": float(np.median(ts)), "heads": int(H), "keys_per_head": int(N), "reps": reps,
+               "kernels": "pca_mean_kernel, pca_cov_kernel, pca_jacobi_kernel",
+               "note": "P of every measurement comes from this calibration"}
+
+
+def fill_cache(L, w, cache, P, n_tokens, g_dev, dev, td):
+    """Bulk-append n_tokens synthetic tokens (keys of the workload's generator,
+    N(0, 1) values) at positions [0, n_tokens) of every row; returns the
+    appended (k, v) tensors."""
+    import torch
+    B, Hkv, D = w.batch, w.n_kv_heads, w.head_dim
+    k_pre = torch.empty((B, Hkv, n_tokens, D), dtype=td, device=dev)
+    for h in range(Hkv):
+        k_pre[:, h] = gen.device_keys(gen.make_key_model(w, h), B, n_tokens, g_dev, dev, td)
+    v_pre = torch.randn((B, Hkv, n_tokens, D), generator=g_dev, device=dev).to(td)
+    L.loki_append(cache, 0, k_pre, v_pre, P)
+    return k_pre, v_pre
+
+
+def time_calls(torch, stream, flush, calls, steps, warmup):
+    """Mean device time (us) of each call in `calls`, each in a loop of its own
+    over `steps` steps (call(i) for step i), the L2 flushed before every step
+    outside the events, every CHUNK steps queued behind a GPU sleep."""
+    res = []
+    for call in calls:
+        for i in range(warmup):
+            call(i)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CHUNK, steps))]
+        tot = 0.0
+        done = 0
+        while done < steps:
+            n = min(CHUNK, steps - done)
+            queue_ahead(torch, n)
+            for i in range(n):
+                flush.fill_(float(i & 7))
+                ev[i][0].record(stream)
+                call(done + i)
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            for i in range(n):
+                tot += ev[i][0].elapsed_time(ev[i][1])
+            done += n
+        res.append(tot * 1000.0 / steps)
+    return res
+
+
+def time_decode_workload(L, name, flush, stream, dev, steps, warmup, peak):
+    """One more decode workload timed in the same run: the Loki step and the
+    dense baseline on its own cache (with the low-rank plane, like the main
+    workload), each in a loop of its own, and the Loki step with the dense
+    kernel run before it."""
+    import torch
+    w = get_workload(name)
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    S, B, Hkv, Hq, D = w.seq_len, w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
+    P, _ = calibrate(L, [gen.calibration_keys(w, g) for g in range(Hkv)], dev, stream, reps=0)
+    cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, lowrank_dim=lowrank_width(w.d, w.dtype, D))
+    g_dev = torch.Generator(device=dev)
+    g_dev.manual_seed(w.seed * 131)
+    k_pre, v_pre = fill_cache(L, w, cache, P, S, g_dev, dev, td)
+    del k_pre, v_pre
+    qs = [torch.randn((B, Hq, D), generator=g_dev, device=dev).to(td) for _ in range(4)]
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    dout = torch.empty_like(out)
+    idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
+    loki = lambda i: L.loki_decode_attention(cache, S, qs[i % 4], P, w.d, w.k, out=out, idx=idx)
+    dense = lambda i: L.dense_decode_attention(cache, S, qs[i % 4], P, out=dout)
+
+    def both(i):
+        dense(i)
+        loki(i)
+    loki_us, dense_us = time_calls(torch, stream, flush, [loki, dense], steps, warmup)
+    # interleaved: events around the Loki call only, the dense call before it
+    for i in range(warmup):
+        both(i)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(CHUNK, steps))]
+    tot, done = 0.0, 0
+    while done < steps:
+        n = min(CHUNK, steps - done)
+        queue_ahead(torch, n)
+        for i in range(n):
+            flush.fill_(float(i & 7))
+            dense(done + i)
+            ev[i][0].record(stream)
+            loki(done + i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            tot += ev[i][0].elapsed_time(ev[i][1])
+        done += n
+    lb, db = w.loki_bytes(), w.dense_bytes()
+    del cache
+    torch.cuda.empty_cache()
+    return {"workload": name, "loki_us": loki_us, "dense_us": dense_us,
+            "loki_frac": lb / (loki_us * 1e-6) / 1e9 / peak, "dense_frac": db / (dense_us * 1e-6) / 1e9 / peak,
+            "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
+            "loki_after_dense_us": tot * 1000.0 / steps, "steps": steps,
+            "algorithmic_bytes": lb, "dense_bytes": db}
+
+
+def time_generation(L, name, flush, stream, dev, peak, warmup):
+    """The generation run as the pages state it: a prompt cache of prompt_len
+    tokens, then gen_steps decode steps, step t appending its token (rotated)
+    at position prompt_len + t inside the call and attending over
+    prompt_len + t + 1 tokens with k = floor(k_f * length).  The Loki step
+    (loki_decode_attention_append) and the dense step
+    (dense_decode_attention_append) each run the whole generation in a loop of
+    their own; mean device time per step, L2 flushed before every step."""
+    import torch
+    from workloads.configs import key_budget
+    w = get_workload(name)
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    B, Hkv, Hq, D = w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
+    T0, NS = w.prompt_len, w.gen_steps
+    cap = T0 + NS
+    P, _ = calibrate(L, [gen.calibration_keys(w, g) for g in range(Hkv)], dev, stream, reps=0)
+    cache = L.LokiCache(B, Hkv, D, cap, dtype=td, device=dev, lowrank_dim=lowrank_width(w.d, w.dtype, D))
+    g_dev = torch.Generator(device=dev)
+    g_dev.manual_seed(w.seed * 131)
+    k_pre, v_pre = fill_cache(L, w, cache, P, T0, g_dev, dev, td)
+    del k_pre, v_pre
+    NSET = 8
+    qs = [torch.randn((B, Hq, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
+    kn = [gen.device_keys(gen.make_key_model(w, 0), B * Hkv, 1, g_dev, dev, td).view(B, Hkv, D)
+          for _ in range(NSET)]
+    vn = [torch.randn((B, Hkv, D), generator=g_dev, device=dev).to(td) for _ in range(NSET)]
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    idxs = {}
+    ws = cache.workspace(cap, Hq)
+
+    def loki(t):
+        S = T0 + t + 1
+        k = key_budget(w.k_f, S)
+        if k not in idxs:
+            idxs[k] = torch.empty((B, Hkv, k), dtype=torch.int32, device=dev)
+        L.loki_decode_attention_append(cache, S, kn[t % NSET], vn[t % NSET], qs[t % NSET], P, w.d, k, out=out,
+                                       idx=idxs[k], workspace=ws)
+
+    def dense(t):
+        S = T0 + t + 1
+        L.dense_decode_attention_append(cache, S, kn[t % NSET], vn[t % NSET], qs[t % NSET], P, out=out)
+
+    for t in range(NS):  # every idx buffer exists before the timed loops
+        k = key_budget(w.k_f, T0 + t + 1)
+        idxs.setdefault(k, torch.empty((B, Hkv, k), dtype=torch.int32, device=dev))
+    loki_us, dense_us = time_calls(torch, stream, flush, [loki, dense], NS, min(warmup, NS))
+    e = w.elem_bytes
+    lb = sum(w.rows * ((T0 + t + 1) * w.d * e + key_budget(w.k_f, T0 + t + 1) * 2 * D * e)
+             for t in range(NS)) / NS
+    db = sum(w.rows * (T0 + t + 1) * 2 * D * e for t in range(NS)) / NS
+    del cache
+    torch.cuda.empty_cache()
+    return {"workload": name, "prompt_len": T0, "gen_steps": NS,
+            "loki_us_per_step": loki_us, "dense_us_per_step": dense_us, "speedup_vs_dense": dense_us / loki_us,
+            "loki_frac": lb / (loki_us * 1e-6) / 1e9 / peak, "dense_frac": db / (dense_us * 1e-6) / 1e9 / peak,
+            "mean_algorithmic_bytes_per_step": lb, "mean_dense_bytes_per_step": db,
+            "note": "each step appends its token inside the call (rotated key, value, low-rank plane) and "
+                    "attends over prompt_len + t + 1 tokens; the bytes exclude the append, as the pages' "
+                    "speedup does"}
 
 
 def time_paged(L, w, cache, qs, P, flush, stream, dev, steps: int, warmup: int, page: int = 16):
@@ -321,7 +539,6 @@ def run_ours(args):
     import torch.distributed as dist
 
     import sparse_decode_attention_loki_b200 as L
-    from sparse_decode_attention_loki_b200.calibration import pca_bases
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -337,10 +554,9 @@ def run_ours(args):
     S, B, Hkv, Hq, D = w.seq_len, w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
     stream = torch.cuda.current_stream(dev)
 
-    # offline calibration (host) and cache prefill: S-1 tokens; each step appends token S-1
-    calib = [gen.calibration_keys(w, g) for g in range(Hkv)]
-    P = pca_bases(calib).to(dev)
-    pca = time_pca(L, calib, dev, stream)
+    # offline calibration (on the GPU, loki_pca_calibrate) and cache prefill:
+    # S-1 tokens; each step appends token S-1
+    P, pca = calibrate(L, [gen.calibration_keys(w, g) for g in range(Hkv)], dev, stream)
     # the cache keeps a low-rank key plane as wide as d (contiguous score rows)
     d_lr = lowrank_width(w.d, w.dtype, D)
     cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, lowrank_dim=d_lr)
@@ -593,6 +809,18 @@ def run_ours(args):
         L.loki_decode_attention(cache, S, qs[j], P, D, w.k, out=out, idx=idx_exact)
         jac.append(L.topk_jaccard(idx, idx_exact))
     jaccard = torch.stack(jac)
+    rot, ncl, nct, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
+    _, dcl, dct, _ = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
+    # ---------------- the short-row decode and the pages' generation run, same session
+    extras = {}
+    if world == 1 and not args.no_extras:
+        peak_gbs, _ = peaks()
+        del cache
+        torch.cuda.empty_cache()
+        extras["short_decode"] = time_decode_workload(L, EXTRA_DECODE, flush, stream, dev,
+                                                      steps=max(args.steps, 200), warmup=args.warmup,
+                                                      peak=peak_gbs)
+        extras["generation"] = time_generation(L, GENERATION, flush, stream, dev, peak_gbs, args.warmup)
     h2d = q_host[0].numel() * q_host[0].element_size()
     d2h = out_host.numel() * 4 + idx_host.numel() * 4
 
@@ -601,8 +829,6 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     t_loki, t_dense, t_app, t_e2e, t_e2g = [float(x) for x in tt.tolist()]
-    rot, ncl, nct, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
-    _, dcl, dct, _ = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
 
     if rank == 0:
         K = args.steps
@@ -667,11 +893,9 @@ def run_ours(args):
                                  "p10": float(np.percentile(per_step_loki, 10)) * 1000.0,
                                  "p90": float(np.percentile(per_step_loki, 90)) * 1000.0},
         }
+        line.update(extras)
         if world == 1 and not args.no_cpu_baseline:
-            cus, rows, threads = oracle_sample_us(w, budget_s=args.cpu_budget)
-            line["cpu_baseline"] = {"value": cus, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": f"{rows} whole (batch, KV head) rows, fp64 numpy oracle, "
-                                              f"scaled to all {w.rows} rows of one layer-step"}
+            line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
         print(json.dumps(line))
     if world > 1:
         dist.barrier()
@@ -687,7 +911,6 @@ def run_sweep(args):
     import torch
 
     import sparse_decode_attention_loki_b200 as L
-    from sparse_decode_attention_loki_b200.calibration import pca_bases
     from workloads import mistral_sweep_points
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
@@ -719,7 +942,7 @@ def run_sweep(args):
     for (S, B), ws in groups.items():
         w0 = ws[0]
         Hkv, Hq, D = w0.n_kv_heads, w0.n_q_heads, w0.head_dim
-        P = pca_bases([gen.calibration_keys(w0, g) for g in range(Hkv)]).to(dev)
+        P, _ = calibrate(L, [gen.calibration_keys(w0, g) for g in range(Hkv)], dev, stream, reps=0)
         cache = L.LokiCache(B, Hkv, D, S, dtype=torch.bfloat16, device=dev)
         g_dev = torch.Generator(device=dev)
         g_dev.manual_seed(w0.seed * 131)
@@ -773,8 +996,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle CPU time")
+    ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle CPU time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the short-row decode and the generation run timed beside the main workload")
     ap.add_argument("--sweep", choices=["mistral"], default=None,
                     help="time Loki and dense on every Mistral sweep point instead of the bench step")
     ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")

@@ -389,6 +389,17 @@ LOKI_API loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t s
                                      int32_t n_q_heads, int32_t k, int32_t dense,
                                      int32_t *shape);
 
+/* Launch-shape override, for tests and tuning: per_row > 0 makes the
+ * following decode launches in this process use that many CTAs per (batch,
+ * KV head) row (the cluster size of the dense kernel; the number of key-stream
+ * units per row of the Loki step) wherever that shape can run, else the
+ * planner's choice; per_row == 0 restores the planner's choice.  The initial
+ * value is read once from the environment variable LOKI_CLUSTER (0 when
+ * unset).  Applies process-wide; an atomic, safe to call from any thread, but
+ * calls already enqueued keep the shape they were planned with.
+ * Returns LOKI_ERR_INVALID_ARG for per_row < 0.  Not part of the method. */
+LOKI_API loki_status loki_set_launch_override(int32_t per_row);
+
 /* Static description of a status code (never NULL). */
 LOKI_API const char *loki_status_string(loki_status s);
 

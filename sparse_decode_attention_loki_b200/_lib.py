@@ -87,6 +87,7 @@ SIGNATURES = {
     "dense_paged_decode_attention": (_i32, [_pcache_p, _seqs_p, _i32, _vp, _vp, ctypes.c_float, _vp, _vp]),
     "loki_pca_workspace_size": (_i32, [_i32, _i32, ctypes.POINTER(ctypes.c_size_t)]),
     "loki_pca_calibrate": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "loki_set_launch_override": (_i32, [_i32]),
     "loki_status_string": (ctypes.c_char_p, [_i32]),
     "loki_last_error": (ctypes.c_char_p, []),
     "loki_version": (_i32, []),

@@ -3,13 +3,11 @@
 The pages calibrate the PCA transform offline on a calibration set ("Loki:
 Low-rank Keys for Efficient Sparse Attention", atlas.scime.ai summary, summary
 paragraph).  Calibration is not on the decode path: it runs once, before any
-decode step, and hands P to the library as an input.  Two routes give the same
-basis: `pca_bases_gpu` runs the library's own kernels (loki_pca_calibrate:
-fp64 covariance and a Jacobi eigensolver on the device); `pca_basis` /
-`pca_bases` use torch's fp64 symmetric eigensolver on the host.  Both order
-the principal directions by descending eigenvalue (column j of P = direction
-j) and fix the sign of each column so that its largest-magnitude entry is
-positive.
+decode step, and hands P to the library as an input.  `pca_bases_gpu` runs
+the library's own kernels (loki_pca_calibrate: fp64 covariance and a Jacobi
+eigensolver on the device).  The principal directions are ordered by
+descending eigenvalue (column j of P = direction j) and the sign of each
+column makes its largest-magnitude entry positive.
 
 `choose_d` is a per-layer reduced-dimension policy: the pages vary d across
 layers in an ablation and report no clear effect on quality (summary page,
@@ -23,26 +21,6 @@ import math
 from typing import Sequence
 
 import torch
-
-
-def pca_basis(keys: torch.Tensor) -> torch.Tensor:
-    """keys: [N, D] calibration keys of one KV head -> P [D, D] fp32 (CPU)."""
-    X = keys.detach().to("cpu", torch.float64)
-    Xc = X - X.mean(dim=0, keepdim=True)
-    C = Xc.T @ Xc / X.shape[0]
-    w, V = torch.linalg.eigh(C)
-    order = torch.argsort(w, descending=True, stable=True)
-    V = V[:, order]
-    lead = V.abs().argmax(dim=0)
-    signs = torch.sign(V[lead, torch.arange(V.shape[1])])
-    signs[signs == 0] = 1.0
-    return (V * signs).to(torch.float32)
-
-
-def pca_bases(calib) -> torch.Tensor:
-    """One basis per KV head: calib is a sequence of [N, D] arrays/tensors ->
-    P [Hkv, D, D] fp32 (CPU)."""
-    return torch.stack([pca_basis(torch.as_tensor(c)) for c in calib])
 
 
 def pca_bases_gpu(calib: torch.Tensor) -> torch.Tensor:

@@ -65,11 +65,21 @@ loki_status device_info(DevInfo *out) {
   return LOKI_OK;
 }
 
-// Tuning override (development only): LOKI_CLUSTER forces the CTAs per row.
-int env_int(const char *name, int dflt) {
-  const char *s = std::getenv(name);
-  if (!s || !*s) return dflt;
-  return std::atoi(s);
+// Launch-shape override for tests and tuning (loki_set_launch_override):
+// the CTAs per row of the next launches, 0 for the planner's own choice.
+// Starts from LOKI_CLUSTER, read once; the library never writes the process
+// environment.
+std::atomic<int> g_override{-1};
+int forced_cluster() {
+  int v = g_override.load(std::memory_order_relaxed);
+  if (v < 0) {
+    const char *s = std::getenv("LOKI_CLUSTER");
+    int e = (s && *s) ? std::atoi(s) : 0;
+    if (e < 0) e = 0;
+    g_override.compare_exchange_strong(v, e, std::memory_order_relaxed);
+    v = g_override.load(std::memory_order_relaxed);
+  }
+  return v;
 }
 
 // ---------------------------------------------------------------------------
@@ -231,11 +241,10 @@ struct Plan {
 constexpr int kDenseMinTokens = 256;
 
 template <typename Kern>
-loki_status plan_dense(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan *p) {
+loki_status plan_dense(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan *p, int forced) {
   const int rows = sh.B * sh.Hkv;
   int dev = 0;
   cudaGetDevice(&dev);
-  const int forced = env_int("LOKI_CLUSTER", 0);
   double best = -1.0;
   Plan bp{0, 0, 0};
   int last_smem = 0;
@@ -255,12 +264,7 @@ loki_status plan_dense(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan
       bp = Plan{n, chunk, smem};
     }
   }
-  if (bp.ncta == 0 && forced) {
-    setenv("LOKI_CLUSTER", "", 1);  // a forced size that cannot run: plan normally
-    loki_status s = plan_dense(kern, di, sh, p);
-    setenv("LOKI_CLUSTER", std::to_string(forced).c_str(), 1);
-    return s;
-  }
+  if (bp.ncta == 0 && forced) return plan_dense(kern, di, sh, p, 0);  // a forced size that cannot run
   if (bp.ncta == 0)
     return fail(LOKI_ERR_UNSUPPORTED,
                 "no dense launch shape fits: %d B of shared memory per CTA (limit %d) or an unschedulable cluster",
@@ -300,7 +304,7 @@ loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a,
   loki_status s = allow_smem(kern, di, DenseGate<T, D, G, PAGED>::gate, true);
   if (s != LOKI_OK) return s;
   Plan pl;
-  s = plan_dense(kern, di, sh, &pl);
+  s = plan_dense(kern, di, sh, &pl, forced_cluster());
   if (s != LOKI_OK) return s;
   if (used) {  // shape query only: launch nothing
     *used = pl;
@@ -326,7 +330,7 @@ struct StepPlan {
 constexpr int kTargetChunk = 8192;
 
 template <typename Kern>
-loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepPlan *p) {
+loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepPlan *p, int forced) {
   const long long rows = (long long)sh.B * sh.Hkv;
   const int S = sh.S;
   int dev = 0;
@@ -337,7 +341,6 @@ loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepP
   if ((S + kMaxCluster - 1) / kMaxCluster > kMaxChunk)
     return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d exceeds %d tokens", S, kMaxChunk * kMaxCluster);
   if (need > kMaxCluster) need = kMaxCluster;
-  const int forced = env_int("LOKI_CLUSTER", 0);
   StepPlan best{0, 0, 0};
   for (int n = 1; n <= kMaxCluster; n *= 2) {
     if (forced ? n != forced : n < need) continue;
@@ -350,12 +353,7 @@ loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepP
     best = StepPlan{n, chunk, smem};
     if (forced || rows * 5 >= 4LL * mc) break;  // covers 80% of a wave
   }
-  if (best.ncta == 0 && forced) {
-    setenv("LOKI_CLUSTER", "", 1);  // a forced size that cannot run: plan normally
-    loki_status s = plan_step(kern, di, sh, p);
-    setenv("LOKI_CLUSTER", std::to_string(forced).c_str(), 1);
-    return s;
-  }
+  if (best.ncta == 0 && forced) return plan_step(kern, di, sh, p, 0);  // a forced size that cannot run
   if (best.ncta == 0)
     return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d: no schedulable cluster fits the keys in shared memory", S);
   *p = best;
@@ -376,7 +374,7 @@ loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da,
   loki_status s = allow_smem(kern, di, StepGate<T, D, G, PAGED>::gate, true);
   if (s != LOKI_OK) return s;
   StepPlan pl;
-  s = plan_step(kern, di, sh, &pl);
+  s = plan_step(kern, di, sh, &pl, forced_cluster());
   if (s != LOKI_OK) return s;
   if (used) {  // shape query only: launch nothing
     *used = pl;
@@ -1092,6 +1090,12 @@ const char *loki_status_string(loki_status s) {
     case LOKI_ERR_CUDA: return "LOKI_ERR_CUDA: the CUDA runtime reported an error";
   }
   return "unknown loki_status";
+}
+
+loki_status loki_set_launch_override(int32_t per_row) {
+  if (per_row < 0) return fail(LOKI_ERR_INVALID_ARG, "per_row %d must be >= 0", per_row);
+  g_override.store(per_row, std::memory_order_relaxed);
+  return LOKI_OK;
 }
 
 const char *loki_last_error(void) { return g_err; }

@@ -32,7 +32,8 @@ def test_header_declares_the_abi():
                           "loki_paged_append", "loki_paged_decode_workspace_size", "loki_paged_decode_attention",
                           "dense_paged_decode_attention", "loki_decode_attention_append",
                           "dense_decode_attention_append", "loki_paged_decode_attention_append",
-                          "loki_pca_calibrate", "loki_status_string", "loki_last_error", "loki_version"}
+                          "loki_pca_calibrate", "loki_set_launch_override", "loki_status_string", "loki_last_error",
+                          "loki_version"}
 
 
 def test_library_exports_every_declared_symbol(lib):

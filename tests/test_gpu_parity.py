@@ -32,18 +32,14 @@ def L():
 
 @contextlib.contextmanager
 def forced_cluster(n):
-    old = os.environ.get("LOKI_CLUSTER")
-    if n is None:
-        os.environ.pop("LOKI_CLUSTER", None)
-    else:
-        os.environ["LOKI_CLUSTER"] = str(n)
+    """Launches inside use n CTAs (dense) or key-stream units (Loki) per row
+    (loki_set_launch_override); None leaves the planner's choice."""
+    from sparse_decode_attention_loki_b200 import _lib
+    _lib.check(_lib.load().loki_set_launch_override(int(n or 0)))
     try:
         yield
     finally:
-        if old is None:
-            os.environ.pop("LOKI_CLUSTER", None)
-        else:
-            os.environ["LOKI_CLUSTER"] = old
+        _lib.check(_lib.load().loki_set_launch_override(0))
 
 
 def small_workload(dtype, D, G, S, Hkv=2, B=2, generator="powerlaw", seed=77):

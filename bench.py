@@ -903,6 +903,101 @@ def run_ours(args):
     return 0
 
 
+PHASES = ("query", "stream", "bucket", "select", "attend", "merge")
+
+
+def phase_summary(st, w, bin_us: float = 1.0):
+    """Phase stamps of one decode (loki_phase_stamps: per CTA the global timer
+    at kernel entry, queries ready, key stream done, first digit known,
+    selection known, attention done, merge done) summarised: the kernel span,
+    per phase the CTAs' durations, the achieved HBM rate of the key stream and
+    of the gather over the span of each phase across CTAs, and a timeline of
+    how many CTAs are in each phase per bin."""
+    st = st[st[:, 0] > 0]
+    t = st[:, :7].astype(np.float64)
+    T0 = t[:, 0].min()
+    t = (t - T0) / 1000.0
+    span = float(t[:, 6].max())
+
+    def q(x):
+        return {"p50": round(float(np.percentile(x, 50)), 2), "p90": round(float(np.percentile(x, 90)), 2),
+                "max": round(float(x.max()), 2)}
+    phases = {nm: q(t[:, i + 1] - t[:, i]) for i, nm in enumerate(PHASES)}
+    e = w.elem_bytes
+    key_bytes = w.rows * w.seq_len * w.d * e
+    gather_bytes = w.rows * w.k * 2 * w.head_dim * e
+    stream_window = float(t[:, 2].max() - t[:, 1].min())
+    gather_window = float(t[:, 5].max() - t[:, 4].min())
+    nb = int(np.ceil(span / bin_us))
+    tl = {nm: np.zeros(nb) for nm in PHASES}
+    for i in range(len(t)):
+        for p_, nm in enumerate(PHASES):
+            a_, b_ = t[i, p_], t[i, p_ + 1]
+            if b_ <= a_:
+                continue
+            for j in range(int(a_ // bin_us), min(nb - 1, int(b_ // bin_us)) + 1):
+                lo, hi = max(a_, j * bin_us), min(b_, (j + 1) * bin_us)
+                if hi > lo:
+                    tl[nm][j] += (hi - lo) / bin_us
+    return {"span_us": round(span, 2), "ctas": int(len(t)), "phase_us": phases,
+            "phase_ends_us": {nm: q(t[:, i + 1]) for i, nm in enumerate(PHASES)},
+            "stream_gbs_over_its_window": key_bytes / (stream_window * 1e-6) / 1e9 if stream_window > 0 else None,
+            "gather_gbs_over_its_window": gather_bytes / (gather_window * 1e-6) / 1e9 if gather_window > 0 else None,
+            "timeline_bin_us": bin_us,
+            "timeline_ctas": {k_: [round(float(x), 1) for x in v] for k_, v in tl.items()}}
+
+
+def run_phases(args):
+    """One Loki decode of the workload on a build with phase stamps
+    (-DLOKI_PHASE_STAMPS, built here as libloki_stamps.so): prints the
+    stamped build's decode time and the summary of its CTAs' phases
+    (phase_summary) as one JSON line."""
+    import ctypes
+    import torch
+
+    from sparse_decode_attention_loki_b200 import _lib
+    from sparse_decode_attention_loki_b200 import build as lbuild
+    path = os.path.join(os.path.dirname(lbuild.LIB), "libloki_stamps.so")
+    lbuild.build(defines=["-DLOKI_PHASE_STAMPS"], lib=path)
+    _lib.load(path)
+    import sparse_decode_attention_loki_b200 as L
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = get_workload(args.workload)
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    S, B, Hkv, Hq, D = w.seq_len, w.batch, w.n_kv_heads, w.n_q_heads, w.head_dim
+    P, _ = calibrate(L, [gen.calibration_keys(w, g) for g in range(Hkv)], dev, stream, reps=0)
+    cache = L.LokiCache(B, Hkv, D, S, dtype=td, device=dev, lowrank_dim=lowrank_width(w.d, w.dtype, D))
+    g_dev = torch.Generator(device=dev)
+    g_dev.manual_seed(w.seed * 131)
+    k_pre, v_pre = fill_cache(L, w, cache, P, S, g_dev, dev, td)
+    del k_pre, v_pre
+    q = torch.randn((B, Hq, D), generator=g_dev, device=dev).to(td)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
+    flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4, dtype=torch.float32,
+                        device=dev)
+    (us,) = time_calls(torch, stream, flush,
+                       [lambda i: L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx)],
+                       max(args.steps, 10), max(args.warmup, 3))
+    flush.fill_(3.0)
+    L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx)
+    torch.cuda.synchronize()
+    rot, ncta, ctas, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
+    buf = np.zeros((ctas, 10), dtype=np.uint64)
+    n = ctypes.c_int32(0)
+    _lib.check(_lib.load().loki_phase_stamps(1 if w.dtype == "bf16" else 0, D, buf.ctypes.data, ctas,
+                                             ctypes.byref(n)))
+    summ = phase_summary(buf[:n.value], w)
+    line = {"phases": w.name, "decode_us_stamped_build": us,
+            "launch": {"rotate_ctas": rot, "cluster_ctas": ncta, "ctas": ctas},
+            "single_cta_select": bool(int(buf[0, 8]) >> 16 & 1),
+            "algorithmic_bytes": w.loki_bytes(), **summ}
+    print(json.dumps(line))
+    return 0
+
+
 def run_sweep(args):
     """Loki against the in-library dense kernel on every point of the
     Mistral-7B-like sweep (S x B x d_f x k_f), one JSON line per point.  The
@@ -1004,6 +1099,8 @@ def main():
                     help="time Loki and dense on every Mistral sweep point instead of the bench step")
     ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
     ap.add_argument("--sweep-reps", type=int, default=20)
+    ap.add_argument("--phases", action="store_true",
+                    help="build the library with phase stamps and print the unit timeline of one decode")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps; the number is not a valid bench value", file=sys.stderr)
@@ -1011,6 +1108,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.phases:
+        return run_phases(args)
     return run_ours(args)
 
 

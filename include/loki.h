@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define LOKI_VERSION 11
+#define LOKI_VERSION 12
 
 /* Symbols are exported from the shared object; everything else is hidden. */
 #if defined(LOKI_BUILD) && defined(__GNUC__)
@@ -143,12 +143,13 @@ LOKI_API loki_status loki_decode_workspace_size(const loki_cache *cache, int32_t
  * the k tokens with the largest scores are selected, ties going to the lower
  * index; out_h = softmax(scale * q_hat_h . k_hat_i over the selected i, full D)
  * weighted sum of v_i.  The scores read the cache's low-rank plane when it has
- * one at least d wide, else k_hat; the gathered rows always come from k_hat.  Requires seq_len <= S_cap and G in {1, 2, 4, 8};
- * otherwise LOKI_ERR_INVALID_ARG or LOKI_ERR_UNSUPPORTED (also for seq_len
- * above 393216 tokens, whose scores would not fit on chip).  Enqueues one
- * kernel on the stream (query rotation, scores, selection, attention); for
- * query groups of 8 heads, two: the query rotation, then the decode kernel as
- * its programmatic dependent. */
+ * one at least d wide, else k_hat; the gathered rows always come from k_hat.
+ * Requires seq_len <= S_cap and G in {1, 2, 4, 8}; otherwise
+ * LOKI_ERR_INVALID_ARG or LOKI_ERR_UNSUPPORTED (also for seq_len above 393216
+ * tokens, whose scores would not fit on chip).  Enqueues one kernel on the
+ * stream (query rotation, scores, selection, attention); for query groups of
+ * 8 heads, two: the query rotation, then the decode kernel as its
+ * programmatic dependent. */
 LOKI_API loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_len,
                                   int32_t n_q_heads, const void *q, const float *P,
                                   int32_t d, int32_t k, float scale, float *out,
@@ -399,6 +400,21 @@ LOKI_API loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t s
  * calls already enqueued keep the shape they were planned with.
  * Returns LOKI_ERR_INVALID_ARG for per_row < 0.  Not part of the method. */
 LOKI_API loki_status loki_set_launch_override(int32_t per_row);
+
+/* Phase stamps of the last Loki decode on a cache of this dtype and head_dim
+ * (for profiling; builds compiled with -DLOKI_PHASE_STAMPS only, else
+ * LOKI_ERR_UNSUPPORTED).  host: host array of capacity * 10 uint64; entry c
+ * (CTA c of the decode kernel, up to 65536 CTAs) holds the device global timer
+ * in ns when the CTA started, when its queries were ready and its first key
+ * stages in flight, when its key stream was done, when the first digit of
+ * the selection was known, when its share of the selected rows was known,
+ * when its attention was done and when the cluster's merge was done; then
+ * its SM, then its rank in the cluster | cluster size << 8 | (1 << 16 when
+ * the row took the single-CTA select), then its (batch, KV head) row.
+ * Entries of CTAs the last decode did not have hold older data.  *n receives
+ * the number of entries copied.  Synchronous.  Not part of the method. */
+LOKI_API loki_status loki_phase_stamps(int32_t dtype, int32_t head_dim, uint64_t *host, int32_t capacity,
+                                       int32_t *n);
 
 /* Static description of a status code (never NULL). */
 LOKI_API const char *loki_status_string(loki_status s);

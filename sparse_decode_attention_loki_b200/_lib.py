@@ -88,6 +88,7 @@ SIGNATURES = {
     "loki_pca_workspace_size": (_i32, [_i32, _i32, ctypes.POINTER(ctypes.c_size_t)]),
     "loki_pca_calibrate": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "loki_set_launch_override": (_i32, [_i32]),
+    "loki_phase_stamps": (_i32, [_i32, _i32, _vp, _i32, ctypes.POINTER(_i32)]),
     "loki_status_string": (ctypes.c_char_p, [_i32]),
     "loki_last_error": (ctypes.c_char_p, []),
     "loki_version": (_i32, []),
@@ -96,16 +97,21 @@ SIGNATURES = {
 _lib = None
 
 
-def load() -> ctypes.CDLL:
-    """Load libloki.so once; raise if it is missing."""
+def load(path: str = None) -> ctypes.CDLL:
+    """Load libloki.so once; raise if it is missing.  `path` (first call only)
+    loads another build of the same library instead, e.g. one compiled with
+    phase stamps."""
     global _lib
     if _lib is not None:
+        if path is not None and path != _lib._name:
+            raise RuntimeError(f"{_lib._name} is already loaded")
         return _lib
-    if not os.path.exists(LIB_PATH):
+    path = path or LIB_PATH
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m sparse_decode_attention_loki_b200.build` "
+            f"{path} is missing: build it with `python -m sparse_decode_attention_loki_b200.build` "
             "(the CUDA library is required; there is no fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.restype = res

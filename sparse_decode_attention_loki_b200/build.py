@@ -2,8 +2,11 @@
 
     python -m sparse_decode_attention_loki_b200.build [--verbose]
 
-Cross-compiles without a GPU.  The shared object lands next to this file, where
-the Python binding loads it from.
+Cross-compiles without a GPU.  The decode kernels are compiled once per
+(cache dtype, head dim) pair from decode_inst.cu, the entry points and the
+other kernels from loki_api.cu; the five units build in parallel and are
+linked into one shared object next to this file, where the Python binding
+loads it from.
 """
 from __future__ import annotations
 
@@ -11,15 +14,23 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libloki.so")
+OBJDIR = os.path.join(PKG, "_build")
 
-SOURCES = ["loki_api.cu"]
-HEADERS = ["common.cuh", "decode.cuh", "append.cuh", "append_tc.cuh", "loki_step.cuh", "pca.cuh", "topk_stats.cuh"]
+# (source, extra defines, object name)
+UNITS = [
+    ("loki_api.cu", [], "loki_api.o"),
+    ("decode_inst.cu", ["-DLOKI_D=64"], "decode_f32_64.o"),
+    ("decode_inst.cu", ["-DLOKI_D=128"], "decode_f32_128.o"),
+    ("decode_inst.cu", ["-DLOKI_D=64", "-DLOKI_T_BF16"], "decode_bf16_64.o"),
+    ("decode_inst.cu", ["-DLOKI_D=128", "-DLOKI_T_BF16"], "decode_bf16_128.o"),
+]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -31,35 +42,56 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def command(verbose: bool = False) -> list:
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
-           "-DLOKI_BUILD", "-o", LIB]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    return cmd
+def _flags(extra=()) -> list:
+    return [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+            "-I", INCLUDE, "-I", CSRC, "-DLOKI_BUILD", *extra]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def commands(verbose: bool = False, defines=(), lib: str = LIB, objdir: str = OBJDIR):
+    """The compile commands of every unit and the link command."""
+    comp = []
+    for src, defs, obj in UNITS:
+        cmd = [nvcc(), *_flags([*defs, *defines]), "-c", "-o", os.path.join(objdir, obj), os.path.join(CSRC, src)]
+        if verbose:
+            cmd[1:1] = ["-Xptxas", "-v"]
+        comp.append(cmd)
+    link = [nvcc(), *ARCH, "--shared", "-o", lib, *[os.path.join(objdir, o) for _, _, o in UNITS]]
+    return comp, link
+
+
+def sources() -> list:
+    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC))] + [os.path.join(INCLUDE, "loki.h"),
+                                                                         os.path.abspath(__file__)]
+
+
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "loki.h"),
-                                                                 os.path.abspath(__file__)]
-    return all(os.path.getmtime(p) <= t for p in deps)
+    t = os.path.getmtime(lib)
+    return all(os.path.getmtime(p) <= t for p in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = command(verbose)
-    r = subprocess.run(cmd, capture_output=True, text=True)
+def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB) -> str:
+    """Compile and link `lib` (extra preprocessor `defines` for instrumented
+    builds, e.g. "-DLOKI_PHASE_STAMPS").  Returns its path."""
+    if not force and up_to_date(lib):
+        return lib
+    objdir = OBJDIR if lib == LIB else OBJDIR + "_" + os.path.splitext(os.path.basename(lib))[0]
+    os.makedirs(objdir, exist_ok=True)
+    comp, link = commands(verbose, defines, lib, objdir)
+    with ThreadPoolExecutor(max_workers=len(comp)) as ex:
+        results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), comp))
+    out = ""
+    for cmd, r in zip(comp, results):
+        if r.returncode != 0:
+            raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+        out += r.stdout + r.stderr
+    r = subprocess.run(link, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+        raise RuntimeError("link failed:\n" + " ".join(link) + "\n" + r.stdout + r.stderr)
     if verbose:
-        sys.stdout.write(r.stdout + r.stderr)
-    return LIB
+        sys.stdout.write(out)
+    return lib
 
 
 if __name__ == "__main__":

@@ -36,11 +36,9 @@
 #pragma once
 
 #include "append.cuh"
+#include "errors.cuh"
 
 namespace loki {
-
-// Device-side error count (timeouts of bounded waits); read by the host.
-static __device__ unsigned int g_loki_device_errors;
 
 constexpr int kTcM = 128;            // vectors per tile (the MMA's M)
 constexpr int kTcTerms = 3;          // bf16 terms of P

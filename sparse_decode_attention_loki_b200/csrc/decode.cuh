@@ -415,6 +415,8 @@ __device__ __forceinline__ void score_keys_loop(const R &rows, int t0, int len, 
   for (int y = 0; y < VEC; ++y) uv[y] = u[(c * VEC + y) % D];
   const int ns = SS::warp_stages(len);
   for (int s = 0; s < ns; ++s) {
+    // NS-1 stages in flight while stage s lands (refilling the slot of stage
+    // s-1 before this wait, NS in flight, measured slower on the long rows)
     cp_async_wait<NS - 2>();
     __syncwarp();
     SS::issue(rows, t0, len, nck, s + NS - 1, wring);
@@ -540,10 +542,11 @@ __device__ __forceinline__ void attend_loop(const R &rows, const int32_t *ids, i
       if (s == 0) cp_async_wait<0>();
       __syncwarp();
     } else {
-      cp_async_wait<kStages - 2>();
-      __syncwarp();
+      __syncwarp();  // stage s-1's slot is consumed: refill it before waiting for stage s
       RS::issue(rows, ids, tok0, cnt, s + kStages - 1, wring);
       cp_async_commit();
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
     }
     const unsigned char *st = wring + (s % kStages) * kWarpStageBytes;
     const int base = (s * kWarps + warp) * RS::TA;
@@ -778,10 +781,11 @@ __device__ __forceinline__ void attend_mma_loop(const R &rows, const int32_t *id
       if (s == 0) cp_async_wait<0>();
       __syncwarp();
     } else {
-      cp_async_wait<RS::NST - 2>();
-      __syncwarp();
+      __syncwarp();  // tile s-1's slot is consumed: refill it before waiting for tile s
       RS::issue(rows, ids, tok0, cnt, s + RS::NST - 1, wring);
       cp_async_commit();
+      cp_async_wait<RS::NST - 1>();
+      __syncwarp();
     }
     const unsigned char *st = wring + (s % RS::NST) * RS::TB;
     const int base = (s * kWarps + warp) * RS::TILE;

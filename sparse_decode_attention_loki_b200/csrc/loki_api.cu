@@ -13,14 +13,12 @@
 #include "loki.h"
 #include "append.cuh"
 #include "append_tc.cuh"
-#include "decode.cuh"
-#include "loki_step.cuh"
+#include "host.h"
 #include "pca.cuh"
+#include "loki_step.cuh"
 #include "topk_stats.cuh"
 
-namespace {
-
-using namespace loki;
+namespace loki {
 
 thread_local char g_err[512];
 
@@ -36,14 +34,6 @@ loki_status cuda_fail(cudaError_t e, const char *what) {
   return fail(LOKI_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-// Per-device attributes, read once per device.
-struct DevInfo {
-  int sms;
-  int smem_optin;
-};
-constexpr int kMaxDevices = 64;
 std::atomic<int> g_dev_ready[kMaxDevices];
 DevInfo g_dev[kMaxDevices];
 
@@ -82,14 +72,33 @@ int forced_cluster() {
   return v;
 }
 
-// ---------------------------------------------------------------------------
-// validation shared by the two decode entry points
-struct DecodeShape {
-  int B, Hkv, D, Scap, S, Hq, G;
-  size_t esize;
-  int d_lr;  // width of the cache's low-rank key plane, 0 without one
-};
+std::mutex g_occ_mu;
+std::vector<OccEntry> g_occ;
 
+bool occ_lookup(const void *kern, int dev, int ncta, int smem_q, int *n) {
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  for (const OccEntry &e : g_occ)
+    if (e.kern == kern && e.dev == dev && e.ncta == ncta && e.smem_q == smem_q) {
+      *n = e.n;
+      return true;
+    }
+  return false;
+}
+
+void occ_store(const void *kern, int dev, int ncta, int smem_q, int n) {
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  g_occ.push_back(OccEntry{kern, dev, ncta, smem_q, n});
+}
+
+
+}  // namespace loki
+
+namespace {
+
+using namespace loki;
+
+// ---------------------------------------------------------------------------
+// validation shared by the decode entry points
 loki_status check_cache(const loki_cache *c, DecodeShape *sh) {
   if (!c) return fail(LOKI_ERR_INVALID_ARG, "cache descriptor is NULL");
   if (c->dtype != LOKI_F32 && c->dtype != LOKI_BF16)
@@ -148,322 +157,6 @@ float resolve_scale(float scale, int D) {
   return s * 1.4426950408889634f;  // log2(e)
 }
 
-// ---------------------------------------------------------------------------
-// launches
-void set_cluster(cudaLaunchAttribute *attr, int ncta) {
-  attr->id = cudaLaunchAttributeClusterDimension;
-  attr->val.clusterDim.x = (unsigned)ncta;
-  attr->val.clusterDim.y = 1;
-  attr->val.clusterDim.z = 1;
-}
-void set_pdl(cudaLaunchAttribute *attr) {
-  attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr->val.programmaticStreamSerializationAllowed = 1;
-}
-
-// Launch `kern` on `grid` CTAs of kThreads threads, as a cluster of `ncta`
-// CTAs when ncta > 0 and as a programmatic dependent of the previous kernel on
-// the stream when pdl is set.
-template <typename Kern, typename Args>
-loki_status launch_ex(Kern kern, long long grid, int smem, int ncta, bool pdl, const Args &args, void *stream,
-                      const char *what) {
-  if (grid < 1 || grid > 0x7fffffffLL) return fail(LOKI_ERR_UNSUPPORTED, "%s: grid of %lld CTAs", what, grid);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  cfg.gridDim = dim3((unsigned)grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cfg.attrs = attr;
-  cfg.numAttrs = 0;
-  if (ncta > 0) set_cluster(&attr[cfg.numAttrs++], ncta);
-  if (pdl) set_pdl(&attr[cfg.numAttrs++]);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args);
-  if (e != cudaSuccess) return cuda_fail(e, what);
-  return LOKI_OK;
-}
-
-// Co-resident clusters of `ncta` CTAs for a kernel with `smem` bytes of
-// dynamic shared memory (cached per device, kernel, cluster size and 4 KB
-// shared-memory bucket).  0 if the device cannot schedule such a cluster.
-struct OccEntry {
-  const void *kern;
-  int dev, ncta, smem_q, clusters;
-};
-std::mutex g_occ_mu;
-std::vector<OccEntry> g_occ;
-
-template <typename Kern>
-int max_active_clusters(Kern kern, int dev, int ncta, int smem, int smem_limit) {
-  int smem_q = (smem + 4095) & ~4095;
-  if (smem_q > smem_limit) smem_q = smem;
-  {
-    std::lock_guard<std::mutex> lk(g_occ_mu);
-    for (const OccEntry &e : g_occ)
-      if (e.kern == (const void *)kern && e.dev == dev && e.ncta == ncta && e.smem_q == smem_q) return e.clusters;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3((unsigned)ncta, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem_q;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  set_cluster(&attr[0], ncta);
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-    (void)cudaGetLastError();
-    n = 0;
-  }
-  std::lock_guard<std::mutex> lk(g_occ_mu);
-  g_occ.push_back(OccEntry{(const void *)kern, dev, ncta, smem_q, n});
-  return n;
-}
-
-// Per-kernel, per-device record of the dynamic shared memory already allowed.
-struct SmemGate {
-  std::atomic<int> bytes[kMaxDevices];
-};
-
-// ---------------------------------------------------------------------------
-// dense decode: one cluster of ncta CTAs per (batch, KV head) row
-struct Plan {
-  int ncta;
-  int chunk;
-  int smem;
-};
-
-// Among cluster sizes whose per-CTA share is at least kDenseMinTokens tokens
-// and whose shared memory fits, take the one that keeps the most CTAs busy per
-// wave of co-resident clusters (rows*n / waves); ties go to the smaller
-// cluster, which spends less on the cross-CTA merge.  LOKI_CLUSTER (tuning
-// only) forces n.
-constexpr int kDenseMinTokens = 256;
-
-template <typename Kern>
-loki_status plan_dense(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan *p, int forced) {
-  const int rows = sh.B * sh.Hkv;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  double best = -1.0;
-  Plan bp{0, 0, 0};
-  int last_smem = 0;
-  for (int n = 1; n <= 16; n *= 2) {
-    if (forced && n != forced) continue;
-    const int chunk = (sh.S + n - 1) / n;
-    if (!forced && n > 1 && chunk < kDenseMinTokens) continue;
-    const int smem = decode_layout(sh.G, sh.D, chunk, false).words * 4;
-    last_smem = smem;
-    if (smem > di.smem_optin) continue;
-    const int mc = max_active_clusters(kern, dev, n, smem, di.smem_optin);
-    if (mc <= 0) continue;
-    const long long waves = (rows + mc - 1) / mc;
-    const double per_wave = (double)rows * n / (double)waves;
-    if (per_wave > best * 1.0001) {
-      best = per_wave;
-      bp = Plan{n, chunk, smem};
-    }
-  }
-  if (bp.ncta == 0 && forced) return plan_dense(kern, di, sh, p, 0);  // a forced size that cannot run
-  if (bp.ncta == 0)
-    return fail(LOKI_ERR_UNSUPPORTED,
-                "no dense launch shape fits: %d B of shared memory per CTA (limit %d) or an unschedulable cluster",
-                last_smem, di.smem_optin);
-  *p = bp;
-  return LOKI_OK;
-}
-
-// Raise a kernel's dynamic shared-memory limit to the device's opt-in maximum
-// (once per device and kernel: `gate` belongs to exactly one kernel) and allow
-// clusters of up to 16 CTAs.  Launches then pass their own smaller sizes.
-template <typename Kern>
-loki_status allow_smem(Kern kern, const DevInfo &di, SmemGate &gate, bool cluster) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (gate.bytes[dev].load(std::memory_order_acquire) >= di.smem_optin) return LOKI_OK;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.smem_optin);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
-  if (cluster) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(NonPortableClusterSizeAllowed)");
-  }
-  gate.bytes[dev].store(di.smem_optin, std::memory_order_release);
-  return LOKI_OK;
-}
-
-template <typename T, int D, int G, bool PAGED>
-struct DenseGate {
-  static SmemGate gate;
-};
-template <typename T, int D, int G, bool PAGED>
-SmemGate DenseGate<T, D, G, PAGED>::gate;
-
-template <typename T, int D, int G, bool PAGED>
-loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a, void *stream, Plan *used) {
-  auto kern = dense_decode_kernel<T, D, G, PAGED>;
-  loki_status s = allow_smem(kern, di, DenseGate<T, D, G, PAGED>::gate, true);
-  if (s != LOKI_OK) return s;
-  Plan pl;
-  s = plan_dense(kern, di, sh, &pl, forced_cluster());
-  if (s != LOKI_OK) return s;
-  if (used) {  // shape query only: launch nothing
-    *used = pl;
-    return LOKI_OK;
-  }
-  a.chunk = pl.chunk;
-  return launch_ex(kern, (long long)sh.B * sh.Hkv * pl.ncta, pl.smem, pl.ncta, false, a, stream,
-                   "dense_decode_kernel launch");
-}
-
-// ---------------------------------------------------------------------------
-// Loki step: rotate grid, then the decode grid as its programmatic dependent
-struct StepPlan {
-  int ncta, chunk, smem;
-};
-
-// CTAs per row (cluster size) of the decode kernel.  Start from the fewest
-// CTAs whose share is at most kTargetChunk tokens (two CTAs then fit on an SM;
-// more only when a share would exceed kMaxChunk), and take the first power of
-// two up to 16 whose grid covers at least 80% of the device's co-resident
-// CTAs, else the largest schedulable one: fewer, longer CTAs spend less on
-// the cross-CTA steps.  LOKI_CLUSTER (a tuning override) forces the size.
-constexpr int kTargetChunk = 8192;
-
-template <typename Kern>
-loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, StepPlan *p, int forced) {
-  const long long rows = (long long)sh.B * sh.Hkv;
-  const int S = sh.S;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  int need = 1;
-  while (need < kMaxCluster && (S + need - 1) / need > kTargetChunk) need *= 2;
-  while (need > 1 && (S + need - 1) / need > kMaxChunk) need *= 2;
-  if ((S + kMaxCluster - 1) / kMaxCluster > kMaxChunk)
-    return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d exceeds %d tokens", S, kMaxChunk * kMaxCluster);
-  if (need > kMaxCluster) need = kMaxCluster;
-  StepPlan best{0, 0, 0};
-  for (int n = 1; n <= kMaxCluster; n *= 2) {
-    if (forced ? n != forced : n < need) continue;
-    const int chunk = round4((S + n - 1) / n);
-    if (chunk > kMaxChunk) continue;
-    const int smem = fused_smem(sh.G, sh.D, chunk).words * 4;
-    if (smem > di.smem_optin) continue;
-    const int mc = max_active_clusters(kern, dev, n, smem, di.smem_optin);
-    if (mc <= 0) continue;
-    best = StepPlan{n, chunk, smem};
-    if (forced || rows * 5 >= 4LL * mc) break;  // covers 80% of a wave
-  }
-  if (best.ncta == 0 && forced) return plan_step(kern, di, sh, p, 0);  // a forced size that cannot run
-  if (best.ncta == 0)
-    return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d: no schedulable cluster fits the keys in shared memory", S);
-  *p = best;
-  return LOKI_OK;
-}
-
-template <typename T, int D, int G, bool PAGED>
-struct StepGate {
-  static SmemGate gate;
-};
-template <typename T, int D, int G, bool PAGED>
-SmemGate StepGate<T, D, G, PAGED>::gate;
-
-template <typename T, int D, int G, bool PAGED>
-loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da, void *ws, void *stream,
-                     StepPlan *used) {
-  auto kern = loki_decode_kernel<T, D, G, PAGED>;
-  loki_status s = allow_smem(kern, di, StepGate<T, D, G, PAGED>::gate, true);
-  if (s != LOKI_OK) return s;
-  StepPlan pl;
-  s = plan_step(kern, di, sh, &pl, forced_cluster());
-  if (s != LOKI_OK) return s;
-  if (used) {  // shape query only: launch nothing
-    *used = pl;
-    return LOKI_OK;
-  }
-  const long long rows = (long long)sh.B * sh.Hkv;
-  const WsLayout W = ws_layout(rows, G, D);
-  unsigned char *w = static_cast<unsigned char *>(ws);
-  da.chunk = pl.chunk;
-  StepArgs<T> a;
-  a.da = da;
-  a.qhat = reinterpret_cast<float *>(w + W.qhat);
-  a.u = reinterpret_cast<float *>(w + W.u);
-  if (!kRotateInKernel<G>) {
-    s = launch_ex(loki_rotate_kernel<T, D, G>, rows * (D / kRotCols), 0, 0, false, a, stream,
-                  "loki_rotate_kernel launch");
-    if (s != LOKI_OK) return s;
-  }
-  return launch_ex(kern, rows * pl.ncta, pl.smem, pl.ncta, !kRotateInKernel<G>, a, stream,
-                   "loki_decode_kernel launch");
-}
-
-// ---------------------------------------------------------------------------
-template <typename T, int D, int G, bool PAGED>
-loki_status dispatch_p(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
-                       void *stream, Plan *used) {
-  if (dense) return run_dense<T, D, G, PAGED>(di, sh, a, stream, used);
-  StepPlan sp;
-  loki_status s = run_step<T, D, G, PAGED>(di, sh, a, ws, stream, used ? &sp : nullptr);
-  if (s == LOKI_OK && used) *used = Plan{sp.ncta, sp.chunk, sp.smem};
-  return s;
-}
-
-template <typename T, int D, bool PAGED>
-loki_status launch_append(AppendArgs<T> a, void *stream);
-
-template <typename T, int D, int G>
-loki_status dispatch(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
-                     void *stream, Plan *used) {
-  if (!dense && a.k_new != nullptr && !kRotateInKernel<G>) {
-    // the decode kernel appends only for query groups of up to 4 heads: for
-    // 8, the append kernel writes the new token first (contiguous caches)
-    if (a.table != nullptr)
-      return fail(LOKI_ERR_UNSUPPORTED, "appending in a paged Loki decode needs query groups of up to 4 heads");
-    if (used == nullptr) {
-      AppendArgs<T> ap{};
-      ap.k_hat = const_cast<T *>(a.k_hat);
-      ap.v = const_cast<T *>(a.v);
-      ap.k_new = a.k_new;
-      ap.v_new = a.v_new;
-      ap.P = a.P;
-      ap.k_lr = const_cast<T *>(a.k_lr);
-      ap.d_lr = a.d_lr;
-      ap.n_kv_heads = a.n_kv_heads;
-      ap.capacity = a.capacity;
-      ap.pos = sh.S - 1;
-      ap.n_new = 1;
-      ap.n_vec = sh.B;
-      loki_status s = launch_append<T, D, false>(ap, stream);
-      if (s != LOKI_OK) return s;
-    }
-    DecodeArgs<T> rest = a;
-    rest.k_new = rest.v_new = nullptr;
-    return dispatch_p<T, D, G, false>(dense, di, sh, rest, ws, stream, used);
-  }
-  if (a.table != nullptr) return dispatch_p<T, D, G, true>(dense, di, sh, a, ws, stream, used);
-  return dispatch_p<T, D, G, false>(dense, di, sh, a, ws, stream, used);
-}
-
-template <typename T, int D>
-loki_status dispatch_g(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
-                       void *stream, Plan *used) {
-  switch (sh.G) {
-    case 1: return dispatch<T, D, 1>(dense, di, sh, a, ws, stream, used);
-    case 2: return dispatch<T, D, 2>(dense, di, sh, a, ws, stream, used);
-    case 4: return dispatch<T, D, 4>(dense, di, sh, a, ws, stream, used);
-    case 8: return dispatch<T, D, 8>(dense, di, sh, a, ws, stream, used);
-  }
-  return fail(LOKI_ERR_UNSUPPORTED, "group size %d", sh.G);
-}
-
-// Per-sequence lengths and paging of a decode call (all null: a contiguous
-// cache where every row has seq_len tokens and takes k).
-struct VarPage {
-  const int32_t *seq_lens = nullptr, *ks = nullptr, *table = nullptr;
-  int32_t pages_per_seq = 0, page_shift = 0, num_pages = 0;
-  const void *k_new = nullptr, *v_new = nullptr;  // a token appended by the call, [B, Hkv, D]
-};
-
 template <typename T>
 loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense, const void *q, const float *P,
                           int32_t d, int32_t k, float scale, float *out, int32_t *idx, void *ws, void *stream,
@@ -502,8 +195,8 @@ loki_status decode_common(const loki_cache *c, const DecodeShape &sh, bool dense
   a.k_lr = sh.d_lr > 0 ? static_cast<const T *>(c->k_lr) : nullptr;
   a.d_lr = sh.d_lr;
   a.lr_read = a.k_lr != nullptr && d <= sh.d_lr;
-  if (sh.D == 64) return dispatch_g<T, 64>(dense, di, sh, a, ws, stream, used);
-  return dispatch_g<T, 128>(dense, di, sh, a, ws, stream, used);
+  if (sh.D == 64) return decode_td<T, 64>(dense, di, sh, a, ws, stream, used);
+  return decode_td<T, 128>(dense, di, sh, a, ws, stream, used);
 }
 
 template <int D, bool PAGED>
@@ -586,6 +279,36 @@ loki_status run_append(const loki_cache *c, int32_t pos, int32_t n_new, const vo
   a.n_vec = c->batch * n_new;
   return launch_append<T, D, false>(a, stream);
 }
+
+}  // namespace
+
+namespace loki {
+
+loki_status append_token(int dtype, int D, void *k_hat, void *v, void *k_lr, int d_lr, int Hkv, int capacity, int pos,
+                         int B, const void *k_new, const void *v_new, const float *P, void *stream) {
+  auto go = [&](auto *tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    AppendArgs<T> ap{};
+    ap.k_hat = static_cast<T *>(k_hat);
+    ap.v = static_cast<T *>(v);
+    ap.k_new = static_cast<const T *>(k_new);
+    ap.v_new = static_cast<const T *>(v_new);
+    ap.P = P;
+    ap.k_lr = static_cast<T *>(k_lr);
+    ap.d_lr = k_lr ? d_lr : 0;
+    ap.n_kv_heads = Hkv;
+    ap.capacity = capacity;
+    ap.pos = pos;
+    ap.n_new = 1;
+    ap.n_vec = B;
+    return D == 64 ? launch_append<T, 64, false>(ap, stream) : launch_append<T, 128, false>(ap, stream);
+  };
+  return dtype == LOKI_F32 ? go(static_cast<float *>(nullptr)) : go(static_cast<__nv_bfloat16 *>(nullptr));
+}
+
+}  // namespace loki
+
+namespace {
 
 // ---------------------------------------------------------------------------
 // Fixed scratch of loki_decode_attention_noalloc: a file-scope device array
@@ -722,6 +445,8 @@ loki_status run_pca(const T *keys, int32_t H, int32_t N, float *P, double *eigva
 }
 
 }  // namespace
+
+using namespace loki;
 
 extern "C" {
 
@@ -903,8 +628,7 @@ loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, i
     s = decode_common<__nv_bfloat16>(cache, sh, dense != 0, nullptr, nullptr, 1, 1, 0.f, nullptr, nullptr, nullptr,
                                      nullptr, &pl);
   if (s != LOKI_OK) return s;
-  const bool rot = !dense && sh.G > 4;  // kRotateInKernel<G> is G <= 4
-  shape[0] = rot ? (int32_t)(rows * (sh.D / kRotCols)) : 0;
+  shape[0] = dense ? 0 : pl.rot;
   shape[1] = pl.ncta;
   shape[2] = (int32_t)(rows * pl.ncta);
   shape[3] = 0;
@@ -1090,6 +814,19 @@ const char *loki_status_string(loki_status s) {
     case LOKI_ERR_CUDA: return "LOKI_ERR_CUDA: the CUDA runtime reported an error";
   }
   return "unknown loki_status";
+}
+
+loki_status loki_phase_stamps(int32_t dtype, int32_t head_dim, uint64_t *host, int32_t capacity, int32_t *n) {
+  if (!host || !n || capacity < 1) return fail(LOKI_ERR_INVALID_ARG, "host, n and capacity >= 1 are required");
+  if (head_dim != 64 && head_dim != 128) return fail(LOKI_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", head_dim);
+  unsigned long long *h = reinterpret_cast<unsigned long long *>(host);
+  if (dtype == LOKI_F32)
+    return head_dim == 64 ? decode_phase_stamps<float, 64>(h, capacity, n)
+                          : decode_phase_stamps<float, 128>(h, capacity, n);
+  if (dtype == LOKI_BF16)
+    return head_dim == 64 ? decode_phase_stamps<__nv_bfloat16, 64>(h, capacity, n)
+                          : decode_phase_stamps<__nv_bfloat16, 128>(h, capacity, n);
+  return fail(LOKI_ERR_INVALID_ARG, "dtype %d", dtype);
 }
 
 loki_status loki_set_launch_override(int32_t per_row) {

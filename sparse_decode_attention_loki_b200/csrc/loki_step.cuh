@@ -44,6 +44,28 @@
 
 namespace loki {
 
+// Phase stamps of the decode kernel (builds with -DLOKI_PHASE_STAMPS only):
+// per CTA, the global timer at eight points of the step, then its SM, rank
+// and row.  Read by loki_phase_stamps.
+constexpr int kMaxStampCtas = 1 << 16;
+constexpr int kStampWords = 10;
+#ifdef LOKI_PHASE_STAMPS
+static __device__ unsigned long long g_phase_stamps[kMaxStampCtas][kStampWords];
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define LOKI_PHASE(i)                                                               \
+  do {                                                                              \
+    if (threadIdx.x == 0 && blockIdx.x < kMaxStampCtas) g_phase_stamps[blockIdx.x][i] = global_ns(); \
+  } while (0)
+#else
+#define LOKI_PHASE(i) \
+  do {                \
+  } while (0)
+#endif
+
 constexpr int kDig1Bits = 11;                   // first radix digit: key bits 31..21
 constexpr int kDig1Bins = 1 << kDig1Bits;       // 2048
 constexpr int kDig2Bits = 11;                   // second digit: bits 20..10
@@ -499,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   const int len = min(S, t0 + a.da.chunk) - t0;
   const Rows<T, D, PAGED> rows = make_rows<T, D, PAGED>(a.da, b, g);
   constexpr int MAXL = D / VecN<T>::value;
+  LOKI_PHASE(0);
 
   // 1. the queries (q_hat, u) and the key stream; the stream's first stages
   // go in flight before u is needed.  An appended token sits at the row's
@@ -525,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   }
   for (int e = tid; e < skewed_words(kDig1Bins); e += kThreads) hist[e] = 0u;
   __syncthreads();
+  LOKI_PHASE(1);
   cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
                     (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(rows, t0, slen, a.da.nck,
@@ -545,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     __syncthreads();
   }
 
+  LOKI_PHASE(2);
   // 2. cluster radix select; the ring is idle until the gather
   const bool leader = rank == 0;
   int32_t *idx_row = a.da.idx + (size_t)row * a.da.k_stride;
@@ -559,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     // chunk a multiple of 4) into its ring and selects alone
     if (!leader) push_skewed(hist, kDig1Bins, dsmem_addr(hist, 0u));
     cluster.sync();  // every stream is done; the leader's histogram holds the row's
+    LOKI_PHASE(3);
     uint32_t *all = rw + kAllKeys;
     if (leader) {
       const int n4 = (S + 3) >> 2;
@@ -645,6 +671,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     }
   }
   cluster.sync();
+  LOKI_PHASE(3);
   uint32_t remaining = k - ctl[kSelFirst + 1];
   const bool refine = ctl[kSelFirst + 2] != remaining;  // else the whole bucket is taken
   uint32_t prefix = ctl[kSelFirst + 0] << (32 - kDig1Bits);
@@ -874,6 +901,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   // 3. attention over this CTA's even share of the k selected rows (the
   // share is at most chunk)
   __syncthreads();
+  LOKI_PHASE(4);
   if constexpr (PAGED) {
     // the share's token positions become rows of the page pools first (one
     // page-table load each, all in flight at once), so that the gather loop
@@ -890,12 +918,24 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
                                    pm, pl, pacc);
   }
 
+  LOKI_PHASE(5);
   // 4. log-sum-exp merge of the cluster's states
   if (gather && !leader) cluster_wait();
   cluster.sync();
   const int Hq = a.da.n_kv_heads * G;
   cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
   cluster.sync();
+  LOKI_PHASE(6);
+#ifdef LOKI_PHASE_STAMPS
+  if (tid == 0 && blockIdx.x < kMaxStampCtas) {
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    g_phase_stamps[blockIdx.x][7] = sm;
+    g_phase_stamps[blockIdx.x][8] = (unsigned long long)rank | ((unsigned long long)ncta << 8) |
+                                    ((unsigned long long)(gather ? 1 : 0) << 16);
+    g_phase_stamps[blockIdx.x][9] = (unsigned long long)row;
+  }
+#endif
 }
 
 }  // namespace loki

@@ -32,7 +32,7 @@ def test_header_declares_the_abi():
                           "loki_paged_append", "loki_paged_decode_workspace_size", "loki_paged_decode_attention",
                           "dense_paged_decode_attention", "loki_decode_attention_append",
                           "dense_decode_attention_append", "loki_paged_decode_attention_append",
-                          "loki_pca_calibrate", "loki_set_launch_override", "loki_status_string", "loki_last_error",
+                          "loki_pca_calibrate", "loki_set_launch_override", "loki_phase_stamps", "loki_status_string", "loki_last_error",
                           "loki_version"}
 
 
@@ -49,12 +49,13 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_library_is_built_for_sm100a():
     from sparse_decode_attention_loki_b200 import build
-    cmd = " ".join(build.command())
-    assert "arch=compute_100a,code=sm_100a" in cmd
+    comp, link = build.commands()
+    for cmd in comp + [link]:
+        assert "arch=compute_100a,code=sm_100a" in " ".join(cmd)
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 11
+    assert lib.loki_version() == 12
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"
@@ -104,11 +105,12 @@ def test_decode_null_pointers(lib):
     assert lib.dense_decode_attention(ctypes.byref(c), 0, 2, FAKE, FAKE, 0.0, FAKE, None) == 1
 
 
-def _ws_bytes(rows, G, D):
+def _ws_bytes(B, Hkv, G, D, S=None):
     """The workspace regions include/loki.h documents, each 256-byte aligned:
     the rotated queries [rows, G, D] and the low-rank group queries [rows, D],
-    fp32."""
+    fp32 (no dependence on the length)."""
     a = lambda x: (x + 255) // 256 * 256
+    rows = B * Hkv
     return a(rows * G * D * 4) + a(rows * D * 4)
 
 
@@ -117,12 +119,12 @@ def test_workspace_size_and_validation(lib):
     n = ctypes.c_size_t(0)
     for S, hq in [(10, 2), (64, 4), (4999, 16), (5000, 2)]:
         assert lib.loki_decode_workspace_size(ctypes.byref(c), S, hq, ctypes.byref(n)) == 0
-        assert n.value == _ws_bytes(6, hq // 2, 128)
+        assert n.value == _ws_bytes(3, 2, hq // 2, 128, S)
     assert lib.loki_decode_workspace_size(ctypes.byref(c), 5001, 2, ctypes.byref(n)) == 1
     assert lib.loki_decode_workspace_size(ctypes.byref(c), 0, 2, ctypes.byref(n)) == 1
     assert lib.loki_decode_workspace_size(ctypes.byref(c), 10, 3, ctypes.byref(n)) == 1
     assert lib.loki_decode_workspace_size(ctypes.byref(c), 10, 2, None) == 1
-    need = _ws_bytes(6, 1, 128)
+    need = _ws_bytes(3, 2, 1, 128, 10)
     args = (ctypes.byref(c), 10, 2, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE)
     assert lib.loki_decode_attention(*args, None, WSB, None) == 1          # no workspace
     assert lib.loki_decode_attention(*args, WS + 16, WSB, None) == 1       # not 256-byte aligned
@@ -205,7 +207,7 @@ def test_paged_workspace_size_and_cache_validation(lib):
     n = ctypes.c_size_t(0)
     c, q = _paged(), _seqs()
     assert lib.loki_paged_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 4, ctypes.byref(n)) == 0
-    assert n.value == _ws_bytes(4, 2, 128)
+    assert n.value == _ws_bytes(2, 2, 2, 128, 50)
     bad_caches = [_paged(page=24), _paged(page=0), _paged(page=1 << 17), _paged(pages=0), _paged(dtype=5),
                   _paged(H=0), _paged(k=0), _paged(v=FAKE + 8)]
     for bc in bad_caches:
@@ -234,7 +236,7 @@ def test_paged_workspace_size_and_cache_validation(lib):
 
 def test_paged_decode_validation(lib):
     c, q = _paged(), _seqs()
-    need = _ws_bytes(4, 2, 128)
+    need = _ws_bytes(2, 2, 2, 128, 50)
     base = dict(hq=4, qp=FAKE, P=FAKE, d=32, ks=FAKE, kmax=10, out=FAKE, idx=FAKE, ws=WS, wsb=need)
     def call(**kw):
         a = dict(base)
@@ -271,7 +273,7 @@ def test_paged_append_validation(lib):
 
 def test_append_decode_validation(lib):
     c = _cache(B=1, H=2, cap=64)
-    need = _ws_bytes(2, 1, 128)
+    need = _ws_bytes(1, 2, 1, 128, 10)
     base = (ctypes.byref(c), 10, 2)
     tail = (FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE, WS, need, None)
     assert lib.loki_decode_attention_append(*base, None, FAKE, *tail) == 1
@@ -283,11 +285,11 @@ def test_append_decode_validation(lib):
     assert lib.dense_decode_attention_append(*base, None, FAKE, FAKE, FAKE, 0.0, FAKE, None) == 1
     assert lib.dense_decode_attention_append(*base, FAKE, FAKE + 4, FAKE, FAKE, 0.0, FAKE, None) == 1
     pc, pq = _paged(), _seqs()
-    pneed = _ws_bytes(4, 2, 128)
+    pneed = _ws_bytes(2, 2, 2, 128, 50)
     assert lib.loki_paged_decode_attention_append(ctypes.byref(pc), ctypes.byref(pq), 4, None, FAKE, FAKE, FAKE, 32,
                                                   None, 10, 0.0, FAKE, FAKE, WS, pneed, None) == 1
     assert lib.loki_paged_decode_attention_append(ctypes.byref(pc), ctypes.byref(pq), 16, FAKE, FAKE, FAKE, FAKE, 32,
-                                                  None, 10, 0.0, FAKE, FAKE, WS, _ws_bytes(4, 8, 128), None) == 2
+                                                  None, 10, 0.0, FAKE, FAKE, WS, _ws_bytes(2, 2, 8, 128), None) == 2
 
 
 def test_cache_struct_layout():

@@ -266,7 +266,8 @@ def test_workspace_needs_no_initialisation_and_is_shared_across_shapes():
                             oracle.default_scale(D), dtype)
 
 
-@pytest.mark.parametrize("S,B,Hkv,G", [(20000, 1, 2, 1), (4096, 16, 8, 4), (257, 3, 2, 2), (70001, 1, 1, 4)])
+@pytest.mark.parametrize("S,B,Hkv,G", [(20000, 1, 2, 1), (4096, 16, 8, 4), (257, 3, 2, 2), (70001, 1, 1, 4),
+                                       (9000, 3, 2, 8)])
 def test_cluster_shapes_and_ragged_chunks(S, B, Hkv, G):
     # rows split over clusters of several CTAs with a ragged last chunk, grids
     # of several waves, and a row longer than one CTA can hold

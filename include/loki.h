@@ -165,9 +165,10 @@ LOKI_API loki_status loki_decode_attention(const loki_cache *cache, int32_t seq_
  * Arguments and results are those of loki_decode_attention, minus the
  * workspace.  The scratch is instead a fixed 4 MiB array in the library's
  * device code, which every GPU that loads the library holds until the process
- * exits; the call allocates and frees nothing.  A call whose
- * loki_decode_workspace_size exceeds 4 MiB returns LOKI_ERR_UNSUPPORTED with a
- * message, and enqueues nothing.  The first call on each device looks up the
+ * exits; the call allocates and frees nothing.  Query groups of up to 4 heads
+ * use none of it; for groups of 8, a call whose loki_decode_workspace_size
+ * exceeds 4 MiB returns LOKI_ERR_UNSUPPORTED with a message, and enqueues
+ * nothing.  The first call on each device looks up the
  * array's device address (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture.  Every call on a device
  * shares the one array and leaves its contents behind (nothing in it needs to

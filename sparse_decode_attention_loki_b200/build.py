@@ -4,9 +4,9 @@
 
 Cross-compiles without a GPU.  The decode kernels are compiled once per
 (cache dtype, head dim) pair from decode_inst.cu, the entry points and the
-other kernels from loki_api.cu; the five units build in parallel and are
-linked into one shared object next to this file, where the Python binding
-loads it from.
+other kernels from loki_api.cu; the five units build in parallel (objects in
+a temporary directory) and are linked into one shared object next to this
+file, where the Python binding loads it from.
 """
 from __future__ import annotations
 
@@ -14,6 +14,7 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
 from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -21,7 +22,6 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libloki.so")
-OBJDIR = os.path.join(PKG, "_build")
 
 # (source, extra defines, object name)
 UNITS = [
@@ -47,7 +47,7 @@ def _flags(extra=()) -> list:
             "-I", INCLUDE, "-I", CSRC, "-DLOKI_BUILD", *extra]
 
 
-def commands(verbose: bool = False, defines=(), lib: str = LIB, objdir: str = OBJDIR):
+def commands(verbose: bool = False, defines=(), lib: str = LIB, objdir: str = "_build"):
     """The compile commands of every unit and the link command."""
     comp = []
     for src, defs, obj in UNITS:
@@ -76,19 +76,18 @@ def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB
     builds, e.g. "-DLOKI_PHASE_STAMPS").  Returns its path."""
     if not force and up_to_date(lib):
         return lib
-    objdir = OBJDIR if lib == LIB else OBJDIR + "_" + os.path.splitext(os.path.basename(lib))[0]
-    os.makedirs(objdir, exist_ok=True)
-    comp, link = commands(verbose, defines, lib, objdir)
-    with ThreadPoolExecutor(max_workers=len(comp)) as ex:
-        results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), comp))
-    out = ""
-    for cmd, r in zip(comp, results):
+    with tempfile.TemporaryDirectory(prefix="loki_build_") as objdir:  # objects live only for the link
+        comp, link = commands(verbose, defines, lib, objdir)
+        with ThreadPoolExecutor(max_workers=len(comp)) as ex:
+            results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), comp))
+        out = ""
+        for cmd, r in zip(comp, results):
+            if r.returncode != 0:
+                raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+            out += r.stdout + r.stderr
+        r = subprocess.run(link, capture_output=True, text=True)
         if r.returncode != 0:
-            raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
-        out += r.stdout + r.stderr
-    r = subprocess.run(link, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError("link failed:\n" + " ".join(link) + "\n" + r.stdout + r.stderr)
+            raise RuntimeError("link failed:\n" + " ".join(link) + "\n" + r.stdout + r.stderr)
     if verbose:
         sys.stdout.write(out)
     return lib

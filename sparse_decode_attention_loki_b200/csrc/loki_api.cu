@@ -509,7 +509,10 @@ loki_status loki_decode_attention_noalloc(const loki_cache *cache, int32_t seq_l
   size_t need = 0;
   loki_status s = loki_decode_workspace_size(cache, seq_len, n_q_heads, &need);
   if (s != LOKI_OK) return s;
-  if (need > kNoAllocScratchBytes)
+  // query groups of up to 4 heads rotate their queries on chip and use no
+  // scratch: only groups of 8 need the array to hold their workspace
+  const bool small_group = n_q_heads / cache->n_kv_heads <= 4;
+  if (!small_group && need > kNoAllocScratchBytes)
     return fail(LOKI_ERR_UNSUPPORTED,
                 "this call needs %zu bytes of scratch; the fixed scratch of loki_decode_attention_noalloc holds "
                 "%zu (use loki_decode_attention with a workspace)",
@@ -517,8 +520,10 @@ loki_status loki_decode_attention_noalloc(const loki_cache *cache, int32_t seq_l
   void *scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != LOKI_OK) return s;
+  // small groups: the decode never reads or writes the workspace, whatever
+  // size loki_decode_attention would ask of a caller's one
   return loki_decode_attention(cache, seq_len, n_q_heads, q, P, d, k, scale, out, idx, scratch,
-                               kNoAllocScratchBytes, stream);
+                               small_group ? need : kNoAllocScratchBytes, stream);
 }
 
 loki_status loki_device_error_count(uint32_t *count) {

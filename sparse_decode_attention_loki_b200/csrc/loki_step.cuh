@@ -66,6 +66,19 @@ __device__ __forceinline__ unsigned long long global_ns() {
   } while (0)
 #endif
 
+// Geometry of the low-rank key stream's per-warp ring slice: stages of
+// kScoreStageBytes, kScoreStages of them (kScoreStages - 1 in flight).  The
+// slice is the same 8 KB per warp as the attention's.
+#ifndef LOKI_SCORE_STAGE_BYTES
+#define LOKI_SCORE_STAGE_BYTES 2048
+#endif
+#ifndef LOKI_SCORE_STAGES
+#define LOKI_SCORE_STAGES 4
+#endif
+constexpr int kScoreStageBytes = LOKI_SCORE_STAGE_BYTES;
+constexpr int kScoreStages = LOKI_SCORE_STAGES;
+static_assert(kScoreStageBytes * kScoreStages <= kWarpRingBytes, "the key stream fits the ring slice");
+
 constexpr int kDig1Bits = 11;                   // first radix digit: key bits 31..21
 constexpr int kDig1Bins = 1 << kDig1Bits;       // 2048
 constexpr int kDig2Bits = 11;                   // second digit: bits 20..10
@@ -536,12 +549,16 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
     // zeroed), with the stream's first stages in flight behind the loads
     rotate_queries<T, D, G>(
         a.da, b, g, qhat, u, reinterpret_cast<float *>(hist), true,
-        [&] { LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, slen, a.da.nck, ring))); },
+        [&] {
+          LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
+                            (score_prologue<T, D, L_, kScoreStageBytes, kScoreStages>(rows, t0, slen, a.da.nck, ring)));
+        },
         own ? a.da.k_new + ((size_t)b * a.da.n_kv_heads + g) * D : nullptr, xkh);
     if (own) store_appended<T, D, PAGED>(a.da, rows, b, g, S - 1, xkh);
   } else {
     // q_hat and u from the rotate grid (a programmatic dependency)
-    LOKI_LPT_DISPATCH(a.da.lpt, MAXL, (score_prologue<T, D, L_>(rows, t0, len, a.da.nck, ring)));
+    LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
+                      (score_prologue<T, D, L_, kScoreStageBytes, kScoreStages>(rows, t0, len, a.da.nck, ring)));
     griddep_wait();
     if (tid < D) u[tid] = __ldcg(a.u + (size_t)row * D + tid);
     for (int e = tid; e < G * D; e += kThreads) qhat[e] = __ldcg(a.qhat + (size_t)row * G * D + e);
@@ -551,8 +568,8 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   LOKI_PHASE(1);
   cluster_arrive();  // this CTA's histogram is zero (the leader's receives the others')
   LOKI_LPT_DISPATCH(a.da.lpt, MAXL,
-                    (score_keys_loop<T, D, L_, kWarpStageBytes, kStages, 32 - kDig1Bits>(rows, t0, slen, a.da.nck,
-                                                                                       ring, u, keys, hist)));
+                    (score_keys_loop<T, D, L_, kScoreStageBytes, kScoreStages, 32 - kDig1Bits>(
+                        rows, t0, slen, a.da.nck, ring, u, keys, hist)));
   if (own) {
     // the appended token's key, from its stored (rounded) values
     if (warp == 0) {

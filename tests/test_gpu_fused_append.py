@@ -125,3 +125,64 @@ def test_paged_step_with_append():
         parity.check_append(K[b:b + 1, :, S - 1:S], _widen(kt)[b:b + 1, :, None], su.P.astype(np.float64), "bf16")
         assert np.array_equal(su.logical(su.cache.v)[b, :, S - 1], _widen(vt)[b])
     _check_decode_rows(su, lens, ks, 32, out, idx)
+
+
+def test_generation_run_of_the_pages_shape():
+    """The Llama2-13B-like generation run (batch 16, 40 heads, D 128, bf16):
+    a prompt of 3072 tokens, then 64 consecutive steps, step t appending its
+    token at position 3072 + t inside the call and attending over 3073 + t
+    tokens with k = floor(S / 4), d = 32, on a cache with a 32-dim low-rank
+    plane.  Checked against the oracle: every appended row of the sampled
+    (batch, KV head) rows, and the last step's outputs and selections of those
+    rows (on the cache as the GPU left it); every row's last selection is
+    valid."""
+    from test_gpu_parity import fill_cache_on_device
+    from workloads import get_workload
+    w = get_workload("llama2-13b-generation")
+    T0, steps, d = w.prompt_len, 64, w.d
+    B, Hkv, D = w.batch, w.n_kv_heads, w.head_dim
+    P32 = basis(w)
+    P_dev = torch.from_numpy(P32).to(DEV)
+    cache = fill_cache_on_device(w, P_dev, T0, T0 + steps, d_lr=32)
+    rows = [(0, 0), (7, 21), (15, 39)]
+    pre = {}
+    for (b, g) in rows:  # host-drawn prompts for the rows the oracle checks
+        kt, k64 = gen.to_cache_dtype(gen.row_keys(w, b, g, T0), "bf16")
+        vt, v64 = gen.to_cache_dtype(gen.row_values(w, b, g, T0), "bf16")
+        K_hat = oracle.rotate_keys(k64[None, None], P32[g:g + 1].astype(np.float64), "bf16")
+        cache.k_hat[b, g, :T0] = torch.from_numpy(K_hat[0, 0]).to(torch.bfloat16).to(DEV)
+        cache.v[b, g, :T0] = vt.to(DEV)
+        pre[(b, g)] = v64
+    cache.k_lr[:, :, :T0].copy_(cache.k_hat[:, :, :T0, :32])
+    models = [gen.make_key_model(w, g) for g in range(Hkv)]
+    news = []
+    for t in range(steps):
+        tok = [gen.new_token(w, b, t, models) for b in range(B)]
+        kn = np.stack([x[0] for x in tok])
+        vn = np.stack([x[1] for x in tok])
+        knt, kn64 = gen.to_cache_dtype(kn, "bf16")
+        vnt, vn64 = gen.to_cache_dtype(vn, "bf16")
+        Q = np.stack([gen.queries(w, b, step=t) for b in range(B)])
+        qt, q64 = gen.to_cache_dtype(Q, "bf16")
+        S = T0 + t + 1
+        out, idx = L().loki_decode_attention_append(cache, S, knt.to(DEV), vnt.to(DEV), qt.to(DEV), P_dev, d,
+                                                    S // 4)
+        news.append((kn64, vn64))
+    torch.cuda.synchronize()
+    S = T0 + steps
+    out, idx = out.cpu().numpy(), idx.cpu().numpy()
+    Kall = cache.k_hat[:, :, :S].double().cpu().numpy()
+    Vall = cache.v[:, :, :S].double().cpu().numpy()
+    assert torch.equal(cache.k_lr[:, :, T0:S], cache.k_hat[:, :, T0:S, :32])  # the plane follows every append
+    for (b, g) in rows:
+        kn64 = np.stack([news[t][0][b, g] for t in range(steps)])
+        vn64 = np.stack([news[t][1][b, g] for t in range(steps)])
+        parity.check_append(Kall[b:b + 1, g:g + 1, T0:S], kn64[None, None], P32[g:g + 1].astype(np.float64),
+                            "bf16")
+        assert np.array_equal(Vall[b, g, T0:S], vn64)
+        assert np.array_equal(Vall[b, g, :T0], pre[(b, g)])
+        ref = oracle.loki_decode(q64[b:b + 1, g:g + 1], Kall[b:b + 1, g:g + 1], Vall[b:b + 1, g:g + 1],
+                                 P32[g:g + 1].astype(np.float64), S, d, S // 4)
+        parity.check_decode(out[b:b + 1, g:g + 1], idx[b:b + 1, g:g + 1], ref, ref["q_hat"],
+                            Kall[b:b + 1, g:g + 1], Vall[b:b + 1, g:g + 1], oracle.default_scale(D), "bf16")
+    assert idx.min() >= 0 and idx.max() < S and np.all(np.diff(idx, axis=-1) > 0)

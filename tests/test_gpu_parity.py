@@ -363,20 +363,23 @@ def test_invalid_arguments_raise_without_launch():
 
 
 # ----------------------------------------------------------------------------- full-size workloads
-def fill_cache_on_device(w, P_dev, S, capacity, seed=123, d_lr=0):
+def fill_cache_on_device(w, P_dev, S, capacity, seed=123, d_lr=0, chunk=16384):
     """Whole cache through the GPU append kernel from device-drawn keys (with
-    a low-rank key plane d_lr wide when d_lr > 0)."""
+    a low-rank key plane d_lr wide when d_lr > 0), `chunk` tokens per append
+    so that the keys in flight stay a few GB even for the largest caches."""
     td = TORCH_DTYPE[w.dtype]
     cache = L().LokiCache(w.batch, w.n_kv_heads, w.head_dim, capacity, dtype=td, device=DEV,
                           lowrank_dim=d_lr or None)
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
-    k_new = torch.empty((w.batch, w.n_kv_heads, S, w.head_dim), dtype=td, device=DEV)
-    for h in range(w.n_kv_heads):
-        k_new[:, h] = gen.device_keys(gen.make_key_model(w, h), w.batch, S, g, DEV, td)
-    v_new = torch.randn((w.batch, w.n_kv_heads, S, w.head_dim), generator=g, device=DEV).to(td)
-    L().loki_append(cache, 0, k_new, v_new, P_dev)
-    del k_new, v_new
+    for t0 in range(0, S, chunk):
+        n = min(chunk, S - t0)
+        k_new = torch.empty((w.batch, w.n_kv_heads, n, w.head_dim), dtype=td, device=DEV)
+        for h in range(w.n_kv_heads):
+            k_new[:, h] = gen.device_keys(gen.make_key_model(w, h), w.batch, n, g, DEV, td)
+        v_new = torch.randn((w.batch, w.n_kv_heads, n, w.head_dim), generator=g, device=DEV).to(td)
+        L().loki_append(cache, t0, k_new, v_new, P_dev)
+        del k_new, v_new
     return cache
 
 
@@ -442,9 +445,14 @@ def test_llama2_13b_generation_lengths(S):
 SWEEP_SAMPLE = [
     "mistral-7b-gqa-s4096-b1-d0.25-k0.25",
     "mistral-7b-gqa-s16384-b8-d0.125-k0.5",
+    "mistral-7b-gqa-s16384-b8-d0.5-k0.5",       # the largest d and k together
+    "mistral-7b-gqa-s16384-b32-d0.25-k0.25",    # 256 rows: several waves of clusters
+    "mistral-7b-gqa-s16384-b64-d0.125-k0.125",  # 512 rows
     "mistral-7b-gqa-s65536-b1-d0.5-k0.125",
     "mistral-7b-gqa-s131072-b1-d0.25-k0.25",
     "mistral-7b-gqa-s131072-b8-d0.125-k0.125",
+    "mistral-7b-gqa-s131072-b32-d0.25-k0.125",  # 256 rows of 131072 tokens (17 GB of cache)
+    "mistral-7b-gqa-s131072-b64-d0.125-k0.25",  # 512 rows (34 GB of cache)
 ]
 
 

@@ -176,12 +176,15 @@ constexpr int kRingWords = kWarps * kWarpRingBytes / 4;
 
 __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 
+// Words of the receive buffer of the pushed cluster merge (push_state).
+constexpr int kPushRecvWords = 1088;
+
 // rotation scratch: q staging + partial dot products
 // rotation scratch: G query heads and one appended key, then per-part sums
 __host__ __device__ constexpr int rot_words(int G, int D) { return (G + 1) * D * (1 + kThreads / D); }
 
 struct SmemLayout {
-  int qhat, u, pm, pl, pacc, ctl, slots, ring, keys, words;
+  int qhat, u, pm, pl, pacc, ctl, slots, ring, keys, recv, words;
 };
 
 // Layout in 4-byte words, identical on host and device.  `slots` serves as
@@ -206,6 +209,7 @@ __host__ __device__ inline SmemLayout decode_layout(int G, int D, int chunk, boo
   }
   L.ring = o;  o += kRingWords;
   L.keys = o;  o += ids ? round4(chunk) : 0;
+  L.recv = o;  o += kPushRecvWords;
   L.words = o;
   return L;
 }
@@ -977,6 +981,77 @@ __device__ __forceinline__ void cluster_combine(int ncta, int rank, const float 
   }
 }
 
+// 5'. the same merge by pushing: output elements are owned in blocks of
+//    kThreads (block i by CTA i % ncta); right after its attention each CTA
+//    stores its accumulator for each owner's elements, and its max and sum of
+//    every head, into that owner's receive buffer (`recv`: push_slot_words per
+//    sender, in shared memory the owner no longer uses), so that after one
+//    cluster barrier every owner merges from its own shared memory and no CTA
+//    reads another's afterwards (no second barrier).  Used when the buffers
+//    fit in kPushRecvWords.
+__host__ __device__ inline int push_slot_words(int G, int D, int ncta) {
+  const int blocks = (G * D + kThreads - 1) / kThreads;
+  const int per = (blocks + ncta - 1) / ncta;
+  const int elems = per * kThreads < G * D ? per * kThreads : G * D;
+  return elems + 2 * G;
+}
+__host__ __device__ inline bool push_merge_fits(int G, int D, int ncta) {
+  return ncta > 1 && ncta * push_slot_words(G, D, ncta) <= kPushRecvWords;
+}
+
+// The CTA's state (pm, pl, pacc, final) into the owners' receive buffers.
+template <int D, int G>
+__device__ __forceinline__ void push_state(int ncta, int rank, const float *pm, const float *pl, const float *pacc,
+                                           float *recv) {
+  const int slot = push_slot_words(G, D, ncta);
+  const int elems = slot - 2 * G;
+  const int blocks = (G * D + kThreads - 1) / kThreads;
+  for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    const int bi = e / kThreads;
+    const int local = (bi / ncta) * kThreads + (e - bi * kThreads);
+    dsmem_st(dsmem_addr(recv + rank * slot + local, (uint32_t)(bi % ncta)), __float_as_uint(pacc[e]));
+  }
+  if ((int)threadIdx.x < G) {
+    const int h = threadIdx.x;
+    for (int r = 0; r < ncta && r < blocks; ++r) {
+      dsmem_st(dsmem_addr(recv + rank * slot + elems + h, (uint32_t)r), __float_as_uint(pm[h]));
+      dsmem_st(dsmem_addr(recv + rank * slot + elems + G + h, (uint32_t)r), __float_as_uint(pl[h]));
+    }
+  }
+}
+
+// After the cluster barrier that follows every push_state: this CTA's owned
+// output elements from its receive buffer.
+template <int D, int G>
+__device__ __forceinline__ void push_combine(int ncta, int rank, const float *recv, float *out) {
+  const int slot = push_slot_words(G, D, ncta);
+  const int elems = slot - 2 * G;
+  const int blocks = (G * D + kThreads - 1) / kThreads;
+  for (int bi = rank; bi < blocks; bi += ncta) {
+    const int e = bi * kThreads + (int)threadIdx.x;
+    if (e < G * D) {
+      const int local = (bi / ncta) * kThreads + (int)threadIdx.x;
+      const int h = e / D;
+      float M = -INFINITY;
+      for (int s = 0; s < ncta; ++s) M = fmaxf(M, recv[s * slot + elems + h]);
+      const float mref = (M == -INFINITY) ? 0.f : M;
+      float A = 0.f, Ls = 0.f;
+      for (int s = 0; s < ncta; ++s) {
+        const float c = exp2f(recv[s * slot + elems + h] - mref);
+        A = fmaf(c, recv[s * slot + local], A);
+        Ls = fmaf(c, recv[s * slot + elems + G + h], Ls);
+      }
+      out[e] = A / Ls;
+    }
+  }
+}
+
+// The CTA's own state as the output (clusters of one CTA).
+template <int D, int G>
+__device__ __forceinline__ void local_combine(const float *pl, const float *pacc, float *out) {
+  for (int e = threadIdx.x; e < G * D; e += kThreads) out[e] = pacc[e] / pl[e / D];
+}
+
 template <typename T, int D, int G, bool PAGED>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kernel(const __grid_constant__ DecodeArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
@@ -1011,10 +1086,21 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) dense_decode_kerne
   attend_loop_any<T, D, G, false>(rows, nullptr, t0, slen, qhat, reinterpret_cast<unsigned char *>(scratch), ring,
                                   pm, pl, pacc);
   if (own) fold_token<T, D, G>(qhat, xkh, a.v_new + nv, pm, pl, pacc, scratch);
-  cluster.sync();
   const int Hq = a.n_kv_heads * G;
-  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.out + ((size_t)b * Hq + (size_t)g * G) * D);
-  cluster.sync();
+  float *out = a.out + ((size_t)b * Hq + (size_t)g * G) * D;
+  __syncthreads();  // the CTA's state is complete
+  if (ncta == 1) {
+    local_combine<D, G>(pl, pacc, out);
+  } else if (push_merge_fits(G, D, ncta)) {
+    float *recv = reinterpret_cast<float *>(smem + L.recv);
+    push_state<D, G>(ncta, rank, pm, pl, pacc, recv);
+    cluster.sync();
+    push_combine<D, G>(ncta, rank, recv, out);
+  } else {
+    cluster.sync();
+    cluster_combine<D, G>(ncta, rank, pm, pl, pacc, out);
+    cluster.sync();
+  }
 }
 
 }  // namespace loki

@@ -207,12 +207,16 @@ __host__ __device__ inline FusedSmem fused_smem(int G, int D, int chunk) {
   L.ctl = o;  o += 128;
   L.tbl = o;  o += 2 * kMaxCluster;
   L.hist = o; o += round4(skewed_words(kDig1Bins) > 8 * D ? skewed_words(kDig1Bins) : 8 * D);
+
   L.ring = o; o += kRingWords;
   L.keys = o; o += round4(chunk);
   L.words = o;
   return L;
 }
 
+
+static_assert(skewed_words(kDig1Bins) - 8 * 128 >= kPushRecvWords && skewed_words(kDig1Bins) - 8 * 64 >= kPushRecvWords,
+              "the pushed merge's receive buffer fits in the histogram words above the query tiles");
 
 // select buffers inside the ring (word offsets).  The leader (rank 0) keeps
 // the candidate slots of every CTA and its own refinement histogram; the
@@ -936,12 +940,26 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   }
 
   LOKI_PHASE(5);
-  // 4. log-sum-exp merge of the cluster's states
-  if (gather && !leader) cluster_wait();
-  cluster.sync();
+  // 4. log-sum-exp merge of the cluster's states: pushed into the owners'
+  // receive buffers (above the tensor-core query tiles in the histogram words,
+  // dead since the select) when they fit, else read from every CTA
   const int Hq = a.da.n_kv_heads * G;
-  cluster_combine<D, G>(ncta, rank, pm, pl, pacc, a.da.out + ((size_t)b * Hq + (size_t)g * G) * D);
-  cluster.sync();
+  float *out = a.da.out + ((size_t)b * Hq + (size_t)g * G) * D;
+  __syncthreads();  // the CTA's state is complete
+  const bool push = push_merge_fits(G, D, ncta);
+  float *recv = reinterpret_cast<float *>(hist) + 8 * D;
+  if (push) push_state<D, G>(ncta, rank, pm, pl, pacc, recv);
+  if (gather && !leader) cluster_wait();
+  if (ncta == 1) {
+    local_combine<D, G>(pl, pacc, out);
+  } else if (push) {
+    cluster.sync();
+    push_combine<D, G>(ncta, rank, recv, out);
+  } else {
+    cluster.sync();
+    cluster_combine<D, G>(ncta, rank, pm, pl, pacc, out);
+    cluster.sync();
+  }
   LOKI_PHASE(6);
 #ifdef LOKI_PHASE_STAMPS
   if (tid == 0 && blockIdx.x < kMaxStampCtas) {

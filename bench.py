@@ -13,7 +13,9 @@ steps of its own.  The same run also times a short-row decode
 prompt 3072, then 512 steps that append their token inside the call), Loki
 against dense, and the fp64 oracle on the host (one thread and the BLAS
 pool) with its dense attention beside it.
-L2 is flushed before every step by writing a buffer twice the L2 size; the flush
+L2 is flushed before every step by writing a buffer twice the L2 size and then
+reading another of that size (a write alone left part of a small workload's
+inputs in L2, and its dirty lines cost the next kernel write-backs); the flush
 is outside the timed events.  Device time from CUDA events on the launching
 stream, summed over the K steps, max over ranks.
 
@@ -117,7 +119,7 @@ def workload_config(w, n_gpus):
             "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
             "seq_len": w.seq_len, "d": w.d, "k": w.k, "d_f": w.d_f, "k_f": w.k_f,
             "cache_dtype": w.dtype, "keys": f"{w.generator} spectrum (alpha {w.alpha})",
-            "l2": "flushed before every timed step (write of 2x L2, outside the timed events)",
+            "l2": "flushed before every timed step (write of 2x L2, then a read of 2x L2, outside the timed events)",
             "launch_queue": f"every {CHUNK} timed steps are enqueued behind a GPU sleep, so the host's "
                             "launch rate stays outside the events (not in e2e)",
             "parallelism": f"weak: batch shard per GPU, {n_gpus} GPU(s), no collective"}
@@ -279,11 +281,10 @@ def time_prefill(L, cache, k_pre, v_pre, P, stream, dev, reps: int = 5):
     """Device time of the bulk append of the prompt (rewriting the same cache
     rows), L2 flushed before each repetition; median over reps."""
     import torch
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(torch, dev)
     ts = []
     for i in range(reps + 2):
-        flush.fill_(float(i))
+        flush(float(i))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         L.loki_append(cache, 0, k_pre, v_pre, P)
@@ -341,6 +342,25 @@ def fill_cache(L, w, cache, P, n_tokens, g_dev, dev, td):
     return k_pre, v_pre
 
 
+class L2Flush:
+    """Evicts the L2 before a timed call: writes a buffer twice the L2 size,
+    then reads another of that size.  On B200 a written buffer alone (even 4x
+    the L2) left part of a small workload's inputs cached, and its dirty lines
+    made the next kernel pay their write-back; the read leaves clean lines of
+    a buffer the timed call never touches."""
+
+    def __init__(self, torch, dev):
+        n = 2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4
+        self.torch = torch
+        self.w = torch.empty(n, dtype=torch.float32, device=dev)
+        self.r = torch.ones(n, dtype=torch.float32, device=dev)
+        self.sink = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def __call__(self, v):
+        self.w.fill_(float(v))
+        self.torch.sum(self.r, 0, True, out=self.sink)
+
+
 def time_calls(torch, stream, flush, calls, steps, warmup):
     """Mean device time (us) of each call in `calls`, each in a loop of its own
     over `steps` steps (call(i) for step i), the L2 flushed before every step
@@ -357,7 +377,7 @@ def time_calls(torch, stream, flush, calls, steps, warmup):
             n = min(CHUNK, steps - done)
             queue_ahead(torch, n)
             for i in range(n):
-                flush.fill_(float(i & 7))
+                flush(float(i & 7))
                 ev[i][0].record(stream)
                 call(done + i)
                 ev[i][1].record(stream)
@@ -405,7 +425,7 @@ def time_decode_workload(L, name, flush, stream, dev, steps, warmup, peak):
         n = min(CHUNK, steps - done)
         queue_ahead(torch, n)
         for i in range(n):
-            flush.fill_(float(i & 7))
+            flush(float(i & 7))
             dense(done + i)
             ev[i][0].record(stream)
             loki(done + i)
@@ -521,7 +541,7 @@ def time_paged(L, w, cache, qs, P, flush, stream, dev, steps: int, warmup: int, 
     for i in range(steps):
         if i % CHUNK == 0:
             queue_ahead(torch, min(CHUNK, steps - i))
-        flush.fill_(float(i & 7))
+        flush(float(i & 7))
         evs[i][0].record(stream)
         L.loki_paged_decode_attention(pcache, seqs, qs[i % len(qs)], P, w.d, w.k, out=out, idx=idx, workspace=ws)
         evs[i][1].record(stream)
@@ -579,8 +599,7 @@ def run_ours(args):
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
     idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
     dout = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(torch, dev)
     torch.cuda.synchronize()
 
     # One Loki step: the one-token append, then the decode.  The dense baseline
@@ -588,7 +607,7 @@ def run_ours(args):
     # decode of the same step instead, for the interleaved figure.
     def step(i, ev=None, with_dense=False):
         j = i % NSET
-        flush.fill_(float(i & 7))
+        flush(float(i & 7))
         if ev is not None:
             ev[0].record(stream)
         L.loki_append(cache, S - 1, kn[j], vn[j], P)
@@ -601,7 +620,7 @@ def run_ours(args):
             L.dense_decode_attention(cache, S, qs[j], P, out=dout)
 
     def dense_step(i, ev):
-        flush.fill_(float(i & 7))
+        flush(float(i & 7))
         ev[0].record(stream)
         L.dense_decode_attention(cache, S, qs[i % NSET], P, out=dout)
         ev[1].record(stream)
@@ -685,7 +704,7 @@ def run_ours(args):
     while done < e2e_steps:
         n = min(CH, e2e_steps - done)
         for i in range(n):
-            flush.fill_(float(i & 7))
+            flush(float(i & 7))
             e2e_ev[i][0].record(stream)
             q_dev.copy_(q_host[(done + i) % NSET], non_blocking=True)
             L.loki_decode_attention(cache, S, q_dev, P, w.d, w.k, out=out, idx=idx)
@@ -709,7 +728,7 @@ def run_ours(args):
     while done < e2e_steps:
         n = min(CH, e2e_steps - done)
         for i in range(n):
-            flush.fill_(float(i & 7))
+            flush(float(i & 7))
             e2e_ev[i][0].record(stream)
             graphs[(done + i) % NSET].replay()
             e2e_ev[i][1].record(stream)
@@ -734,7 +753,7 @@ def run_ours(args):
             n = min(CH, np_steps - done)
             queue_ahead(torch, n)
             for i in range(n):
-                flush.fill_(float(i & 7))
+                flush(float(i & 7))
                 ev[i][0].record(stream)
                 L.loki_decode_attention(c, S, qs[(done + i) % NSET], P, w.d, w.k, out=out, idx=idx)
                 ev[i][1].record(stream)
@@ -760,7 +779,7 @@ def run_ours(args):
         n = min(CH, ex_steps - done)
         queue_ahead(torch, n)
         for i in range(n):
-            flush.fill_(float(i & 7))
+            flush(float(i & 7))
             ex_ev[i][0].record(stream)
             L.loki_decode_attention(cache, S, qs[(done + i) % NSET], P, D, w.k, out=out, idx=idx_exact)
             ex_ev[i][1].record(stream)
@@ -787,7 +806,7 @@ def run_ours(args):
             queue_ahead(torch, n)
             for i in range(n):
                 j = (done + i) % NSET
-                flush.fill_(float(i & 7))
+                flush(float(i & 7))
                 ga_ev[i][0].record(stream)
                 call(j)
                 ga_ev[i][1].record(stream)
@@ -976,12 +995,11 @@ def run_phases(args):
     q = torch.randn((B, Hq, D), generator=g_dev, device=dev).to(td)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
     idx = torch.empty((B, Hkv, w.k), dtype=torch.int32, device=dev)
-    flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4, dtype=torch.float32,
-                        device=dev)
+    flush = L2Flush(torch, dev)
     (us,) = time_calls(torch, stream, flush,
                        [lambda i: L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx)],
                        max(args.steps, 10), max(args.warmup, 3))
-    flush.fill_(3.0)
+    flush(3.0)
     L.loki_decode_attention(cache, S, q, P, w.d, w.k, out=out, idx=idx)
     torch.cuda.synchronize()
     rot, ncta, ctas, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
@@ -1011,8 +1029,7 @@ def run_sweep(args):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(torch, dev)
     peak, _ = peaks()
     pts = [w for w in mistral_sweep_points() if args.sweep_filter in w.name]
     groups = {}
@@ -1021,11 +1038,11 @@ def run_sweep(args):
 
     def timed(fn, reps):
         for _ in range(3):
-            flush.fill_(1.0)
+            flush(1.0)
             fn()
         ts = []
         for i in range(reps):
-            flush.fill_(float(i & 7))
+            flush(float(i & 7))
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()

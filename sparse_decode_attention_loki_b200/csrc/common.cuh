@@ -175,6 +175,11 @@ __device__ __forceinline__ void dsmem_red_add(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void dsmem_st(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ void dsmem_st_v4(uint32_t addr, const uint4 &v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ uint4 dsmem_ld_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -199,6 +204,9 @@ __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -221,6 +229,26 @@ __device__ __forceinline__ uint32_t block_excl_suffix_sum(uint32_t v, uint32_t *
     if (w > warp) higher += wtot[w];
   __syncthreads();
   return higher + (s - v);
+}
+
+// Sum of v over all threads with a smaller threadIdx.x (exclusive prefix sum).
+// wtot: kWarps words of shared memory.  Contains two __syncthreads().
+__device__ __forceinline__ uint32_t block_excl_prefix_sum(uint32_t v, uint32_t *wtot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t s = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t t = __shfl_up_sync(kFull, s, off);
+    if (lane >= off) s += t;
+  }
+  if (lane == 31) wtot[warp] = s;
+  __syncthreads();
+  uint32_t lower = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w < warp) lower += wtot[w];
+  __syncthreads();
+  return lower + (s - v);
 }
 
 // Sum over the CTA; the result is returned to every thread.

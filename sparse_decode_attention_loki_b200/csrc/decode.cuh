@@ -365,7 +365,8 @@ struct ScoreStream {
   }
 
   // keys[token] = score_key(score) for the tokens of stage s, and bin
-  // key >> HSHIFT of the skewed histogram hist (see hskew) += 1 for each.
+  // key >> HSHIFT of the skewed histogram hist (see hskew) += 1 for each
+  // (no histogram when HSHIFT is 32).
   template <int HSHIFT>
   __device__ __forceinline__ static void consume_keys(int len, int nck, int s, const unsigned char *wring,
                                                       const float (&uv)[VEC], uint32_t *keys, uint32_t *hist) {
@@ -380,7 +381,7 @@ struct ScoreStream {
       if (c == 0 && base + t < len) {
         const uint32_t key = score_key(sc);
         keys[base + t] = key;
-        atomicAdd(&hist[hskew((int)(key >> HSHIFT))], 1u);
+        if constexpr (HSHIFT < 32) atomicAdd(&hist[hskew((int)(key >> HSHIFT))], 1u);
       }
     }
   }

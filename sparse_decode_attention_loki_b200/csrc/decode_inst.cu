@@ -5,7 +5,7 @@
 #include <type_traits>
 
 #include "host.h"
-#include "loki_step.cuh"
+#include "short_step.cuh"
 
 #ifndef LOKI_D
 #error "LOKI_D (64 or 128) must be defined"
@@ -87,7 +87,9 @@ loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a,
 
 // ---------------------------------------------------------------------------
 // Loki step: rotate grid (query groups of 8), then the decode grid as its
-// programmatic dependent.  CTAs per row (cluster size) of the decode kernel:
+// programmatic dependent: loki_short_kernel for rows of at most
+// kShortMaxTokens tokens, else loki_decode_kernel.  CTAs per row (cluster
+// size) of the decode kernel:
 // start from the fewest CTAs whose share is at most kTargetChunk tokens (two
 // CTAs then fit on an SM; more only when a share would exceed kMaxChunk), and
 // take the first power of two up to 16 whose grid covers at least 80% of the
@@ -97,7 +99,7 @@ loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a,
 constexpr int kTargetChunk = 8192;
 
 template <typename Kern>
-loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan *p, int forced) {
+loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan *p, int forced, bool short_row) {
   const long long rows = (long long)sh.B * sh.Hkv;
   const int S = sh.S;
   int dev = 0;
@@ -113,35 +115,37 @@ loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan 
     if (forced ? n != forced : n < need) continue;
     const int chunk = round4((S + n - 1) / n);
     if (chunk > kMaxChunk) continue;
-    const int smem = fused_smem(sh.G, sh.D, chunk).words * 4;
+    const int smem = (short_row ? short_smem(sh.G, sh.D, chunk, n, sh.S).words : fused_smem(sh.G, sh.D, chunk).words) * 4;
     if (smem > di.smem_optin) continue;
     const int mc = max_active(kern, dev, n, smem, di.smem_optin);
     if (mc <= 0) continue;
     best = Plan{n, chunk, smem, (int)(rows * n), sh.G > 4 ? (int)(rows * (sh.D / kRotCols)) : 0, 0};
     if (forced || rows * 5 >= 4LL * mc) break;  // covers 80% of a wave
   }
-  if (best.ncta == 0 && forced) return plan_step(kern, di, sh, p, 0);  // a forced size that cannot run
+  if (best.ncta == 0 && forced) return plan_step(kern, di, sh, p, 0, short_row);  // a forced size that cannot run
   if (best.ncta == 0)
     return fail(LOKI_ERR_UNSUPPORTED, "seq_len %d: no schedulable cluster fits the keys in shared memory", S);
   *p = best;
   return LOKI_OK;
 }
 
-template <typename T, int D, int G, bool PAGED>
+template <typename T, int D, int G, bool PAGED, bool SHORT>
 struct StepGate {
   static SmemGate gate;
 };
-template <typename T, int D, int G, bool PAGED>
-SmemGate StepGate<T, D, G, PAGED>::gate;
+template <typename T, int D, int G, bool PAGED, bool SHORT>
+SmemGate StepGate<T, D, G, PAGED, SHORT>::gate;
 
 template <typename T, int D, int G, bool PAGED>
 loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da, void *ws, void *stream,
                      Plan *used) {
-  auto kern = loki_decode_kernel<T, D, G, PAGED>;
-  loki_status s = allow_smem(kern, di, StepGate<T, D, G, PAGED>::gate, true);
+  const bool short_row = sh.S <= kShortMaxTokens;
+  auto kern = short_row ? loki_short_kernel<T, D, G, PAGED> : loki_decode_kernel<T, D, G, PAGED>;
+  loki_status s = allow_smem(kern, di, short_row ? StepGate<T, D, G, PAGED, true>::gate
+                                                 : StepGate<T, D, G, PAGED, false>::gate, true);
   if (s != LOKI_OK) return s;
   Plan pl;
-  s = plan_step(kern, di, sh, &pl, forced_cluster());
+  s = plan_step(kern, di, sh, &pl, forced_cluster(), short_row);
   if (s != LOKI_OK) return s;
   if (used) {  // shape query only: launch nothing
     *used = pl;

@@ -80,6 +80,14 @@ def source_hash() -> str:
     return h.hexdigest()[:12]
 
 
+def decode_kernel_name(rot: int, short_kernel: int) -> str:
+    """The kernel(s) of a Loki step, from loki_decode_launch_shape."""
+    k = "loki_short_kernel" if short_kernel else "loki_decode_kernel"
+    if rot == 0:
+        return f"{k} (rotates its own queries)"
+    return f"loki_rotate_kernel + {k} (programmatic dependent pair)"
+
+
 def measured_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source; else None."""
@@ -435,9 +443,11 @@ def time_decode_workload(L, name, flush, stream, dev, steps, warmup, peak):
             tot += ev[i][0].elapsed_time(ev[i][1])
         done += n
     lb, db = w.loki_bytes(), w.dense_bytes()
+    rot, ncta, ctas, short_kernel = L.loki_decode_launch_shape(cache, S, Hq, w.k)
     del cache
     torch.cuda.empty_cache()
     return {"workload": name, "loki_us": loki_us, "dense_us": dense_us,
+            "launch": {"kernel": decode_kernel_name(rot, short_kernel), "cluster_ctas": ncta, "ctas": ctas},
             "loki_frac": lb / (loki_us * 1e-6) / 1e9 / peak, "dense_frac": db / (dense_us * 1e-6) / 1e9 / peak,
             "speedup_vs_dense": dense_us / loki_us, "byte_ratio": db / lb,
             "loki_after_dense_us": tot * 1000.0 / steps, "steps": steps,
@@ -828,7 +838,7 @@ def run_ours(args):
         L.loki_decode_attention(cache, S, qs[j], P, D, w.k, out=out, idx=idx_exact)
         jac.append(L.topk_jaccard(idx, idx_exact))
     jaccard = torch.stack(jac)
-    rot, ncl, nct, _ = L.loki_decode_launch_shape(cache, S, Hq, w.k)
+    rot, ncl, nct, short_kernel = L.loki_decode_launch_shape(cache, S, Hq, w.k)
     _, dcl, dct, _ = L.loki_decode_launch_shape(cache, S, Hq, dense=True)
     # ---------------- the short-row decode and the pages' generation run, same session
     extras = {}
@@ -869,8 +879,7 @@ def run_ours(args):
             "hbm_gbs": ach,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                          "traffic": measured_traffic("loki_decode_step", w.name),
-                         "kernel": ("loki_decode_kernel (rotates its own queries)" if rot == 0 else
-                                    "loki_rotate_kernel + loki_decode_kernel (programmatic dependent pair)"),
+                         "kernel": decode_kernel_name(rot, short_kernel),
                          "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
                          "algorithmic_bytes_per_launch": lb},
             "dense": {"us": dense_us, "hbm_gbs": dach, "frac": dach / peak, "bytes_per_launch": db,
@@ -898,7 +907,8 @@ def run_ours(args):
             "exact_topk": {"us": t_exact * 1000.0 / ex_steps, "d": D, "k": w.k, "steps": ex_steps,
                            "jaccard_vs_loki": {"mean": float(jaccard.mean()), "min": float(jaccard.min()),
                                                "rows": int(jaccard.numel())}},
-            "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256},
+            "launch": {"rotate_ctas": rot, "decode_cluster_ctas": ncl, "decode_ctas": nct, "threads_per_cta": 256,
+                       "decode_kernel": decode_kernel_name(rot, short_kernel)},
             "e2e": {"value": e2e_us / world, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps,
                     "path": "DecodeGraph.replay(): query copied in from pinned host memory, the decode, out "

@@ -119,7 +119,7 @@ loki_status plan_step(Kern kern, const DevInfo &di, const DecodeShape &sh, Plan 
     if (smem > di.smem_optin) continue;
     const int mc = max_active(kern, dev, n, smem, di.smem_optin);
     if (mc <= 0) continue;
-    best = Plan{n, chunk, smem, (int)(rows * n), sh.G > 4 ? (int)(rows * (sh.D / kRotCols)) : 0, 0};
+    best = Plan{n, chunk, smem, (int)(rows * n), sh.G > 4 ? (int)(rows * (sh.D / kRotCols)) : 0, short_row ? 1 : 0};
     if (forced || rows * 5 >= 4LL * mc) break;  // covers 80% of a wave
   }
   if (best.ncta == 0 && forced) return plan_step(kern, di, sh, p, 0, short_row);  // a forced size that cannot run

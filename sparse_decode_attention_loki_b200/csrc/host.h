@@ -43,7 +43,7 @@ struct Plan {
   int smem;    // dynamic shared memory per CTA
   int grid;    // CTAs of the decode kernel
   int rot;     // Loki: CTAs of the rotate kernel (query groups of 8), else 0
-  int spare;
+  int spare;   // Loki: 1 when the short-row kernel runs, else 0
 };
 
 // Per-sequence lengths and paging of a decode call (all null: a contiguous
@@ -157,8 +157,8 @@ loki_status append_token(int dtype, int D, void *k_hat, void *v, void *k_lr, int
                          int B, const void *k_new, const void *v_new, const float *P, void *stream);
 
 // The decode calls of one (dtype, head dim), compiled in decode_inst.cu once
-// per pair: dense == true runs the dense kernel, else the Loki work queue
-// (ws: the caller's workspace).  used != nullptr: plan only, launch nothing.
+// per pair: dense == true runs the dense kernel, else the Loki step (ws:
+// the caller's workspace).  used != nullptr: plan only, launch nothing.
 template <typename T, int D>
 loki_status decode_td(bool dense, const DevInfo &di, const DecodeShape &sh, const DecodeArgs<T> &a, void *ws,
                       void *stream, Plan *used);

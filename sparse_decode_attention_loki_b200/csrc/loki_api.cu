@@ -636,7 +636,7 @@ loki_status loki_decode_launch_shape(const loki_cache *cache, int32_t seq_len, i
   shape[0] = dense ? 0 : pl.rot;
   shape[1] = pl.ncta;
   shape[2] = (int32_t)(rows * pl.ncta);
-  shape[3] = 0;
+  shape[3] = dense ? 0 : pl.spare;
   return LOKI_OK;
 }
 

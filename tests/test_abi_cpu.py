@@ -55,7 +55,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.loki_version() == 12
+    assert lib.loki_version() == 13
     for s, word in [(0, b"LOKI_OK"), (1, b"INVALID_ARG"), (2, b"UNSUPPORTED"), (3, b"CUDA")]:
         assert word in lib.loki_status_string(s)
     assert lib.loki_status_string(99) == b"unknown loki_status"

@@ -272,9 +272,10 @@ def test_cluster_shapes_and_ragged_chunks(S, B, Hkv, G):
     # rows split over clusters of several CTAs with a ragged last chunk, grids
     # of several waves, and a row longer than one CTA can hold
     w = small_workload("bf16", 128, G, S, Hkv=Hkv, B=B, seed=S)
-    rot, ncta, ctas, zero = L().loki_decode_launch_shape(
+    rot, ncta, ctas, short_kernel = L().loki_decode_launch_shape(
         L().LokiCache(B, Hkv, 128, S, dtype=torch.bfloat16, device=DEV), S, Hkv * G, max(1, S // 8))
-    assert rot == (B * Hkv * 4 if G == 8 else 0) and ctas == B * Hkv * ncta and zero == 0
+    assert rot == (B * Hkv * 4 if G == 8 else 0) and ctas == B * Hkv * ncta
+    assert short_kernel == (1 if S <= 8192 else 0)
     assert ncta in (1, 2, 4, 8, 16) and ncta * 24576 >= S
     out, idx, ref, K_hat, V, *_ = run_decode(w, S, 32, max(1, S // 8))
     parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(128), "bf16")

@@ -2,7 +2,9 @@
 // Attention", atlas.scime.ai summary, section "Approach": PCA-project
 // queries and keys, rank tokens on the top-d principal dimensions, exact
 // attention over the top-k tokens), one kernel for query groups of up to 4
-// heads, two for 8:
+// heads, two for 8.  This file holds the rotate kernel and the decode kernel
+// of rows longer than kShortMaxTokens; short_step.cuh holds the short-row
+// decode kernel, which reuses the pieces here.
 //
 //   rotate  (groups of 8 only) D/32 CTAs per (batch, KV head) row: q_hat_h =
 //           q_h . P_g for the G query heads of the row (fp32, pre-scaled for
@@ -17,8 +19,8 @@
 //        shared memory and histograms the keys' top 11 bits on the way;
 //     2. cluster radix select over 11/11/10-bit digits: every CTA adds the
 //        non-zero bins of its histogram into the leader CTA's (distributed
-//        shared memory reductions).  A short row (S + k within the leader's
-//        ring) is then selected by the leader alone on all its keys, read
+//        shared memory reductions).  A row with S + k within the leader's
+//        ring is then selected by the leader alone on all its keys, read
 //        from the cluster's shared memory, into an ascending list of k
 //        indices.  On a longer row the leader finds the bucket of the k-th
 //        largest key and tells every CTA; each CTA sends the leader its keys
@@ -600,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_decode_kernel
   const bool gather = S + (int)k <= kGatherWords;    // uniform over the cluster
   cluster_wait();  // every CTA, the leader in particular, zeroed its histogram before its stream
   if (gather) {
-    // a short row: the leader collects the histogram, then reads every CTA's
+    // S + k within the leader's ring: the leader collects the histogram, then reads every CTA's
     // keys (distributed shared memory; CTA r holds tokens [r*chunk, ..),
     // chunk a multiple of 4) into its ring and selects alone
     if (!leader) push_skewed(hist, kDig1Bins, dsmem_addr(hist, 0u));

@@ -383,9 +383,10 @@ LOKI_API loki_status loki_pca_calibrate(const void *keys, int32_t dtype, int32_t
  *     queries, query groups of up to 4 heads), shape[1] CTAs per (batch, KV
  *     head) row in one cluster of the decode kernel, shape[2] CTAs of the
  *     decode kernel, shape[3] = 1 when the decode kernel is the short-row
- *     one (every row of at most 8192 tokens: each CTA of a cluster selects
- *     on the whole row's keys) and 0 for the long-row one (cluster select
- *     through a leader CTA).
+ *     one (each CTA of a cluster selects on the whole row's keys: rows of at
+ *     most 8192 tokens whose keys leave it as many CTAs per SM as the
+ *     long-row kernel) and 0 for the long-row one (cluster select through a
+ *     leader CTA).
  *   dense != 0 (dense_decode_attention): shape[1] CTAs per row in one
  *     cluster, shape[2] CTAs in all, shape[0] = shape[3] = 0.
  * k is checked (1 <= k <= seq_len) for dense == 0 but does not change the

@@ -453,7 +453,8 @@ def loki_decode_launch_shape(cache: LokiCache, seq_len: int, n_q_heads: int, k: 
                              dense: bool = False) -> Tuple[int, int, int, int]:
     """Grid sizes of a decode call.  Loki: (rotation CTAs, decode CTAs per row
     in one cluster, decode CTAs, 1 for the short-row kernel (rows of at most
-    8192 tokens) else 0).  Dense: (0, CTAs per row in one cluster, CTAs, 0)."""
+    8192 tokens, where it fits as many CTAs per SM as the long-row kernel)
+    else 0).  Dense: (0, CTAs per row in one cluster, CTAs, 0)."""
     shape = (ctypes.c_int32 * 4)()
     with torch.cuda.device(cache.device):
         _lib.check(_lib.load().loki_decode_launch_shape(cache.desc(), int(seq_len), int(n_q_heads), int(k),

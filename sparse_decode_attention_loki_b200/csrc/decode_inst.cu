@@ -88,7 +88,8 @@ loki_status run_dense(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> a,
 // ---------------------------------------------------------------------------
 // Loki step: rotate grid (query groups of 8), then the decode grid as its
 // programmatic dependent: loki_short_kernel for rows of at most
-// kShortMaxTokens tokens, else loki_decode_kernel.  CTAs per row (cluster
+// kShortMaxTokens tokens when it keeps as many CTAs per SM as the long-row
+// kernel, else loki_decode_kernel.  CTAs per row (cluster
 // size) of the decode kernel:
 // start from the fewest CTAs whose share is at most kTargetChunk tokens (two
 // CTAs then fit on an SM; more only when a share would exceed kMaxChunk), and
@@ -139,14 +140,31 @@ SmemGate StepGate<T, D, G, PAGED, SHORT>::gate;
 template <typename T, int D, int G, bool PAGED>
 loki_status run_step(const DevInfo &di, const DecodeShape &sh, DecodeArgs<T> da, void *ws, void *stream,
                      Plan *used) {
-  const bool short_row = sh.S <= kShortMaxTokens;
-  auto kern = short_row ? loki_short_kernel<T, D, G, PAGED> : loki_decode_kernel<T, D, G, PAGED>;
-  loki_status s = allow_smem(kern, di, short_row ? StepGate<T, D, G, PAGED, true>::gate
-                                                 : StepGate<T, D, G, PAGED, false>::gate, true);
+  auto kshort = loki_short_kernel<T, D, G, PAGED>;
+  auto klong = loki_decode_kernel<T, D, G, PAGED>;
+  loki_status s = allow_smem(klong, di, StepGate<T, D, G, PAGED, false>::gate, true);
   if (s != LOKI_OK) return s;
   Plan pl;
-  s = plan_step(kern, di, sh, &pl, forced_cluster(), short_row);
-  if (s != LOKI_OK) return s;
+  bool short_row = sh.S <= kShortMaxTokens;
+  if (short_row) {
+    // the short-row kernel holds the whole row's keys in every CTA: it runs
+    // only where that leaves as many CTAs per SM as the long-row kernel has
+    // with the same cluster shape (measured: fewer loses to the long kernel)
+    s = allow_smem(kshort, di, StepGate<T, D, G, PAGED, true>::gate, true);
+    if (s != LOKI_OK) return s;
+    s = plan_step(kshort, di, sh, &pl, forced_cluster(), true);
+    if (s != LOKI_OK) return s;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int occ_short = max_active(kshort, dev, 0, pl.smem, di.smem_optin);
+    const int occ_long = max_active(klong, dev, 0, fused_smem(sh.G, sh.D, pl.chunk).words * 4, di.smem_optin);
+    short_row = occ_short >= occ_long;
+  }
+  if (!short_row) {
+    s = plan_step(klong, di, sh, &pl, forced_cluster(), false);
+    if (s != LOKI_OK) return s;
+  }
+  auto kern = short_row ? kshort : klong;
   if (used) {  // shape query only: launch nothing
     *used = pl;
     return LOKI_OK;

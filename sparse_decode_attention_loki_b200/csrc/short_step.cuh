@@ -139,6 +139,19 @@ __device__ __forceinline__ void short_hist_pass(const uint32_t *all, int S, uint
   }
 }
 
+// The select's two block-wide steps as single out-of-line copies: each runs
+// two or three times per call, and a second call then executes from the
+// instruction cache instead of fetching another inlined copy from memory
+// (measured: llama2-7b-decode 27.3 -> 26.6 us).
+static __device__ __noinline__ void short_find_bucket(const uint32_t *hist, int nb, uint32_t remaining,
+                                                      uint32_t *ctl) {
+  find_bucket(hist, nb, remaining, ctl);
+}
+static __device__ __noinline__ void short_hist(const uint32_t *all, int S, uint32_t prefix, uint32_t mask, int shift,
+                                               int nb, uint32_t *hist) {
+  short_hist_pass(all, S, prefix, mask, shift, nb, hist);
+}
+
 template <typename T, int D, int G, bool PAGED>
 __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_short_kernel(const __grid_constant__ StepArgs<T> a) {
   extern __shared__ __align__(16) uint32_t smem[];
@@ -230,9 +243,9 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_short_kernel(
 
   // 3. the select, the same in every CTA: the first digit's bucket of the
   // k-th largest key, then up to two refinement passes over the keys in it
-  short_hist_pass(all, S, 0u, 0u, 32 - kDig1Bits, kDig1Bins, href);
+  short_hist(all, S, 0u, 0u, 32 - kDig1Bits, kDig1Bins, href);
   __syncthreads();
-  find_bucket(href, kDig1Bins, k, ctl);
+  short_find_bucket(href, kDig1Bins, k, ctl);
   uint32_t rem = k - ctl[kSelBucket + 1], inb = ctl[kSelBucket + 2];
   uint32_t pre = ctl[kSelBucket + 0] << (32 - kDig1Bits), msk = ~0u << (32 - kDig1Bits);
 #pragma unroll 1
@@ -243,9 +256,9 @@ __global__ void __launch_bounds__(kThreads, (G >= 8) ? 1 : 2) loki_short_kernel(
     // closing barrier
     for (int e = tid; e < skewed_words(nb); e += kThreads) href[e] = 0u;
     __syncthreads();
-    short_hist_pass(all, S, pre, msk, shift, nb, href);
+    short_hist(all, S, pre, msk, shift, nb, href);
     __syncthreads();
-    find_bucket(href, nb, rem, ctl);
+    short_find_bucket(href, nb, rem, ctl);
     rem -= ctl[kSelBucket + 1];
     inb = ctl[kSelBucket + 2];
     pre |= ctl[kSelBucket + 0] << shift;

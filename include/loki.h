@@ -412,10 +412,12 @@ LOKI_API loki_status loki_set_launch_override(int32_t per_row);
  * (CTA c of the decode kernel, up to 65536 CTAs) holds the device global timer
  * in ns when the CTA started, when its queries were ready and its first key
  * stages in flight, when its key stream was done, when the first digit of
- * the selection was known, when its share of the selected rows was known,
- * when its attention was done and when the cluster's merge was done; then
- * its SM, then its rank in the cluster | cluster size << 8 | (1 << 16 when
- * the row took the single-CTA select), then its (batch, KV head) row.
+ * the selection was known (short-row kernel: when every key of the row had
+ * arrived), when its share of the selected rows was known, when its
+ * attention was done and when the cluster's merge was done; then its SM,
+ * then its rank in the cluster | cluster size << 8 | (1 << 16 when the row
+ * took a single-CTA select) | (1 << 17 for the short-row kernel), then its
+ * (batch, KV head) row.
  * Entries of CTAs the last decode did not have hold older data.  *n receives
  * the number of entries copied.  Synchronous.  Not part of the method. */
 LOKI_API loki_status loki_phase_stamps(int32_t dtype, int32_t head_dim, uint64_t *host, int32_t capacity,

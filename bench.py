@@ -1021,6 +1021,7 @@ def run_phases(args):
     line = {"phases": w.name, "decode_us_stamped_build": us,
             "launch": {"rotate_ctas": rot, "cluster_ctas": ncta, "ctas": ctas},
             "single_cta_select": bool(int(buf[0, 8]) >> 16 & 1),
+            "short_row_kernel": bool(int(buf[0, 8]) >> 17 & 1),
             "algorithmic_bytes": w.loki_bytes(), **summ}
     print(json.dumps(line))
     return 0

@@ -281,6 +281,20 @@ def test_cluster_shapes_and_ragged_chunks(S, B, Hkv, G):
     parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(128), "bf16")
 
 
+@pytest.mark.parametrize("S,B,Hkv,G", [(6144, 1, 8, 4), (5120, 4, 8, 4), (4608, 2, 2, 8), (8192, 1, 4, 1)])
+def test_rows_between_4096_and_8192_tokens(S, B, Hkv, G):
+    # the short-row kernel takes these only where its shared memory (the whole
+    # row's keys in every CTA) keeps the long-row kernel's CTAs per SM, so both
+    # kernels serve rows of this length; either way the selection and the
+    # attention must match the oracle
+    w = small_workload("bf16", 128, G, S, Hkv=Hkv, B=B, seed=S + G)
+    rot, ncta, ctas, short_kernel = L().loki_decode_launch_shape(
+        L().LokiCache(B, Hkv, 128, S, dtype=torch.bfloat16, device=DEV), S, Hkv * G, S // 4)
+    assert short_kernel in (0, 1) and ctas == B * Hkv * ncta
+    out, idx, ref, K_hat, V, *_ = run_decode(w, S, 32, S // 4)
+    parity.check_decode(out, idx, ref, ref["q_hat"], K_hat, V, oracle.default_scale(128), "bf16")
+
+
 def test_repeated_calls_are_identical():
     w = small_workload("bf16", 128, 4, 3001)
     out, idx, ref, K_hat, V, inp, P32, cache, q, P = run_decode(w, 3001, 64, 375)
